@@ -1,0 +1,70 @@
+"""QLoRA linear layer forward and backward in fp64 (oracle -- test
+infrastructure only).
+
+Shapes follow the PyTorch Linear convention: x [M, in], W0 [out, in],
+A [r, in], B [out, r], h [M, out]; s = alpha / r.
+
+Forward ("QLoRA", llm-compass, 方法与公式, the displayed formula):
+    h = dequant(W0) x + (alpha/r) B A x
+written for row-major token batches as
+    h = x W^T + s (x A^T) B^T,            W = dequant(W0)
+
+Backward: the base is frozen and only the adapters are trained, while the
+gradient still flows through the quantized base to the layer input
+("QLoRA", aigrafen.se, opening paragraph; llm-compass, 方法与公式, the
+sentence after the formula).  With dh = dL/dh:
+    dx = dh W + s (dh B) A
+    dB = s dh^T (x A^T)
+    dA = s (dh B)^T x
+dequant(W0) is treated as a constant: there is no gradient for the codes.
+
+Everything is computed in fp64 on the bf16 inputs' exact values and on the
+oracle's own dequantized weight; no intermediate rounding is applied.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def linear_fwd(x, W, A, B, alpha: float):
+    """h = x W^T + s (x A^T) B^T in fp64; also returns u = x A^T (pre-scale)."""
+    x, W, A, B = _f64(x), _f64(W), _f64(A), _f64(B)
+    r = A.shape[0]
+    s = float(alpha) / float(r)
+    u = x @ A.T                       # [M, r]
+    h = x @ W.T + s * (u @ B.T)       # [M, out]
+    return h, u
+
+
+def linear_bwd(dh, x, W, A, B, alpha: float):
+    """(dx, dA, dB) of L = sum(dh * h) for the forward above, in fp64."""
+    dh, x, W, A, B = _f64(dh), _f64(x), _f64(W), _f64(A), _f64(B)
+    r = A.shape[0]
+    s = float(alpha) / float(r)
+    g = dh @ B                        # [M, r]
+    u = x @ A.T                       # [M, r]
+    dx = dh @ W + s * (g @ A)         # [M, in]
+    dB = s * (dh.T @ u)               # [out, r]
+    dA = s * (g.T @ x)                # [r, in]
+    return dx, dA, dB
+
+
+def linear_fwd_rows(x, W, A, B, alpha: float, rows):
+    """Forward restricted to the token rows ``rows`` (for sampled checks of
+    full-size outputs); identical arithmetic to :func:`linear_fwd`."""
+    rows = np.asarray(rows)
+    h, _ = linear_fwd(_f64(x)[rows], W, A, B, alpha)
+    return h
+
+
+def linear_dx_rows(dh, W, A, B, alpha: float, rows):
+    """dx restricted to the token rows ``rows``; same arithmetic as
+    :func:`linear_bwd`."""
+    dh, W, A, B = _f64(dh)[np.asarray(rows)], _f64(W), _f64(A), _f64(B)
+    s = float(alpha) / float(A.shape[0])
+    return dh @ W + s * ((dh @ B) @ A)

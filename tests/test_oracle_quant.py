@@ -1,0 +1,232 @@
+"""Pins for the oracle's blockwise quantizer, double quantization and
+dequantization (CPU only): brute force in exact rational arithmetic, exact
+round trips, error bounds, zero handling and the storage arithmetic the pages
+print."""
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import nf4, overhead
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def brute_nearest(v: float, levels) -> int:
+    """argmin_j |v - q_j| in exact rational arithmetic, ties to the lower j."""
+    fv = Fraction(float(v))
+    best, best_d = 0, None
+    for j, q in enumerate(levels):
+        d = abs(fv - Fraction(float(q)))
+        if best_d is None or d < best_d:
+            best, best_d = j, d
+    return best
+
+
+def test_nearest_level_matches_brute_force_on_all_fp16_values():
+    levels = nf4.codebook()
+    h = np.arange(0, 1 << 16, dtype=np.uint16).view(np.float16).astype(np.float64)
+    h = h[np.isfinite(h) & (np.abs(h) <= 1.1)]
+    got = nf4.nearest_level(h)
+    # brute force on a deterministic subsample plus every value within 1e-3
+    # of a midpoint (where a wrong tie rule or threshold would show)
+    mids = nf4.midpoints()
+    near = np.min(np.abs(h[:, None] - mids[None, :]), axis=1) < 1e-3
+    idx = np.unique(np.concatenate([np.nonzero(near)[0], np.arange(0, h.size, 37)]))
+    for i in idx:
+        assert got[i] == brute_nearest(h[i], levels), h[i]
+
+
+def test_nearest_level_ties_go_to_lower_index():
+    levels = nf4.codebook()
+    for j, m in enumerate(nf4.midpoints()):
+        if float(np.float32(m)) == m:            # representable midpoint: a true tie
+            assert nf4.nearest_level(np.array([m]))[0] == j
+            assert brute_nearest(m, levels) == j
+
+
+def test_encode_matches_brute_force_on_tiny_blocks():
+    rng = np.random.default_rng(5)
+    W = (rng.standard_normal((2, 128)) * 0.02).astype(np.float32)
+    W[1, 64:] = (rng.standard_t(3, 64) * 0.05).astype(np.float32)
+    c = nf4.block_absmax(W)
+    codes = nf4.encode(W, c)
+    levels = nf4.codebook()
+    for b in range(4):
+        row, col0 = divmod(b * 64, 128)
+        cb = np.float32(np.abs(W[row, col0:col0 + 64]).max())
+        assert float(cb) == c[b]
+        r = np.float32(1.0) / cb                      # fp32 reciprocal
+        for k in range(64):
+            v = np.float32(W[row, col0 + k]) * r      # fp32 product
+            assert codes[row, col0 + k] == brute_nearest(float(v), levels)
+
+
+def test_exact_levels_round_trip():
+    levels = nf4.codebook()
+    for c in [1.0, 0.0371, 3.5e-3, 17.25]:
+        w = np.float32(c) * levels.astype(np.float32)     # includes +-c (levels 0, 15)
+        W = np.tile(w, 4).reshape(1, 64)
+        q = nf4.quantize(W)
+        assert q["absmax"][0] == np.float32(c)
+        assert np.array_equal(q["codes"][0], np.tile(np.arange(16), 4))
+
+
+def test_first_level_round_trip_bound():
+    """|w - q[code] * c| <= c * G/2 with G the largest codebook gap."""
+    rng = np.random.default_rng(11)
+    W = np.concatenate([rng.standard_normal((64, 256)) * 0.02,
+                        rng.standard_t(5, (64, 256)) * 0.02]).astype(np.float32)
+    q = nf4.quantize(W)
+    levels = nf4.codebook()
+    c = q["absmax"].repeat(64).reshape(W.shape)
+    recon = levels[q["codes"]] * c
+    G2 = np.diff(levels).max() / 2
+    err = np.abs(W.astype(np.float64) - recon)
+    # reciprocal normalisation moves v by at most a couple of fp32 ulps
+    assert np.all(err <= c * (G2 + 1e-6))
+    # and the bound is attained closely somewhere (it is not vacuous)
+    assert (err / c).max() > 0.9 * G2
+
+
+def test_dequantized_round_trip_bound_with_double_quant():
+    rng = np.random.default_rng(12)
+    W = (rng.standard_normal((128, 512)) * 0.02).astype(np.float32)
+    q = nf4.quantize(W)
+    c = q["absmax"]
+    c_hat = nf4.dequant_scales(q["q8"], q["step2"], q["mean"])
+    g = np.arange(c.size) // 256
+    # second-level error: half a step plus fp32 rounding
+    assert np.all(np.abs(c - c_hat) <= q["step2"][g] * 0.5 + 4 * np.spacing(np.float32(c.max())))
+    w_hat = nf4.dequantize(q["codes"], q["q8"], q["step2"], q["mean"])
+    G2 = np.diff(nf4.codebook()).max() / 2
+    cb = c.repeat(64).reshape(W.shape)
+    dc = np.abs(c - c_hat).repeat(64).reshape(W.shape)
+    bound = cb * (G2 + 1e-6) + dc + np.abs(w_hat) * 2.0 ** -8 + 1e-30
+    assert np.all(np.abs(W - w_hat) <= bound)
+
+
+def test_zero_blocks_and_negative_zero():
+    W = np.zeros((2, 128), dtype=np.float32)
+    W[0, 64:] = np.linspace(-0.03, 0.05, 64, dtype=np.float32)
+    W[1, :64] = np.float32(-0.0)
+    q = nf4.quantize(W)
+    assert np.all(q["codes"][0, :64] == 7)
+    assert np.all(q["codes"][1] == 7)
+    w_hat = nf4.dequantize(q["codes"], q["q8"], q["step2"], q["mean"])
+    assert np.all(w_hat[0, :64] == 0.0) and np.all(w_hat[1] == 0.0)
+    # -0.0 inside a nonzero block also maps to the zero level
+    W2 = np.linspace(-1, 1, 64, dtype=np.float32).reshape(1, 64)
+    W2[0, 10] = np.float32(-0.0)
+    assert nf4.quantize(W2)["codes"][0, 10] == 7
+
+
+def test_equal_absmax_blocks_give_zero_second_level_codes():
+    # every block has absmax exactly 0.5 -> c - mean = 0 -> step 0 -> q8 = 0,
+    # and the dequantized scale is exactly the mean
+    rng = np.random.default_rng(3)
+    W = (rng.uniform(-0.5, 0.5, (8, 256))).astype(np.float32)
+    W[:, ::64] = 0.5
+    q = nf4.quantize(W)
+    assert q["mean"] == 0.5
+    assert np.all(q["q8"] == 0) and np.all(q["step2"] == 0)
+    assert np.all(nf4.dequant_scales(q["q8"], q["step2"], q["mean"]) == 0.5)
+
+
+def test_second_level_codes_use_full_int8_range():
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((64, 1024)) * 0.02).astype(np.float32)   # 1024 blocks = 4 groups
+    q = nf4.quantize(W)
+    assert q["q8"].min() >= -127 and q["q8"].max() <= 127
+    for g in range(4):
+        assert np.abs(q["q8"][g * 256:(g + 1) * 256]).max() == 127
+    assert q["step2"].shape == (4,)
+
+
+def test_partial_last_group():
+    rng = np.random.default_rng(6)
+    W = (rng.standard_normal((5, 64 * 61)) * 0.02).astype(np.float32)  # 305 blocks
+    q = nf4.quantize(W)
+    assert q["step2"].shape == (2,) and q["q8"].shape == (305,)
+    d_last = nf4.fl32(q["absmax"][256:] - q["mean"])
+    assert q["step2"][1] == nf4.fl32(np.abs(d_last).max() / 127.0)
+
+
+def test_pairwise_tree_fixtures():
+    with open(os.path.join(GOLDEN, "pairwise_tree.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            want, vals = line.split(";")
+            vals = [float(v) for v in vals.split()]
+            assert nf4.pairwise_sum(np.array(vals)) == float(want), line
+
+
+def test_pairwise_sum_accuracy_bound():
+    rng = np.random.default_rng(7)
+    v = rng.uniform(0, 0.1, 100003)
+    import math
+    exact = math.fsum(v)
+    # pairwise summation error <= ceil(log2 n) * eps * sum|v|
+    assert abs(nf4.pairwise_sum(v) - exact) <= 17 * 2.0 ** -53 * exact
+
+
+def test_pack_unpack_nibble_order():
+    codes = np.arange(32, dtype=np.uint8).reshape(1, 32) % 16
+    p = nf4.pack(codes)
+    assert p[0, 0] == (0 | (1 << 4)) and p[0, 1] == (2 | (3 << 4))
+    assert np.array_equal(nf4.unpack(p), codes)
+
+
+def test_bf16_rounding_matches_torch():
+    import torch
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(20000).astype(np.float32),
+                        np.array([1.00390625, 1.01171875, -1.00390625, 0.0, -0.0,
+                                  3.0e-39, 1e-45], dtype=np.float32)])
+    ours = nf4.bf16_bits_from_f32(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def _golden_figures():
+    out = {}
+    with open(os.path.join(GOLDEN, "pages_figures.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                name, val, tol = line.split()[:3]
+                out[name] = (float(val), float(tol))
+    return out
+
+
+def test_overhead_arithmetic_matches_pages():
+    fig = _golden_figures()
+
+    def near(name, x):
+        v, tol = fig[name]
+        assert abs(x - v) <= tol, (name, x, v)
+
+    fp32 = overhead.scale_bits_per_param(64, 32)
+    dq = overhead.dq_bits_per_param(64, 256)
+    assert fp32 == 0.5
+    assert abs(dq - (8 / 64 + 32 / (64 * 256))) < 1e-15
+    near("fp32_const_bits_per_param", fp32)
+    near("dq_const_bits_per_param", dq)
+    near("dq_saving_bits_per_param", fp32 - dq)
+    near("dq_saving_bits_rounded", fp32 - dq)
+    near("nf4_base_bytes_per_param", overhead.bits_per_param() / 8)
+    near("base_7b_gigabytes", 7e9 * 4 / 8 / 1e9)
+
+
+def test_stored_bytes_match_oracle_arrays():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((64, 64 * 40)) * 0.02).astype(np.float32)   # 2560 blocks
+    q = nf4.quantize(W)
+    nbytes = q["packed"].nbytes + q["q8"].nbytes + 4 * q["step2"].size + 4
+    assert nbytes == overhead.stored_bytes(*W.shape)
+    bits = 8.0 * nbytes / W.size
+    assert abs(bits - overhead.bits_per_param(n_params=W.size)) < 1e-12
