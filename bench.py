@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear layer on B200; prints ONE JSON line.
+
+Step = one QLoRA linear forward + backward (all kernels of the hot path:
+LoRA down-projection, fused dequant GEMM forward, du, fused dequant GEMM dx,
+dA, dB) on the Llama-7B attention-projection workload: in = out = 4096,
+M = 4096 tokens (batch 4 x seq 1024), r = 16, alpha = 32, frozen weight
+quantized once to NF4 with double quantization before timing.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1: launched with torch.distributed.run, one rank per GPU; every rank runs
+its own batch (data parallel, weak scaling) and the adapter gradients dA, dB
+are summed across ranks with one NCCL all-reduce per step.  Time = max over
+ranks of the CUDA-event time of exactly K steps, bracketed by barrier +
+synchronize.  `--impl reference` times the fp64 CPU oracle (rank 0 only) on a
+bounded token sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_nf4_quantized_11_b200 import synth, workloads  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 quant/GEMV GB/s, % of B200 roofline"
+L2_BYTES = 126 * 2 ** 20
+WL = workloads.ATTN_7B
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------- helpers
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rotations", type=int, default=4)
+    ap.add_argument("--no-components", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_nf4_quantized_11_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        if t.get("source_hash") != source_hash():
+            return None
+        return t["kernels"][workload][kernel]["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ---------------------------------------------------------------------------- our arm
+def step_flops(M, n_in, n_out, r):
+    return workloads.fwd_bwd_flops(M, n_in, n_out, r)
+
+
+def make_copies(q, M, n_in, n_out, r, n_rot, seed0, dev):
+    copies = []
+    for i in range(n_rot):
+        p = synth.problem(M, n_in, n_out, r, WL.w_std, WL.w_dist, seed=seed0 + 17 * i)
+        c = {k: p[k].to(dev) for k in ("x", "A", "B", "dh")}
+        c["w"] = q.quantize_nf4(p["W"].to(dev))
+        copies.append(c)
+    torch.cuda.synchronize()
+    return copies
+
+
+def run_ours(args, world, rank, local):
+    import bit_nf4_quantized_11_b200 as q
+    q.load()
+    dev = torch.device("cuda", local)
+    (_, n_in, n_out), = WL.projections
+    M, r, alpha = WL.M[0], WL.r, WL.alpha
+    copies = make_copies(q, M, n_in, n_out, r, args.rotations, 1000 * rank, dev)
+    h = torch.empty(M, n_out, dtype=torch.bfloat16, device=dev)
+    us = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    dx = torch.empty(M, n_in, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, n_in, dtype=torch.float32, device=dev)
+    dB = torch.empty(n_out, r, dtype=torch.float32, device=dev)
+    ws_f = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_FWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_BWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
+
+    def step(i):
+        c = copies[i % len(copies)]
+        q.linear_fwd(c["x"], c["w"], c["A"], c["B"], alpha, h=h, us=us, workspace=ws_f)
+        q.linear_bwd(c["dh"], c["x"], us, c["w"], c["A"], c["B"], alpha, dx=dx, dA=dA, dB=dB, workspace=ws_b)
+        if world > 1:                       # data-parallel adapter-gradient sync
+            torch.distributed.all_reduce(dA)
+            torch.distributed.all_reduce(dB)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if q.last_device_status() != 0:
+        raise RuntimeError("device wait timed out during warm-up")
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q.timing_reset()
+    q.timing_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    q.timing_enable(False)
+    ms = e0.elapsed_time(e1)
+    ms_max = max_over_ranks(ms, world)
+    if q.last_device_status() != 0:
+        raise RuntimeError("device wait timed out in the timed region")
+
+    flops = step_flops(M, n_in, n_out, r)
+    value = world * args.steps * flops / (ms_max * 1e-3) / 1e12
+
+    kern = {}
+    launches = 0
+    for name in q.KERNEL_NAMES:
+        t, n = q.timing_collect(name)
+        if n:
+            kern[name] = {"ms_per_step": t / args.steps, "launches": n, "avg_us": 1e3 * t / n}
+            launches += n
+    total_k = sum(v["ms_per_step"] for v in kern.values())
+    for v in kern.values():
+        v["share"] = v["ms_per_step"] / total_k if total_k else None
+
+    peaks, peak_src = load_peaks()
+    dom = max(("gemm_fwd", "gemm_dx"), key=lambda k: kern.get(k, {}).get("ms_per_step", 0.0))
+    dom_flops = 2.0 * M * (n_out * (n_in + r) if dom == "gemm_fwd" else n_in * (n_out + r))
+    achieved = dom_flops / (kern[dom]["avg_us"] * 1e-6) / 1e12
+    roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "peak_source": f"bf16_tflops_sustained of {peak_src} (kernel timed inside a long run of steps)",
+                "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "flops_per_launch": dom_flops,
+                "traffic": profiled_traffic(dom, WL.name)}
+
+    e2e = measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev)
+
+    rot_bytes = args.rotations * (2 * M * n_in + 2 * M * n_out + copies[0]["w"].nbytes())
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 activations and output grads, N(0,0.02^2) fp32 "
+                "weight quantized once to NF4 + double quant, U(+-1/64) A, N(0,0.01^2) B",
+        "config": {"workload": WL.name, "in_features": n_in, "out_features": n_out,
+                   "tokens_per_gpu": M, "r": r, "alpha": alpha, "global_tokens": M * world,
+                   "parallelism": f"dp{world}",
+                   "l2": f"inputs rotated over {args.rotations} copies ({rot_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "flops_per_step_per_gpu": flops},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "kernels": kern,
+    }
+    return line
+
+
+def measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev):
+    """Same step through the public API with inputs in pinned host memory:
+    every step copies x, dh host->device and h, dx, dA, dB device->host."""
+    c = copies[0]
+    xh = c["x"].cpu().pin_memory()
+    dhh = c["dh"].cpu().pin_memory()
+    x = torch.empty_like(c["x"])
+    dh = torch.empty_like(c["dh"])
+    h_host = torch.empty(M, n_out, dtype=torch.bfloat16).pin_memory()
+    dx_host = torch.empty(M, n_in, dtype=torch.bfloat16).pin_memory()
+    dA_host = torch.empty(r, n_in, dtype=torch.float32).pin_memory()
+    dB_host = torch.empty(n_out, r, dtype=torch.float32).pin_memory()
+    n = max(10, min(100, args.steps // 10))
+
+    def step():
+        x.copy_(xh, non_blocking=True)
+        dh.copy_(dhh, non_blocking=True)
+        h, us = q.linear_fwd(x, c["w"], c["A"], c["B"], alpha)
+        dx, dA, dB = q.linear_bwd(dh, x, us, c["w"], c["A"], c["B"], alpha)
+        if world > 1:
+            torch.distributed.all_reduce(dA)
+            torch.distributed.all_reduce(dB)
+        h_host.copy_(h, non_blocking=True)
+        dx_host.copy_(dx, non_blocking=True)
+        dA_host.copy_(dA, non_blocking=True)
+        dB_host.copy_(dB, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(n):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    flops = step_flops(M, n_in, n_out, r)
+    return {"value": world * n * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": 2 * M * n_in + 2 * M * n_out,
+            "d2h_bytes_per_step": 2 * M * n_out + 2 * M * n_in + 4 * r * n_in + 4 * n_out * r,
+            "steps": n, "ms_per_step": ms / n}
+
+
+# ---------------------------------------------------------------------------- oracle legs
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+class OracleLayer:
+    """The fp64 oracle set up once on the workload's weight (quantized and
+    dequantized by the oracle itself)."""
+
+    def __init__(self, seed=0):
+        from oracle import linear, nf4
+        (_, n_in, n_out), = WL.projections
+        self.linear, self.n_in, self.n_out, self.r, self.alpha = linear, n_in, n_out, WL.r, WL.alpha
+        p = synth.problem(WL.M[0], n_in, n_out, WL.r, WL.w_std, WL.w_dist, seed)
+        qo = nf4.quantize(p["W"].numpy())
+        self.Wd = nf4.dequantize(qo["codes"], qo["q8"], qo["step2"], qo["mean"])
+        self.x = p["x"].float().numpy().astype("float64")
+        self.dh = p["dh"].float().numpy().astype("float64")
+        self.A = p["A"].float().numpy().astype("float64")
+        self.B = p["B"].float().numpy().astype("float64")
+
+    def step(self, m0, m):
+        sl = slice(m0 % WL.M[0], m0 % WL.M[0] + m)
+        x, dh = self.x[sl], self.dh[sl]
+        self.linear.linear_fwd(x, self.Wd, self.A, self.B, self.alpha)
+        self.linear.linear_bwd(dh, x, self.Wd, self.A, self.B, self.alpha)
+        return step_flops(x.shape[0], self.n_in, self.n_out, self.r)
+
+
+def cpu_baseline(budget_s=15.0):
+    ol = OracleLayer()
+    t0 = time.perf_counter()
+    ol.step(0, 64)
+    per_tok = (time.perf_counter() - t0) / 64
+    m = int(max(64, min(WL.M[0], budget_s / max(per_tok, 1e-9))))
+    t0 = time.perf_counter()
+    flops = ol.step(0, m)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle fwd+bwd of {m} of the {WL.M[0]} tokens through the full "
+                      f"{ol.n_out}x{ol.n_in} layer (r={ol.r}); {dt:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    ol = OracleLayer()
+    t0 = time.perf_counter()
+    ol.step(0, 16)
+    per_tok = (time.perf_counter() - t0) / 16
+    budget = 120.0
+    m = int(max(1, min(WL.M[0], budget / max(per_tok, 1e-9) / max(1, args.steps + args.warmup))))
+    for i in range(args.warmup):
+        ol.step(i * m, m)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for i in range(args.steps):
+        flops += ol.step((args.warmup + i) * m, m)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    cores = blas_threads()
+    sample = f"fp64 NumPy oracle fwd+bwd of {m} tokens per step through the full {ol.n_out}x{ol.n_in} layer"
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded inputs as the GPU arm)",
+        "config": {"workload": WL.name, "in_features": ol.n_in, "out_features": ol.n_out,
+                   "tokens_per_step": m, "r": ol.r, "alpha": ol.alpha},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------- components
+def components(q, dev):
+    """Extra measurements outside the timed region: quantizer and dequantizer
+    HBM throughput, the few-token GEMV, and the other fwd+bwd workloads."""
+    out = {}
+    peaks, src = load_peaks()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    # quantizer + dequantizer on the 65B decoder layer's seven weights (3.2 GB fp32 > L2)
+    quant_res = []
+    ws = None
+    weights = []
+    for i, (label, n_in, n_out) in enumerate(workloads.LAYER_65B.projections):
+        W = synth.weight(n_out, n_in, workloads.LAYER_65B.w_std, seed=i).to(dev)
+        weights.append((label, W, q.alloc_nf4(n_out, n_in, dev)))
+    ws = torch.empty(max(q.workspace_size(q.OP_QUANTIZE, 0, W.shape[1], W.shape[0], 0)
+                         for _, W, _ in weights), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        for _, W, w in weights:
+            q.quantize_nf4(W, out=w, workspace=ws)
+    torch.cuda.synchronize()
+    q.timing_reset()
+    q.timing_enable(True)
+    a, b = ev(), ev()
+    reps = 3
+    a.record()
+    for _ in range(reps):
+        for _, W, w in weights:
+            q.quantize_nf4(W, out=w, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    q.timing_enable(False)
+    tot = a.elapsed_time(b) / reps
+    qbytes = sum(workloads.quant_bytes(*W.shape) for _, W, _ in weights)
+    kq, nq = q.timing_collect("quantize_blocks")
+    out["quantize_65b_layer"] = {
+        "weights": sum(W.numel() for _, W, _ in weights), "ms": tot, "GB/s": qbytes / (tot * 1e-3) / 1e9,
+        "frac_hbm": qbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "quantize_blocks_ms": kq / reps if nq else None,
+        "peak_source": f"hbm_gbs of {src}"}
+    # dequantizer (0.52 B/weight in, 2 B/weight out)
+    deq_out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _, _, w in weights]
+    for (_, _, w), o in zip(weights, deq_out):
+        q.dequantize_nf4(w, out=o)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        for (_, _, w), o in zip(weights, deq_out):
+            q.dequantize_nf4(w, out=o)
+    b.record()
+    torch.cuda.synchronize()
+    tot = a.elapsed_time(b) / reps
+    dbytes = sum(workloads.gemv_weight_bytes(w.rows, w.cols) + 2 * w.rows * w.cols for _, _, w in weights)
+    out["dequantize_65b_layer"] = {"ms": tot, "GB/s": dbytes / (tot * 1e-3) / 1e9,
+                                   "frac_hbm": dbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del deq_out, weights, ws
+    torch.cuda.empty_cache()
+
+    # few-token GEMV on the 70B MLP shapes
+    g = workloads.GEMV_70B
+    gres = {}
+    for (label, n_in, n_out) in g.projections:
+        ws_list = []
+        for i in range(3):              # 3 weight copies: 3 x 121 MB > L2
+            W = synth.weight(n_out, n_in, g.w_std, seed=10 + i).to(dev)
+            ws_list.append(q.quantize_nf4(W))
+            del W
+        A = synth.lora_A(g.r, n_in).to(dev)
+        B = synth.lora_B(n_out, g.r).to(dev)
+        for M in g.M:
+            x = synth.activations(M, n_in, seed=M).to(dev)
+            for i in range(3):
+                q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha)
+            torch.cuda.synchronize()
+            q.timing_reset()
+            q.timing_enable(True)
+            n = 60
+            a.record()
+            for i in range(n):
+                q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha)
+            b.record()
+            torch.cuda.synchronize()
+            q.timing_enable(False)
+            call_ms = a.elapsed_time(b) / n
+            kms, kn = q.timing_collect("gemv")
+            wbytes = workloads.gemv_weight_bytes(n_out, n_in)
+            gres[f"{label}_{n_in}x{n_out}_M{M}"] = {
+                "call_us": 1e3 * call_ms, "gemv_kernel_us": 1e3 * kms / kn if kn else None,
+                "packed_weight_GB/s_call": wbytes / (call_ms * 1e-3) / 1e9,
+                "packed_weight_GB/s_kernel": wbytes / (kms / kn * 1e-3) / 1e9 if kn else None,
+                "frac_hbm_kernel": (wbytes / (kms / kn * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kn else None}
+        del ws_list
+        torch.cuda.empty_cache()
+    out["gemv_70b"] = gres
+
+    # other fwd+bwd workloads: 7B MLP (3 projections) and 65B decoder layer (7 projections)
+    for wl in (workloads.MLP_7B, workloads.LAYER_65B):
+        M = wl.M[0]
+        tot_ms, tot_flops = 0.0, 0.0
+        for i, (label, n_in, n_out) in enumerate(wl.projections):
+            p = synth.problem(M, n_in, n_out, wl.r, wl.w_std, wl.w_dist, seed=i)
+            w = q.quantize_nf4(p["W"].to(dev))
+            x, A, B, dh = (p[k].to(dev) for k in ("x", "A", "B", "dh"))
+            del p
+            for _ in range(2):
+                hh, us = q.linear_fwd(x, w, A, B, wl.alpha)
+                q.linear_bwd(dh, x, us, w, A, B, wl.alpha)
+            torch.cuda.synchronize()
+            n = 5
+            a.record()
+            for _ in range(n):
+                hh, us = q.linear_fwd(x, w, A, B, wl.alpha)
+                q.linear_bwd(dh, x, us, w, A, B, wl.alpha)
+            b.record()
+            torch.cuda.synchronize()
+            tot_ms += a.elapsed_time(b) / n
+            tot_flops += step_flops(M, n_in, n_out, wl.r)
+            del w, x, A, B, dh, hh, us
+            torch.cuda.empty_cache()
+        out[wl.name] = {"ms": tot_ms, "TFLOP/s": tot_flops / (tot_ms * 1e-3) / 1e12,
+                        "frac_bf16_sustained": tot_flops / (tot_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+    return out
+
+
+# ---------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+            if line is not None:
+                print(json.dumps(line), flush=True)
+            return
+        line = run_ours(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        elif rank == 0:
+            line["cpu_baseline"] = None
+        if rank == 0 and world == 1 and not args.no_components:
+            import bit_nf4_quantized_11_b200 as q
+            line["components"] = components(q, torch.device("cuda", local))
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

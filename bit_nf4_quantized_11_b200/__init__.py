@@ -1,0 +1,270 @@
+"""QLoRA NF4 linear layer for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libqlora_nf4.so`` (declared in
+``include/qlora_nf4.h``).  This module only marshals arguments: it checks
+dtypes and devices, allocates the caller-owned outputs and workspaces with
+PyTorch, and passes raw pointers plus the current CUDA stream to the library.
+Every step of the computation runs in the library's CUDA kernels; there is no
+fallback path.  If the shared library is missing, :func:`load` raises.
+
+Entry points (same names as the C ABI, without the ``qlora_`` prefix):
+  codebook()                      -> (levels[16], thresholds[15])
+  quantize_nf4(W)                 -> NF4Weight
+  dequantize_nf4(w)               -> bf16 [rows, cols]
+  linear_fwd(x, w, A, B, alpha)   -> (h, us)
+  linear_bwd(dh, x, us, w, A, B, alpha) -> (dx, dA, dB)
+  workspace_size(op, M, in_features, out_features, r)
+  last_device_status(), set_wait_timeout_ns(ns), selftest_wait_timeout()
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "load", "library_path", "codebook", "NF4Weight", "quantize_nf4", "dequantize_nf4",
+    "linear_fwd", "linear_bwd", "workspace_size", "last_device_status",
+    "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
+    "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES",
+    "OP_QUANTIZE", "OP_DEQUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD",
+]
+
+OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
+STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTED_SHAPE",
+          -3: "QLORA_ERR_WORKSPACE", -4: "QLORA_ERR_CUDA", -5: "QLORA_ERR_TIMEOUT"}
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+def library_path() -> str:
+    return os.path.join(_PKG_DIR, "libqlora_nf4.so")
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status_string(status)})")
+        self.status = status
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("q8", ctypes.c_void_p), ("step2", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+def load():
+    """Load libqlora_nf4.so (built in-tree); raises if it is missing."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m bit_nf4_quantized_11_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    P, I64, I, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    W = ctypes.POINTER(_Weight)
+    sig = {
+        "qlora_nf4_codebook": (I, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
+        "qlora_workspace_size": (SZ, [I, I64, I64, I64, I]),
+        "qlora_quantize_nf4": (I, [P, I64, I64, P, P, P, P, P, SZ, P]),
+        "qlora_dequantize_nf4": (I, [W, P, P]),
+        "qlora_linear_fwd": (I, [P, I64, W, P, P, I, F, P, P, P, SZ, P]),
+        "qlora_linear_bwd": (I, [P, P, P, I64, W, P, P, I, F, P, P, P, P, SZ, P]),
+        "qlora_last_device_status": (I, [P]),
+        "qlora_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+        "qlora_selftest_wait_timeout": (I, [P]),
+        "qlora_status_string": (ctypes.c_char_p, [I]),
+        "qlora_timing_enable": (I, [I]),
+        "qlora_timing_reset": (None, []),
+        "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
+                                     ctypes.POINTER(ctypes.c_int64)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _LIB = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().qlora_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise QLoRAError(status, what)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t, dtype, name, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+@dataclass
+class NF4Weight:
+    """A quantized weight W0 [rows=out, cols=in] in the library's storage format."""
+    codes: torch.Tensor   # uint8 [rows, cols/2]
+    q8: torch.Tensor      # int8  [rows*cols/64]
+    step2: torch.Tensor   # fp32  [ceil(n_blocks/256)]
+    mean: torch.Tensor    # fp32  [1]
+    rows: int
+    cols: int
+
+    def _c(self) -> _Weight:
+        return _Weight(self.codes.data_ptr(), self.q8.data_ptr(), self.step2.data_ptr(),
+                       self.mean.data_ptr(), self.rows, self.cols)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.q8, self.step2, self.mean))
+
+
+def codebook():
+    """The 16 NF4 levels and 15 thresholds computed by the library (host)."""
+    lib = load()
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(lib.qlora_nf4_codebook(lv, th), "qlora_nf4_codebook")
+    return list(lv), list(th)
+
+
+def workspace_size(op: int, M: int, in_features: int, out_features: int, r: int) -> int:
+    n = load().qlora_workspace_size(int(op), int(M), int(in_features), int(out_features), int(r))
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid workspace query")
+    return int(n)
+
+
+def _workspace(nbytes: int, device, ws=None):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def alloc_nf4(rows: int, cols: int, device) -> NF4Weight:
+    n_blocks = rows * cols // 64
+    n_groups = -(-n_blocks // 256)
+    return NF4Weight(
+        codes=torch.empty((rows, cols // 2), dtype=torch.uint8, device=device),
+        q8=torch.empty(n_blocks, dtype=torch.int8, device=device),
+        step2=torch.empty(n_groups, dtype=torch.float32, device=device),
+        mean=torch.empty(1, dtype=torch.float32, device=device),
+        rows=rows, cols=cols)
+
+
+def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, workspace=None) -> NF4Weight:
+    """NF4 + double quantization of an fp32 weight [rows, cols] (cols % 64 == 0)."""
+    _need(W, torch.float32, "W")
+    rows, cols = W.shape
+    w = out if out is not None else alloc_nf4(rows, cols, W.device)
+    ws = _workspace(workspace_size(OP_QUANTIZE, 0, cols, rows, 0), W.device, workspace)
+    _check(load().qlora_quantize_nf4(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2),
+                                     _ptr(w.mean), _ptr(ws), ws.numel() if ws is not None else 0,
+                                     _stream()), "qlora_quantize_nf4")
+    return w
+
+
+def dequantize_nf4(w: NF4Weight, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [rows, cols] dequantized weight."""
+    o = out if out is not None else torch.empty((w.rows, w.cols), dtype=torch.bfloat16, device=w.codes.device)
+    _need(o, torch.bfloat16, "out", (w.rows, w.cols))
+    cw = w._c()
+    _check(load().qlora_dequantize_nf4(ctypes.byref(cw), _ptr(o), _stream()), "qlora_dequantize_nf4")
+    return o
+
+
+def linear_fwd(x, w: NF4Weight, A, B, alpha: float, h=None, us=None, workspace=None):
+    """h = x dequant(W0)^T + us B^T with us = bf16((alpha/r) x A^T); returns (h, us)."""
+    M = x.shape[0]
+    r = A.shape[0]
+    _need(x, torch.bfloat16, "x", (M, w.cols))
+    _need(A, torch.bfloat16, "A", (r, w.cols))
+    _need(B, torch.bfloat16, "B", (w.rows, r))
+    h = h if h is not None else torch.empty((M, w.rows), dtype=torch.bfloat16, device=x.device)
+    us = us if us is not None else torch.empty((M, r), dtype=torch.bfloat16, device=x.device)
+    _need(h, torch.bfloat16, "h", (M, w.rows))
+    _need(us, torch.bfloat16, "us", (M, r))
+    ws = _workspace(workspace_size(OP_LINEAR_FWD, M, w.cols, w.rows, r), x.device, workspace)
+    cw = w._c()
+    _check(load().qlora_linear_fwd(_ptr(x), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha),
+                                   _ptr(h), _ptr(us), _ptr(ws), ws.numel() if ws is not None else 0,
+                                   _stream()), "qlora_linear_fwd")
+    return h, us
+
+
+def linear_bwd(dh, x, us, w: NF4Weight, A, B, alpha: float, dx=None, dA=None, dB=None, workspace=None):
+    """Backward with W0 frozen; returns (dx bf16 [M, in], dA fp32 [r, in], dB fp32 [out, r])."""
+    M = x.shape[0]
+    r = A.shape[0]
+    _need(dh, torch.bfloat16, "dh", (M, w.rows))
+    _need(x, torch.bfloat16, "x", (M, w.cols))
+    _need(us, torch.bfloat16, "us", (M, r))
+    _need(A, torch.bfloat16, "A", (r, w.cols))
+    _need(B, torch.bfloat16, "B", (w.rows, r))
+    dev = x.device
+    dx = dx if dx is not None else torch.empty((M, w.cols), dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty((r, w.cols), dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty((w.rows, r), dtype=torch.float32, device=dev)
+    ws = _workspace(workspace_size(OP_LINEAR_BWD, M, w.cols, w.rows, r), dev, workspace)
+    cw = w._c()
+    _check(load().qlora_linear_bwd(_ptr(dh), _ptr(x), _ptr(us), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                   float(alpha), _ptr(dx), _ptr(dA), _ptr(dB), _ptr(ws),
+                                   ws.numel() if ws is not None else 0, _stream()), "qlora_linear_bwd")
+    return dx, dA, dB
+
+
+def last_device_status() -> int:
+    """Synchronize the current stream, read and clear the device error flag."""
+    return int(load().qlora_last_device_status(_stream()))
+
+
+def set_wait_timeout_ns(ns: int) -> int:
+    return int(load().qlora_set_wait_timeout_ns(int(ns)))
+
+
+def selftest_wait_timeout() -> int:
+    return int(load().qlora_selftest_wait_timeout(_stream()))
+
+
+KERNEL_NAMES = ("quantize_blocks", "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
+                "gemv", "gemv_finalize", "lora_rowwise", "lora_colwise", "sum_chunks", "transpose")
+
+
+def timing_enable(on: bool = True) -> bool:
+    """Bracket every library kernel launch with CUDA events on its stream."""
+    return bool(load().qlora_timing_enable(1 if on else 0))
+
+
+def timing_reset() -> None:
+    load().qlora_timing_reset()
+
+
+def timing_collect(kernel: str):
+    """(total device ms, launches) of one kernel since the last reset."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int64(0)
+    _check(load().qlora_timing_collect(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)),
+           "qlora_timing_collect")
+    return ms.value, n.value
+

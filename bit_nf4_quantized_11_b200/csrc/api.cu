@@ -1,0 +1,562 @@
+// api.cu -- the C ABI of libqlora_nf4.so: argument validation, workspace
+// layout, tensor-map encoding and kernel launches.  Declarations and the
+// contract of every entry point are in include/qlora_nf4.h.
+#include "qlora_nf4.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "gemm_sm100.cuh"
+#include "gemv.cuh"
+#include "quant.cuh"
+#include "skinny.cuh"
+
+namespace qnf4_host {
+void build_codebook(float levels[16], float thresholds[15]);
+}
+
+namespace {
+
+using qnf4::Levels;
+using qnf4::Thresholds;
+
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+
+struct Tables {
+  Levels L;
+  Thresholds T;
+};
+
+const Tables& tables() {
+  static Tables t;
+  static std::once_flag once;
+  std::call_once(once, [] { qnf4_host::build_codebook(t.L.v, t.T.v); });
+  return t;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+
+// ------------------------------------------------------------------ timing
+struct TimedLaunch {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timing_mu;
+std::atomic<int> g_timing_on{0};
+std::vector<TimedLaunch> g_timed;       // recorded launches since the last reset
+std::vector<cudaEvent_t> g_event_pool;  // events free for reuse
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets the kernel launches made during its lifetime with two events.
+class LaunchTimer {
+ public:
+  LaunchTimer(const char* name, cudaStream_t st) : name_(name), st_(st) {
+    if (!g_timing_on.load()) return;
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    start_ = pool_event();
+    stop_ = pool_event();
+    if (start_ && stop_) cudaEventRecord(start_, st_);
+  }
+  ~LaunchTimer() {
+    if (!start_ || !stop_) return;
+    cudaEventRecord(stop_, st_);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timed.push_back({name_, start_, stop_});
+  }
+  LaunchTimer(const LaunchTimer&) = delete;
+  LaunchTimer& operator=(const LaunchTimer&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t st_;
+  cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
+#define QLORA_CUDA_TRY(expr)                          \
+  do {                                                \
+    if ((expr) != cudaSuccess) return QLORA_ERR_CUDA; \
+  } while (0)
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] tensor, box {64 cols, 128 rows}, 128B swizzle,
+// out-of-range elements read as zero.
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------------------ workspace
+struct QuantWs {
+  size_t absmax_off, tree_off, total;
+  int64_t tree_count;  // doubles reserved for all tree passes
+};
+
+QuantWs quant_ws(int64_t rows, int64_t cols) {
+  QuantWs w{};
+  const int64_t n_blocks = rows * cols / 64;
+  w.absmax_off = 0;
+  w.tree_off = round256(static_cast<size_t>(n_blocks) * 4);
+  int64_t count = 0, n = n_blocks;
+  do {
+    n = cdiv(n, qnf4::kTreeChunk);
+    count += n;
+  } while (n > 1);
+  w.tree_count = count;
+  w.total = w.tree_off + round256(static_cast<size_t>(count) * 8);
+  return w;
+}
+
+struct GemvPlan {
+  int splits, blocks_per_split;
+};
+
+GemvPlan gemv_plan(int64_t in, int64_t out) {
+  const int64_t nb = in / 64;
+  const int64_t row_ctas = cdiv(out, qnf4::kGemvRowsPerCta);
+  const int64_t target = 4 * static_cast<int64_t>(device_sm_count());
+  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(nb, cdiv(target, row_ctas)));
+  const int64_t bps = cdiv(nb, splits);
+  splits = cdiv(nb, bps);
+  return {static_cast<int>(splits), static_cast<int>(bps)};
+}
+
+size_t fwd_ws(int64_t M, int64_t in, int64_t out) {
+  if (M <= 16) {
+    const GemvPlan p = gemv_plan(in, out);
+    return round256(static_cast<size_t>(p.splits) * 16 * out * 4);
+  }
+  return 0;
+}
+
+struct BwdWs {
+  size_t du_off, bt_off, dbp_off, dap_off, total;
+  int chunks;
+};
+
+BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
+  BwdWs w{};
+  w.chunks = static_cast<int>(cdiv(M, qnf4::kColChunk));
+  w.du_off = 0;
+  w.bt_off = w.du_off + round256(static_cast<size_t>(M) * r * 2);
+  w.dbp_off = w.bt_off + round256(static_cast<size_t>(r) * out * 2);
+  w.dap_off = w.dbp_off + round256(static_cast<size_t>(w.chunks) * out * r * 4);
+  w.total = w.dap_off + round256(static_cast<size_t>(w.chunks) * in * r * 4);
+  return w;
+}
+
+// ------------------------------------------------------------------ launches
+int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
+                    float* mean, void* ws, cudaStream_t st) {
+  const Tables& tb = tables();
+  const int64_t n_blocks = rows * cols / 64;
+  const QuantWs w = quant_ws(rows, cols);
+  float* absmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.absmax_off);
+  double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + w.tree_off);
+
+  const int sms = device_sm_count();
+  const int64_t want = cdiv(n_blocks, 16);
+  const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
+  {
+    LaunchTimer lt_("quantize_blocks", st);
+    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.T);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+
+  // fixed summation tree, one pass per 4096x reduction
+  int64_t n = n_blocks;
+  int64_t parts = cdiv(n, qnf4::kTreeChunk);
+  {
+    LaunchTimer lt_("scale_mean_tree", st);
+    qnf4::pairwise_tree_kernel<float><<<static_cast<unsigned>(parts), 256, 0, st>>>(
+      absmax, n, tree, n_blocks, parts == 1 ? mean : nullptr);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  double* prev = tree;
+  while (parts > 1) {
+    n = parts;
+    parts = cdiv(n, qnf4::kTreeChunk);
+    double* next = prev + n;
+    {
+    LaunchTimer lt_("scale_mean_tree", st);
+    qnf4::pairwise_tree_kernel<double><<<static_cast<unsigned>(parts), 256, 0, st>>>(
+        prev, n, next, n_blocks, parts == 1 ? mean : nullptr);
+  }
+    QLORA_CUDA_TRY(cudaGetLastError());
+    prev = next;
+  }
+
+  const int64_t n_groups = cdiv(n_blocks, qnf4::kGroup);
+  {
+    LaunchTimer lt_("dq_scales", st);
+    qnf4::dq_scales_kernel<<<static_cast<unsigned>(cdiv(n_groups * 32, 256)), 256, 0, st>>>(absmax, n_blocks, mean,
+                                                                                          q8, step2);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+int gemm_tile_m(int64_t M) {
+  static int forced = [] {
+    const char* e = std::getenv("QLORA_NF4_GEMM_TILE_M");
+    return e ? std::atoi(e) : 0;
+  }();
+  if (forced == 128 || forced == 256) return forced;
+  return M >= 1024 ? 256 : 128;
+}
+
+template <int MS, bool kDx, int kStages>
+int launch_gemm_t(const qnf4::GemmArgs& args, const CUtensorMap& tm_act, const CUtensorMap& tm_lora,
+                  cudaStream_t st) {
+  using Cfg = qnf4::GemmCfg<MS, kStages>;
+  auto kern = qnf4::qlora_gemm_kernel<MS, kDx, kStages>;
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+  const int64_t tiles = cdiv(args.M, Cfg::BM) * cdiv(args.N, Cfg::BN);
+  {
+    LaunchTimer lt_(kDx ? "gemm_dx" : "gemm_fwd", st);
+    kern<<<static_cast<unsigned>(tiles), Cfg::THREADS, Cfg::SMEM, st>>>(tm_act, tm_lora, args);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+// act [M, K] and lora_act [M, r] are the A operands; the output has N columns.
+int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t M, int64_t K,
+                const uint16_t* lora_act, const uint16_t* lora_w, int r, uint16_t* out, int64_t N,
+                cudaStream_t st) {
+  CUtensorMap tm_act, tm_lora;
+  if (!make_tmap_bf16(&tm_act, act, M, K)) return QLORA_ERR_CUDA;
+  if (!make_tmap_bf16(&tm_lora, lora_act, M, r)) return QLORA_ERR_CUDA;
+  qnf4::GemmArgs a{};
+  a.codes = w->codes;
+  a.q8 = w->q8;
+  a.step2 = w->step2;
+  a.mean = w->mean;
+  a.lora_w = lora_w;
+  a.out = out;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.r = r;
+  a.w_cols = static_cast<int>(w->cols);
+  a.L = tables().L;
+  a.timeout_ns = g_timeout_ns.load();
+  const int tm = gemm_tile_m(M);
+  if (!dx) {
+    return tm == 256 ? launch_gemm_t<2, false, 3>(a, tm_act, tm_lora, st)
+                     : launch_gemm_t<1, false, 4>(a, tm_act, tm_lora, st);
+  }
+  return tm == 256 ? launch_gemm_t<2, true, 3>(a, tm_act, tm_lora, st)
+                   : launch_gemm_t<1, true, 4>(a, tm_act, tm_lora, st);
+}
+
+int launch_rowwise(const uint16_t* act, const uint16_t* Wt, uint16_t* out, int64_t M, int64_t K, int R,
+                   float scale, cudaStream_t st) {
+  {
+    LaunchTimer lt_("lora_rowwise", st);
+    qnf4::rowwise_skinny_kernel<<<static_cast<unsigned>(cdiv(M, 16)), qnf4::kRowThreads, 0, st>>>(
+      act, Wt, out, static_cast<int>(M), static_cast<int>(K), R, scale);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+int launch_colwise_sum(const uint16_t* act, const uint16_t* u, float* part, int64_t M, int64_t P, int R,
+                       float* out, bool transpose, cudaStream_t st) {
+  const int chunks = static_cast<int>(cdiv(M, qnf4::kColChunk));
+  dim3 grid(static_cast<unsigned>(cdiv(P, 128)), static_cast<unsigned>(chunks));
+  {
+    LaunchTimer lt_("lora_colwise", st);
+    qnf4::colwise_skinny_kernel<<<grid, qnf4::kColThreads, 0, st>>>(act, u, part, static_cast<int>(M),
+                                                                  static_cast<int>(P), R);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  const int64_t n_el = P * R;
+  const int grid2 = static_cast<int>(std::min<int64_t>(cdiv(n_el, 256), 4096));
+  {
+    LaunchTimer lt_("sum_chunks", st);
+    qnf4::sum_chunks_kernel<<<grid2, 256, 0, st>>>(part, chunks, static_cast<int>(P), R, out, transpose ? 1 : 0);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+// ------------------------------------------------------------------ validation
+bool weight_ok(const qlora_nf4_weight* w) {
+  return w != nullptr && w->codes && w->q8 && w->step2 && w->mean && aligned(w->codes, 16) &&
+         aligned(w->q8, 16) && aligned(w->step2, 16) && aligned(w->mean, 16);
+}
+
+int check_linear_shapes(int64_t M, const qlora_nf4_weight* w, int r) {
+  if (M < 1 || w->rows < 64 || w->cols < 64) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (w->cols % 64 != 0 || w->rows % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (r < 8 || r > 256 || r % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1ll << 31) - 1024 || w->rows > (1ll << 30) || w->cols > (1ll << 30))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (w->rows * w->cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return QLORA_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+int qlora_nf4_codebook(float levels[16], float thresholds[15]) {
+  if (levels == nullptr) return QLORA_ERR_INVALID_ARG;
+  const Tables& t = tables();
+  std::memcpy(levels, t.L.v, sizeof(t.L.v));
+  if (thresholds != nullptr) std::memcpy(thresholds, t.T.v, sizeof(t.T.v));
+  return QLORA_OK;
+}
+
+size_t qlora_workspace_size(int op, int64_t M, int64_t in_features, int64_t out_features, int r) {
+  if (M < 0 || in_features < 0 || out_features < 0 || r < 0) return static_cast<size_t>(-1);
+  switch (op) {
+    case QLORA_OP_QUANTIZE:
+      if (in_features < 64 || out_features < 1) return 0;
+      return quant_ws(out_features, in_features).total;
+    case QLORA_OP_DEQUANTIZE:
+      return 0;
+    case QLORA_OP_LINEAR_FWD:
+      if (M < 1) return 0;
+      return fwd_ws(M, in_features, out_features);
+    case QLORA_OP_LINEAR_BWD:
+      if (M < 1 || r < 1) return 0;
+      return bwd_ws(M, in_features, out_features, r).total;
+    default:
+      return static_cast<size_t>(-1);
+  }
+}
+
+int qlora_quantize_nf4(const float* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
+                       float* mean, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!W || !codes || !q8 || !step2 || !mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(q8, 16) || !aligned(step2, 16) || !aligned(mean, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 64 || cols % 64 != 0 || rows * cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const QuantWs w = quant_ws(rows, cols);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
+  return launch_quantize(W, rows, cols, codes, q8, step2, mean, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
+  if (!weight_ok(w) || !W_out || !aligned(W_out, 16)) return QLORA_ERR_INVALID_ARG;
+  if (w->rows < 1 || w->cols < 64 || w->cols % 64 != 0 || w->rows * w->cols > (1ll << 40))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t halves = w->rows * w->cols / 32;
+  const int64_t want = cdiv(halves, 256);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, device_sm_count() * 16)));
+  {
+    LaunchTimer lt_("dequantize", static_cast<cudaStream_t>(stream));
+    qnf4::nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      w->codes, w->q8, w->step2, w->mean, halves, W_out, tables().L);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
+                     const uint16_t* B, int r, float alpha, uint16_t* h, uint16_t* us_out, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  if (!x || !weight_ok(w) || !A || !B || !h || !us_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(h, 16) || !aligned(us_out, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  const int sc = check_linear_shapes(M, w, r);
+  if (sc != QLORA_OK) return sc;
+  const int64_t in = w->cols, out = w->rows;
+  const size_t need = fwd_ws(M, in, out);
+  if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float s = alpha / static_cast<float>(r);
+
+  int rc = launch_rowwise(x, A, us_out, M, in, r, s, st);           // us = bf16(s x A^T)
+  if (rc != QLORA_OK) return rc;
+  if (M <= 16) {
+    const GemvPlan p = gemv_plan(in, out);
+    qnf4::GemvArgs g{};
+    g.codes = w->codes;
+    g.q8 = w->q8;
+    g.step2 = w->step2;
+    g.mean = w->mean;
+    g.x = x;
+    g.part = static_cast<float*>(workspace);
+    g.M = static_cast<int>(M);
+    g.in = static_cast<int>(in);
+    g.out = static_cast<int>(out);
+    g.blocks_per_split = p.blocks_per_split;
+    g.L = tables().L;
+    const int smem = 256 * 32 * 4;
+    QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::nf4_gemv_splitk_kernel,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    dim3 grid(static_cast<unsigned>(cdiv(out, qnf4::kGemvRowsPerCta)), static_cast<unsigned>(p.splits));
+    {
+    LaunchTimer lt_("gemv", st);
+    qnf4::nf4_gemv_splitk_kernel<<<grid, qnf4::kGemvThreads, smem, st>>>(g);
+  }
+    QLORA_CUDA_TRY(cudaGetLastError());
+    const int64_t n_el = M * out;
+    {
+    LaunchTimer lt_("gemv_finalize", st);
+    qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(cdiv(n_el, 256)), 256, 0, st>>>(
+        g.part, p.splits, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
+  }
+    QLORA_CUDA_TRY(cudaGetLastError());
+    return QLORA_OK;
+  }
+  return launch_gemm(false, w, x, M, in, us_out, B, r, h, out, st);  // h = [x|us] [W0|B]^T
+}
+
+int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
+                     const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* dx, float* dA, float* dB, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dh || !x || !us || !weight_ok(w) || !A || !B || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(dh, 16) || !aligned(x, 16) || !aligned(us, 16) || !aligned(A, 16) || !aligned(B, 16) ||
+      !aligned(dx, 16) || !aligned(dA, 16) || !aligned(dB, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  const int sc = check_linear_shapes(M, w, r);
+  if (sc != QLORA_OK) return sc;
+  const int64_t in = w->cols, out = w->rows;
+  const BwdWs ws = bwd_ws(M, in, out, r);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
+  uint16_t* Bt = reinterpret_cast<uint16_t*>(base + ws.bt_off);
+  float* dBp = reinterpret_cast<float*>(base + ws.dbp_off);
+  float* dAp = reinterpret_cast<float*>(base + ws.dap_off);
+  const float s = alpha / static_cast<float>(r);
+
+  dim3 tg(static_cast<unsigned>(cdiv(r, 32)), static_cast<unsigned>(cdiv(out, 32)));
+  {
+    LaunchTimer lt_("transpose", st);
+    qnf4::transpose_bf16_kernel<<<tg, 256, 0, st>>>(B, static_cast<int>(out), r, Bt);     // B^T [r, out]
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  int rc = launch_rowwise(dh, Bt, du, M, out, r, s, st);                             // du = bf16(s dh B)
+  if (rc != QLORA_OK) return rc;
+  rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
+  if (rc != QLORA_OK) return rc;
+  rc = launch_colwise_sum(dh, us, dBp, M, out, r, dB, false, st);                     // dB = dh^T us
+  if (rc != QLORA_OK) return rc;
+  return launch_colwise_sum(x, du, dAp, M, in, r, dA, true, st);                      // dA = du^T x
+}
+
+int qlora_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return QLORA_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, qnf4::g_device_error, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (flag != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(qnf4::g_device_error, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_ERR_TIMEOUT;
+  }
+  return QLORA_OK;
+}
+
+uint64_t qlora_set_wait_timeout_ns(uint64_t ns) {
+  if (ns < 1000) ns = 1000;
+  return g_timeout_ns.exchange(ns);
+}
+
+int qlora_selftest_wait_timeout(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  qnf4::wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(g_timeout_ns.load());
+  if (cudaGetLastError() != cudaSuccess) return QLORA_ERR_CUDA;
+  return qlora_last_device_status(stream);
+}
+
+int qlora_timing_enable(int on) { return g_timing_on.exchange(on != 0 ? 1 : 0); }
+
+void qlora_timing_reset(void) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  for (auto& t : g_timed) {
+    g_event_pool.push_back(t.start);
+    g_event_pool.push_back(t.stop);
+  }
+  g_timed.clear();
+}
+
+int qlora_timing_collect(const char* kernel, double* total_ms, int64_t* launches) {
+  if (kernel == nullptr) return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  double sum = 0.0;
+  int64_t n = 0;
+  for (auto& t : g_timed) {
+    if (std::strcmp(t.name, kernel) != 0) continue;
+    if (cudaEventSynchronize(t.stop) != cudaSuccess) return QLORA_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t.start, t.stop) != cudaSuccess) return QLORA_ERR_CUDA;
+    sum += ms;
+    ++n;
+  }
+  if (total_ms) *total_ms = sum;
+  if (launches) *launches = n;
+  return QLORA_OK;
+}
+
+const char* qlora_status_string(int status) {
+  switch (status) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad scalar)";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case QLORA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "a device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,187 @@
+// quant.cuh -- NF4 blockwise quantizer with double quantization, and the
+// standalone dequantizer (sm_100a, CUDA cores; all HBM-streaming kernels).
+//
+// Method ("QLoRA", llm-compass, 方法与公式 items 1-2; learn-interview-questions
+// QLoRA page, section 2): 64-weight blocks, one absmax per block, nearest of
+// 16 normal-quantile levels; the fp32 block absmaxes are quantized again to
+// 8 bit around their mean, one fp32 step per group of 256 blocks.
+//
+// Every fp32 operation below is a separately rounded IEEE operation
+// (__fmul_rn/__fadd_rn/__fsub_rn/__fdiv_rn/__frcp_rn, fp64 __dadd_rn/__ddiv_rn),
+// so the packed codes, the int8 scale codes, the steps, the mean and the
+// dequantized bf16 weights are bit-reproducible.
+#pragma once
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+constexpr int kBlock = 64;        // weights per first-level block
+constexpr int kGroup = 256;       // blocks per second-level group
+constexpr int kTreeChunk = 4096;  // leaves summed by one CTA of the scale-mean tree
+
+// ---------------------------------------------------------------------------
+// K1: per-block absmax, nearest-level code, nibble packing.
+// One half-warp per 64-weight block: each lane loads 4 fp32 (16 B), the
+// absmax is reduced over the 16 lanes, and each lane packs its 4 codes into
+// 2 bytes, so a block's 32 code bytes are written by one coalesced store.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t nearest_code(float v, const float* s_thr) {
+  // number of thresholds strictly below v, by binary search over the 15
+  // ascending thresholds (thresholds in shared memory: every lane may read a
+  // different one without serialising)
+  uint32_t c = (v > s_thr[7]) ? 8u : 0u;
+  c += (v > s_thr[c + 3]) ? 4u : 0u;
+  c += (v > s_thr[c + 1]) ? 2u : 0u;
+  c += (v > s_thr[c]) ? 1u : 0u;
+  return c;
+}
+
+__global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
+    const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
+    float* __restrict__ absmax, Thresholds thr) {
+  __shared__ float s_thr[16];
+  if (threadIdx.x < 15) s_thr[threadIdx.x] = thr.v[threadIdx.x];
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;          // which of the warp's two blocks
+  const int l16 = lane & 15;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t pair = warp; pair * 2 < n_blocks; pair += n_warps) {
+    const int64_t b = pair * 2 + half;
+    const bool valid = b < n_blocks;
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) {
+      const uint4 u = ld_stream_v4(W + b * kBlock + l16 * 4);
+      w = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+    }
+    float m = fmaxf(fmaxf(fabsf(w.x), fabsf(w.y)), fmaxf(fabsf(w.z), fabsf(w.w)));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    // m is now the exact absmax of this half-warp's block
+    uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
+    if (m > 0.f) {
+      const float r = __frcp_rn(m);
+      c0 = nearest_code(__fmul_rn(w.x, r), s_thr);
+      c1 = nearest_code(__fmul_rn(w.y, r), s_thr);
+      c2 = nearest_code(__fmul_rn(w.z, r), s_thr);
+      c3 = nearest_code(__fmul_rn(w.w, r), s_thr);
+    }
+    if (valid) {
+      const uint16_t packed = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
+      reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = packed;
+      if (l16 == 0) absmax[b] = m;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K2: fixed fp64 summation tree over the block absmaxes.
+// The tree is defined on the whole array zero-padded to a power of two, with
+// adjacent pairs added level by level.  One CTA (256 threads) sums an aligned
+// chunk of 4096 leaves: 16 consecutive leaves per thread (in-register tree),
+// then a xor-butterfly across the warp (offset 1, 2, 4, ... adds adjacent
+// pairs), then the 8 warp sums pairwise.  Chunks are aligned subtrees, so
+// repeating the pass over the chunk sums reproduces the full tree exactly;
+// missing leaves are exact zeros.  The pass that leaves one value also writes
+// mean = fp32(T / n_leaves) with the division in fp64.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(256) pairwise_tree_kernel(
+    const T* __restrict__ in, int64_t n, double* __restrict__ out,
+    int64_t n_leaves_total, float* __restrict__ mean_out) {
+  __shared__ double s_warp[8];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTreeChunk + threadIdx.x * 16;
+  double v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (base + i < n) ? static_cast<double>(in[base + i]) : 0.0;
+#pragma unroll
+  for (int width = 8; width >= 1; width >>= 1) {
+#pragma unroll
+    for (int i = 0; i < width; ++i) v[i] = __dadd_rn(v[2 * i], v[2 * i + 1]);
+  }
+  double s = v[0];
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
+  if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double a = __dadd_rn(__dadd_rn(s_warp[0], s_warp[1]), __dadd_rn(s_warp[2], s_warp[3]));
+    const double b = __dadd_rn(__dadd_rn(s_warp[4], s_warp[5]), __dadd_rn(s_warp[6], s_warp[7]));
+    const double t = __dadd_rn(a, b);
+    out[blockIdx.x] = t;
+    if (mean_out != nullptr)   // single-chunk pass: t is the whole tree
+      *mean_out = __double2float_rn(__ddiv_rn(t, static_cast<double>(n_leaves_total)));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K3: second-level codes.  One warp per group of 256 block scales:
+// d = fp32(c - mean), step2 = fp32(max|d| / 127),
+// q8 = clamp(rne(fp32(d * fp32(1/step2))), -127, 127); 0 when step2 == 0 or
+// the product is NaN.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dq_scales_kernel(
+    const float* __restrict__ absmax, int64_t n_blocks, const float* __restrict__ mean_ptr,
+    int8_t* __restrict__ q8, float* __restrict__ step2) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_groups = (n_blocks + kGroup - 1) / kGroup;
+  if (g >= n_groups) return;                       // warp-uniform
+  const float mu = *mean_ptr;
+  float d[8];
+  float S = 0.f;
+  const int64_t base = g * kGroup + lane * 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t idx = base + i;
+    d[i] = (idx < n_blocks) ? __fsub_rn(absmax[idx], mu) : 0.f;
+    S = fmaxf(S, fabsf(d[i]));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) S = fmaxf(S, __shfl_xor_sync(0xffffffffu, S, off));
+  const float st = __fdiv_rn(S, 127.0f);
+  if (lane == 0) step2[g] = st;
+  const float inv = (st != 0.f) ? __frcp_rn(st) : 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t idx = base + i;
+    if (idx >= n_blocks) break;
+    int q = 0;
+    if (st != 0.f) {
+      const float p = __fmul_rn(d[i], inv);
+      if (p == p) q = min(127, max(-127, __float2int_rn(p)));
+    }
+    q8[idx] = static_cast<int8_t>(q);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K4: dequantize to bf16.  One thread per 32 codes (16 bytes, half a block):
+// it forms the block scale, the block's 16-entry bf16 table, decodes with
+// prmt and writes 64 bytes of bf16.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_dequantize_kernel(
+    const uint8_t* __restrict__ codes, const int8_t* __restrict__ q8,
+    const float* __restrict__ step2, const float* __restrict__ mean_ptr,
+    int64_t n_halves, uint16_t* __restrict__ out, Levels L) {
+  const float mu = *mean_ptr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_halves; i += stride) {
+    const int64_t b = i >> 1;
+    const uint4 cw = ld_stream_v4(codes + i * 16);
+    const float c_hat = block_scale(q8[b], step2[b / kGroup], mu);
+    const Nf4Table t = make_table(L, c_hat);
+    uint32_t o[4];
+    uint16_t* dst = out + i * 32;
+    decode8(t, cw.x, o); st_v4(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
+    decode8(t, cw.y, o); st_v4(dst + 8, make_uint4(o[0], o[1], o[2], o[3]));
+    decode8(t, cw.z, o); st_v4(dst + 16, make_uint4(o[0], o[1], o[2], o[3]));
+    decode8(t, cw.w, o); st_v4(dst + 24, make_uint4(o[0], o[1], o[2], o[3]));
+  }
+}
+
+}  // namespace qnf4

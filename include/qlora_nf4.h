@@ -1,0 +1,256 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA NF4 library.
+ *
+ * The library implements the hot path of QLoRA for one linear layer:
+ *
+ *   * the blockwise NF4 quantizer with double quantization that turns a frozen
+ *     fp32 weight W0 into 4-bit codes plus 8-bit second-level scale codes;
+ *   * dequantization of that format to bf16;
+ *   * the QLoRA linear forward  h = dequant(W0) x + (alpha/r) B A x
+ *     ("QLoRA", llm-compass, section 方法与公式, the displayed formula);
+ *   * its backward: dx through the frozen quantized base plus the LoRA branch,
+ *     and dA, dB for the adapters (same section, the sentence after the
+ *     formula: gradients only for B, A; W0 is never updated; "QLoRA",
+ *     aigrafen.se, opening paragraph: gradients flow through the quantized
+ *     base).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   Shapes use the PyTorch Linear convention: x [M, in], W0 [out, in],
+ *   A [r, in], B [out, r], h [M, out], s = alpha / r.  All matrices are dense
+ *   row-major with no padding between rows.
+ *   bf16 tensors are passed as uint16_t bit patterns.
+ *   Every pointer except the host arrays of qlora_nf4_codebook is a DEVICE
+ *   pointer on the current CUDA device and must be 16-byte aligned.
+ *   `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   All device work is enqueued on `stream` and the calls return without
+ *   synchronizing; outputs are valid once the stream reaches that point.
+ *   The caller owns every buffer, including the workspace; the library never
+ *   allocates device memory and keeps no per-call state.
+ *   Arguments are validated before anything is launched: a call that returns
+ *   a negative status has enqueued no work and written no output.
+ *
+ * NF4 storage format (qlora_nf4_weight)
+ * -------------------------------------
+ *   blocks    64 consecutive weights of a row ("QLoRA", llm-compass,
+ *             方法与公式 item 1: one scale per block of 64);
+ *             n_blocks = rows*cols/64, block b = row*(cols/64) + col/64.
+ *   codes     uint8 [rows, cols/2]; weight (row, 2i) in the low nibble of byte
+ *             (row, i), weight (row, 2i+1) in the high nibble.  Code j means
+ *             level j of qlora_nf4_codebook (ascending; level 7 is exactly 0).
+ *   q8        int8 [n_blocks], second-level code of each block's absmax.
+ *   step2     fp32 [ceil(n_blocks/256)], one step per group of 256 blocks.
+ *   mean      fp32 [1], mean of all block absmaxes.
+ *   The block scale is  c_hat = fp32(fp32(q8 * step2) + mean)  and a weight
+ *   is  bf16_rne(fp32(level[code] * c_hat))  (double quantization of the
+ *   block constants to 8 bit: llm-compass, 方法与公式 item 2; auryth glossary
+ *   "Hoe het werkt", item 2).
+ */
+#ifndef QLORA_NF4_H_
+#define QLORA_NF4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call. */
+enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = -1,      /* null or misaligned pointer, bad scalar      */
+  QLORA_ERR_UNSUPPORTED_SHAPE = -2,/* a size rule below is violated               */
+  QLORA_ERR_WORKSPACE = -3,        /* workspace missing or smaller than required  */
+  QLORA_ERR_CUDA = -4,             /* a CUDA runtime/driver call failed           */
+  QLORA_ERR_TIMEOUT = -5           /* a device-side wait gave up (see below)      */
+};
+
+/* Operation selector of qlora_workspace_size. */
+enum {
+  QLORA_OP_QUANTIZE = 0,
+  QLORA_OP_DEQUANTIZE = 1,
+  QLORA_OP_LINEAR_FWD = 2,
+  QLORA_OP_LINEAR_BWD = 3
+};
+
+/* A quantized weight: device pointers in the format described above. */
+typedef struct qlora_nf4_weight {
+  const uint8_t* codes;  /* [rows, cols/2]            */
+  const int8_t* q8;      /* [rows*cols/64]            */
+  const float* step2;    /* [ceil(rows*cols/64/256)]  */
+  const float* mean;     /* [1]                       */
+  int64_t rows;          /* out features              */
+  int64_t cols;          /* in features, multiple of 64 */
+} qlora_nf4_weight;
+
+/*
+ * qlora_nf4_codebook -- the 16 NF4 levels and 15 decision thresholds (host).
+ *
+ * NF4 places 16 levels at standard-normal quantiles with equal expected mass
+ * per bin, normalised to [-1, 1] ("QLoRA", llm-compass, 方法与公式 item 1;
+ * learn-interview-questions QLoRA page, section 2).  The exact construction
+ * (an exact zero, 8 positive and 7 negative levels): with
+ * delta = 1 - (1/32 + 1/30)/2, positive levels Phi^-1(delta - i(delta-1/2)/8),
+ * i = 0..7, negative levels -Phi^-1(delta - i(delta-1/2)/7), i = 0..6, and 0,
+ * all divided by Phi^-1(delta), rounded to fp32, ascending.
+ * thresholds[j] is the exact midpoint of levels j and j+1 rounded toward
+ * -infinity to fp32, so that for fp32 v: v > thresholds[j] <=> v lies above
+ * the midpoint (nearest level, ties to the lower index).
+ *
+ * levels: host array of 16 floats (written).  thresholds: host array of 15
+ * floats, or NULL.  Pure host computation, no CUDA call.
+ * Returns QLORA_OK, or QLORA_ERR_INVALID_ARG if levels is NULL.
+ */
+int qlora_nf4_codebook(float levels[16], float thresholds[15]);
+
+/*
+ * qlora_workspace_size -- bytes of device workspace a call needs.
+ *
+ * op is one of QLORA_OP_*.  Sizes are those the call will receive (for
+ * QLORA_OP_QUANTIZE and _DEQUANTIZE: rows = out_features, cols = in_features;
+ * M and r are ignored).  Returns 0 when the call needs no workspace, and
+ * (size_t)-1 for an unknown op or negative sizes.  The workspace must be
+ * 256-byte aligned; its contents on entry do not matter.
+ */
+size_t qlora_workspace_size(int op, int64_t M, int64_t in_features,
+                            int64_t out_features, int r);
+
+/*
+ * qlora_quantize_nf4 -- blockwise NF4 quantization with double quantization.
+ *
+ * Per block b of 64 weights: c_b = max|w| (exact); if c_b = 0 every code is 7;
+ * otherwise v = fp32(w * fp32(1/c_b)) and code = #{j : v > thresholds[j]}.
+ * Second level: mean = fp32(T / n_blocks) where T is the fp64 sum of all c_b
+ * in a fixed binary tree (zero-padded to a power of two, adjacent pairs added
+ * level by level) and the division is done in fp64; d_b = fp32(c_b - mean);
+ * per group g of 256 blocks step2_g = fp32(max|d_b| / 127);
+ * q8_b = clamp(round_half_even(fp32(d_b * fp32(1/step2_g))), -127, 127), or 0
+ * when step2_g = 0 or the product is NaN.  All fp32 operations are correctly
+ * rounded (no fused multiply-add), so the result is bit-reproducible.
+ * ("QLoRA", llm-compass, 方法与公式 items 1-2.)
+ *
+ * W       device fp32 [rows, cols], finite values.
+ * codes   device uint8 [rows, cols/2]      (written)
+ * q8      device int8 [rows*cols/64]       (written)
+ * step2   device fp32 [ceil(n_blocks/256)] (written)
+ * mean    device fp32 [1]                  (written)
+ * workspace / workspace_bytes: at least
+ *         qlora_workspace_size(QLORA_OP_QUANTIZE, 0, cols, rows, 0) bytes.
+ * Size rules: rows >= 1, cols >= 64, cols % 64 == 0.
+ */
+int qlora_quantize_nf4(const float* W, int64_t rows, int64_t cols,
+                       uint8_t* codes, int8_t* q8, float* step2, float* mean,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qlora_dequantize_nf4 -- NF4 weight to bf16, bit-exact with the formula in
+ * the format description above ("QLoRA", auryth glossary, "Hoe het werkt":
+ * dequantize NF4 on the fly per layer).
+ *
+ * w      quantized weight (device pointers), cols % 64 == 0.
+ * W_out  device bf16 [rows, cols] (written).
+ */
+int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream);
+
+/*
+ * qlora_linear_fwd -- QLoRA linear forward
+ *   h  = x dequant(W0)^T + us B^T,   us = bf16(s * x A^T),   s = alpha / r
+ * ("QLoRA", llm-compass, 方法与公式, displayed formula).  The dequantized
+ * weight is produced tile by tile inside the GEMM and never written to memory.
+ * M > 16 runs the fused tensor-core GEMM; M <= 16 a split-K streaming GEMV.
+ *
+ * x       device bf16 [M, in]
+ * w       quantized W0, rows = out, cols = in
+ * A       device bf16 [r, in];  B  device bf16 [out, r]
+ * h       device bf16 [M, out] (written)
+ * us_out  device bf16 [M, r] (written): the scaled LoRA activation, kept for
+ *         the backward.
+ * workspace: qlora_workspace_size(QLORA_OP_LINEAR_FWD, M, in, out, r) bytes.
+ * Size rules: M >= 1; in % 64 == 0; out % 64 == 0; r % 8 == 0, 8 <= r <= 256.
+ */
+int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w,
+                     const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* h, uint16_t* us_out,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qlora_linear_bwd -- QLoRA linear backward with W0 frozen.
+ *   du = bf16(s * dh B)                 [M, r]
+ *   dx = dh dequant(W0) + du A          [M, in]  (bf16 out)
+ *   dB = dh^T us                        [out, r] (fp32 out)
+ *   dA = du^T x                         [r, in]  (fp32 out)
+ * us is the us_out of the matching forward (us = bf16(s x A^T)), so
+ * dB = s dh^T x A^T and dA = s (dh B)^T x up to bf16 rounding of us and du.
+ * No gradient is formed for W0 ("QLoRA", llm-compass, 方法与公式: gradients
+ * only for B, A; aigrafen.se: gradients back-propagate through the quantized
+ * base, only the adapters are updated).
+ *
+ * dh, x, us, A, B: device bf16 as in the forward; dh [M, out].
+ * dx device bf16 [M, in]; dA device fp32 [r, in]; dB device fp32 [out, r]
+ * (all written, not accumulated).
+ * workspace: qlora_workspace_size(QLORA_OP_LINEAR_BWD, M, in, out, r) bytes.
+ * Size rules as for qlora_linear_fwd.
+ */
+int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us,
+                     int64_t M, const qlora_nf4_weight* w,
+                     const uint16_t* A, const uint16_t* B, int r, float alpha,
+                     uint16_t* dx, float* dA, float* dB,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qlora_last_device_status -- synchronizes `stream`, then reads and clears
+ * the current device's error flag.  Kernels that wait on another part of the
+ * device (pipeline barriers inside the GEMMs) give up after a bounded time
+ * (qlora_set_wait_timeout_ns), set the flag and return.  Returns QLORA_OK,
+ * QLORA_ERR_TIMEOUT when the flag was set, or QLORA_ERR_CUDA when the
+ * synchronization itself reports an error.
+ */
+int qlora_last_device_status(void* stream);
+
+/*
+ * qlora_set_wait_timeout_ns -- bound, in nanoseconds of %globaltimer, of every
+ * device-side wait launched after this call (process-wide; default 2e9 = 2 s).
+ * Values below 1000 are raised to 1000.  Returns the previous bound.
+ */
+uint64_t qlora_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * qlora_selftest_wait_timeout -- diagnostic: launches one kernel that waits on
+ * a pipeline barrier that nothing will ever complete, bounded by the current
+ * wait timeout, so that the timeout path (error flag set, kernel returns,
+ * context stays usable) can be exercised without faulting or hanging a GPU.
+ * Returns the status of qlora_last_device_status after the kernel
+ * (QLORA_ERR_TIMEOUT when the path works).
+ */
+int qlora_selftest_wait_timeout(void* stream);
+
+/*
+ * Per-kernel timing (diagnostics for benchmarks).  While enabled, every kernel
+ * the library launches is bracketed by two CUDA events recorded on the
+ * launching stream; qlora_timing_collect synchronizes on those events and
+ * returns, for one kernel name, the summed device time in milliseconds and
+ * the number of launches since the last reset.  Names: "quantize_blocks",
+ * "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
+ * "gemv", "gemv_finalize", "lora_rowwise", "lora_colwise", "sum_chunks",
+ * "transpose".  Events are created by the library on first use (host-side
+ * CUDA objects, no device memory).  Not for use during stream capture.
+ *
+ * qlora_timing_enable: on != 0 enables, 0 disables; returns the previous state.
+ * qlora_timing_reset: forgets all recorded launches.
+ * qlora_timing_collect: kernel name (NUL-terminated), outputs may be NULL.
+ *   Returns QLORA_OK, QLORA_ERR_INVALID_ARG for a NULL name, or
+ *   QLORA_ERR_CUDA if an event query fails.
+ */
+int qlora_timing_enable(int on);
+void qlora_timing_reset(void);
+int qlora_timing_collect(const char* kernel, double* total_ms, int64_t* launches);
+
+/* qlora_status_string -- static English description of a status code. */
+const char* qlora_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_NF4_H_ */

@@ -68,3 +68,12 @@ def linear_dx_rows(dh, W, A, B, alpha: float, rows):
     dh, W, A, B = _f64(dh)[np.asarray(rows)], _f64(W), _f64(A), _f64(B)
     s = float(alpha) / float(A.shape[0])
     return dh @ W + s * ((dh @ B) @ A)
+
+
+def lora_grads(dh, x, A, B, alpha: float):
+    """(dA, dB) alone, with the same arithmetic as :func:`linear_bwd`."""
+    dh, x, A, B = _f64(dh), _f64(x), _f64(A), _f64(B)
+    s = float(alpha) / float(A.shape[0])
+    g = dh @ B
+    u = x @ A.T
+    return s * (g.T @ x), s * (dh.T @ u)

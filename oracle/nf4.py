@@ -261,17 +261,39 @@ def dequant_scales(q8: np.ndarray, step2: np.ndarray, mean: float) -> np.ndarray
     return fl32(fl32(q8 * np.asarray(step2, dtype=np.float64)[g]) + mean)
 
 
-def dequantize_bits(codes: np.ndarray, q8, step2, mean) -> np.ndarray:
-    """bf16 bit patterns of the dequantized weight [rows, cols] (R6)."""
+def dequantize_bits(codes: np.ndarray, q8, step2, mean, blocks=None) -> np.ndarray:
+    """bf16 bit patterns of the dequantized weight [rows, cols] (R6).
+
+    ``blocks`` optionally gives the global block index of every 64-code block
+    of ``codes`` (row-major), for dequantizing a subset of a tensor's rows."""
     codes = np.asarray(codes, dtype=np.uint8)
     rows, cols = codes.shape
     c_hat = dequant_scales(q8, step2, mean)
+    if blocks is not None:
+        c_hat = c_hat[np.asarray(blocks)]
     levels = codebook()
     lv = levels[codes.reshape(-1, BLOCK)]                 # level[code]
     prod = fl32(lv * c_hat[:, None])                      # fl32(level * c_hat)
     return bf16_bits_from_f32(prod).reshape(rows, cols)
 
 
-def dequantize(codes: np.ndarray, q8, step2, mean) -> np.ndarray:
-    """Dequantized weight [rows, cols] as fp64 values of bf16 numbers."""
-    return bf16_to_f64(dequantize_bits(codes, q8, step2, mean))
+def dequantize(codes: np.ndarray, q8, step2, mean, blocks=None) -> np.ndarray:
+    """Dequantized weight [rows, cols] as fp64 values of bf16 numbers
+    (``blocks`` as in :func:`dequantize_bits`)."""
+    return bf16_to_f64(dequantize_bits(codes, q8, step2, mean, blocks))
+
+
+def quantize_rows(W: np.ndarray, rows) -> dict:
+    """First-level codes of the selected rows of W, with the second-level
+    statistics (q8, step2, mean) of the WHOLE tensor, since the mean and the
+    256-block groups span rows.  Identical to the corresponding rows of
+    :func:`quantize`; used to check large tensors on sampled rows."""
+    W = np.asarray(W, dtype=np.float32)
+    rows = np.asarray(rows)
+    c = block_absmax(W)
+    q8, step2, mean = double_quantize(c)
+    nbr = W.shape[1] // BLOCK
+    blocks = (rows[:, None] * nbr + np.arange(nbr)[None, :]).ravel()
+    codes = encode(W[rows].astype(np.float64), c[blocks])
+    return dict(codes=codes, packed=pack(codes), absmax=c, q8=q8, step2=step2,
+                mean=mean, blocks=blocks)

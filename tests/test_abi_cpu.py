@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the shared library loads, exports every
+function declared in include/qlora_nf4.h, computes the same NF4 codebook as
+the oracle bit for bit (a host-only call), sizes workspaces consistently, and
+rejects bad arguments with the documented status before launching anything.
+
+Only calls that return before any CUDA work are made here; the pointers
+passed are aligned dummies that are never dereferenced.
+"""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_nf4_quantized_11_b200 as q
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+OK, EINVAL, ESHAPE, EWS, ECUDA, ETIMEOUT = 0, -1, -2, -3, -4, -5
+FAKE = 1 << 20          # 16- and 256-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_nf4_quantized_11_b200 import build
+    build.build()
+    return q.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_codebook_equals_oracle_bit_for_bit(lib):
+    lv, th = q.codebook()
+    assert np.array_equal(np.array(lv, dtype=np.float32).view(np.uint32), nf4.f32_bits(nf4.codebook()))
+    assert np.array_equal(np.array(th, dtype=np.float32).view(np.uint32), nf4.f32_bits(nf4.thresholds()))
+
+
+def test_codebook_null_levels_rejected(lib):
+    assert lib.qlora_nf4_codebook(None, None) == EINVAL
+
+
+def test_status_strings(lib):
+    for s in (OK, EINVAL, ESHAPE, EWS, ECUDA, ETIMEOUT):
+        assert len(q.status_string(s)) >= 2
+    assert q.status_string(12345) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    # quantize: absmax fp32 per block + fp64 tree partials
+    n = q.workspace_size(q.OP_QUANTIZE, 0, 4096, 4096, 0)
+    assert n >= 4096 * 4096 // 64 * 4
+    assert q.workspace_size(q.OP_DEQUANTIZE, 0, 512, 512, 0) == 0
+    assert q.workspace_size(q.OP_LINEAR_FWD, 4096, 4096, 4096, 16) == 0     # fused GEMM path
+    assert q.workspace_size(q.OP_LINEAR_FWD, 4, 8192, 28672, 16) > 0        # split-K GEMV partials
+    nb = q.workspace_size(q.OP_LINEAR_BWD, 4096, 4096, 4096, 16)
+    assert nb >= 4096 * 16 * 2
+    assert lib.qlora_workspace_size(99, 1, 64, 64, 8) == ctypes.c_size_t(-1).value
+    assert lib.qlora_workspace_size(q.OP_LINEAR_FWD, -1, 64, 64, 8) == ctypes.c_size_t(-1).value
+
+
+def _weight(rows=64, cols=64, codes=FAKE):
+    return q._Weight(codes, FAKE, FAKE, FAKE, rows, cols)
+
+
+def test_quantize_argument_errors(lib):
+    ws = q.workspace_size(q.OP_QUANTIZE, 0, 128, 64, 0)
+    f = lib.qlora_quantize_nf4
+    assert f(None, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == EINVAL
+    assert f(FAKE + 4, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == EINVAL      # misaligned W
+    assert f(FAKE, 64, 100, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == ESHAPE         # cols % 64
+    assert f(FAKE, 0, 128, FAKE, FAKE, FAKE, FAKE, FAKE, ws, None) == ESHAPE          # rows < 1
+    assert f(FAKE, 64, 128, FAKE, FAKE, FAKE, FAKE, None, ws, None) == EWS            # no workspace
+    assert f(FAKE, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE, ws - 1, None) == EWS        # too small
+    assert f(FAKE, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE + 16, ws, None) == EWS       # misaligned ws
+
+
+def test_dequantize_argument_errors(lib):
+    f = lib.qlora_dequantize_nf4
+    assert f(None, FAKE, None) == EINVAL
+    w = _weight(codes=0)
+    assert f(ctypes.byref(w), FAKE, None) == EINVAL
+    w = _weight(cols=96)
+    assert f(ctypes.byref(w), FAKE, None) == ESHAPE
+    w = _weight()
+    assert f(ctypes.byref(w), FAKE + 2, None) == EINVAL
+
+
+def test_linear_argument_errors(lib):
+    fwd, bwd = lib.qlora_linear_fwd, lib.qlora_linear_bwd
+    w = _weight(128, 128)
+    wb = ctypes.byref(w)
+    # null / misaligned pointers
+    assert fwd(None, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == EINVAL
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE + 8, None, 0, None) == EINVAL
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, float("nan"), FAKE, FAKE, None, 0, None) == EINVAL
+    # shape rules: r multiple of 8 in [8, 256], M >= 1, in/out multiples of 64
+    for r in (0, 4, 12, 264):
+        assert fwd(FAKE, 64, wb, FAKE, FAKE, r, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
+    assert fwd(FAKE, 0, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
+    w2 = _weight(96, 128)
+    assert fwd(FAKE, 64, ctypes.byref(w2), FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
+    # GEMV path needs a workspace
+    assert fwd(FAKE, 4, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == EWS
+    # backward always needs one
+    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, FAKE, None, 0, None) == EWS
+    assert bwd(FAKE, FAKE, None, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == EINVAL
+    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 9, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ESHAPE
+
+
+def test_timeout_setter_roundtrip(lib):
+    prev = q.set_wait_timeout_ns(5_000_000)
+    assert q.set_wait_timeout_ns(prev) == 5_000_000
+    assert q.set_wait_timeout_ns(10) >= 1000      # previous value returned
+    assert q.set_wait_timeout_ns(prev) == 1000     # clamped to the 1 us minimum
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    monkeypatch.setattr(q, "_LIB", None)
+    monkeypatch.setattr(q, "library_path", lambda: str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        q.load()
+    importlib.reload(q)

@@ -1,0 +1,98 @@
+"""GPU parity of the NF4 quantizer and dequantizer against the oracle:
+bit-exact packed codes, second-level int8 codes, steps, mean and bf16
+dequantized weights, on seeded synthetic weights and on the degenerate cases
+(zero blocks, equal-absmax blocks, signed zeros, subnormals, a partial last
+scale group, multi-pass summation trees), through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_11_b200 import synth
+from oracle import nf4
+from parity import bf16_bits, f32_bits
+
+pytestmark = [pytest.mark.gpu, pytest.mark.filterwarnings("ignore::RuntimeWarning")]
+
+
+def _check_quant(q, W_cpu, sample_rows=None):
+    """Quantize on the GPU and compare every stored array with the oracle.
+    With sample_rows, the first-level codes and dequantized weights are
+    compared on those rows only (the scale statistics are still global)."""
+    Wn = W_cpu.numpy()
+    w = q.quantize_nf4(W_cpu.cuda())
+    deq = q.dequantize_nf4(w)
+    assert q.last_device_status() == 0
+    c = nf4.block_absmax(Wn)
+    q8, step2, mean = nf4.double_quantize(c)
+    assert f32_bits(w.mean)[0] == nf4.f32_bits(mean)
+    assert np.array_equal(f32_bits(w.step2), nf4.f32_bits(step2))
+    assert np.array_equal(w.q8.cpu().numpy(), q8)
+    rows = np.arange(Wn.shape[0]) if sample_rows is None else np.asarray(sample_rows)
+    nbr = Wn.shape[1] // 64
+    blk = (rows[:, None] * nbr + np.arange(nbr)[None, :]).ravel()
+    codes = nf4.encode(Wn[rows], c[blk])
+    assert np.array_equal(w.codes.cpu().numpy()[rows], nf4.pack(codes))
+    assert np.array_equal(bf16_bits(deq)[rows], nf4.dequantize_bits(codes, q8, step2, mean, blocks=blk))
+    return w
+
+
+@pytest.mark.parametrize("rows,cols,dist,std,seed", [
+    (1, 64, "normal", 0.02, 0),          # one block
+    (64, 64, "normal", 0.02, 1),
+    (300, 640, "normal", 0.02, 2),       # 3000 blocks: partial last group (3000 % 256 = 184)
+    (512, 512, "normal", 0.02, 0),       # the small parity layer
+    (257, 1088, "student_t5", 0.02, 3),  # heavy tails, odd row count
+    (1024, 1024, "normal", 0.015, 4),    # 16384 blocks: two-pass summation tree
+])
+def test_quantize_bit_exact(cuda_lib, rows, cols, dist, std, seed):
+    _check_quant(cuda_lib, synth.weight(rows, cols, std, dist, seed))
+
+
+def test_degenerate_blocks_bit_exact(cuda_lib):
+    W = synth.weight(64, 512, 0.02, "normal", 7).numpy().copy()
+    W[0, :64] = 0.0                                  # all-zero block
+    W[1, :] = -0.0                                   # a row of negative zeros
+    W[2, 64:128] = np.float32(1e-40)                 # subnormal block
+    W[3, 128:192] = np.linspace(-1e-38, 1e-38, 64, dtype=np.float32)
+    W[4, :64] = 1e4 * np.sign(W[4, :64])             # large magnitude
+    W[5, 3] = -0.0
+    w = _check_quant(cuda_lib, torch.from_numpy(W))
+    codes = w.codes.cpu().numpy()
+    assert np.all(codes[0, :32] == 0x77) and np.all(codes[1] == 0x77)
+
+
+def test_equal_absmax_gives_zero_second_level(cuda_lib):
+    rng = np.random.default_rng(3)
+    W = rng.uniform(-0.5, 0.5, (16, 1024)).astype(np.float32)
+    W[:, ::64] = 0.5
+    w = _check_quant(cuda_lib, torch.from_numpy(W))
+    assert torch.all(w.q8 == 0) and torch.all(w.step2 == 0)
+    assert w.mean.item() == 0.5
+
+
+@pytest.mark.parametrize("shape,dist,std", [
+    ((4096, 4096), "normal", 0.02),        # 7B attention projection, full tensor
+    ((11008, 4096), "student_t5", 0.02),   # 7B MLP gate/up, full tensor
+])
+def test_quantize_full_size_bit_exact(cuda_lib, shape, dist, std):
+    _check_quant(cuda_lib, synth.weight(shape[0], shape[1], std, dist, 0))
+
+
+@pytest.mark.parametrize("shape,std", [((28672, 8192), 0.015), ((8192, 22016), 0.01)])
+def test_quantize_70b_65b_shapes_sampled_rows(cuda_lib, shape, std):
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(shape[0], 48, replace=False))
+    rows[0], rows[-1] = 0, shape[0] - 1
+    _check_quant(cuda_lib, synth.weight(shape[0], shape[1], std, "normal", 0), sample_rows=rows)
+
+
+def test_dequantize_matches_codebook_levels_exactly(cuda_lib):
+    """A block whose values are exactly c * level[j] reproduces its codes."""
+    lv, _ = cuda_lib.codebook()
+    c = np.float32(0.0371)
+    w = (c * np.array(lv, dtype=np.float32)).astype(np.float32)
+    W = np.tile(w, 8).reshape(2, 64)
+    qw = cuda_lib.quantize_nf4(torch.from_numpy(W).cuda())
+    codes = nf4.unpack(qw.codes.cpu().numpy())
+    assert np.array_equal(codes, np.tile(np.arange(16, dtype=np.uint8), 8).reshape(2, 64))

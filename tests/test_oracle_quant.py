@@ -230,3 +230,16 @@ def test_stored_bytes_match_oracle_arrays():
     assert nbytes == overhead.stored_bytes(*W.shape)
     bits = 8.0 * nbytes / W.size
     assert abs(bits - overhead.bits_per_param(n_params=W.size)) < 1e-12
+
+
+def test_quantize_rows_equals_full_quantize_rows():
+    rng = np.random.default_rng(10)
+    W = (rng.standard_normal((40, 640)) * 0.02).astype(np.float32)   # 400 blocks, 2 groups
+    full = nf4.quantize(W)
+    rows = np.array([0, 7, 39])
+    sub = nf4.quantize_rows(W, rows)
+    assert np.array_equal(sub["codes"], full["codes"][rows])
+    assert np.array_equal(sub["q8"], full["q8"]) and sub["mean"] == full["mean"]
+    d_full = nf4.dequantize(full["codes"], full["q8"], full["step2"], full["mean"])
+    d_sub = nf4.dequantize(sub["codes"], sub["q8"], sub["step2"], sub["mean"], blocks=sub["blocks"])
+    assert np.array_equal(d_sub, d_full[rows])
