@@ -52,6 +52,7 @@ def parse():
     ap.add_argument("--rotations", type=int, default=4)
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
 
 
@@ -260,7 +261,7 @@ def run_ours(args, world, rank, local):
                 "flops_per_launch": dom_flops,
                 "traffic": profiled_traffic(dom, WL.name)}
 
-    e2e = measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev)
+    e2e = None if args.no_e2e else measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev)
 
     rot_bytes = args.rotations * (2 * M * n_in + 2 * M * n_out + copies[0]["w"].nbytes())
     line = {
