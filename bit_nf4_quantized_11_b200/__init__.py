@@ -26,7 +26,8 @@ from dataclasses import dataclass
 import torch
 
 __all__ = [
-    "load", "library_path", "codebook", "NF4Weight", "quantize_nf4", "dequantize_nf4",
+    "load", "library_path", "codebook", "NF4Weight", "quantize_nf4", "quantize_nf4_noalloc",
+    "dequantize_nf4", "alloc_nf4",
     "linear_fwd", "linear_bwd", "workspace_size", "last_device_status",
     "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
     "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES",
@@ -35,7 +36,8 @@ __all__ = [
 
 OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
 STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTED_SHAPE",
-          -3: "QLORA_ERR_WORKSPACE", -4: "QLORA_ERR_CUDA", -5: "QLORA_ERR_TIMEOUT"}
+          -3: "QLORA_ERR_WORKSPACE", -4: "QLORA_ERR_CUDA", -5: "QLORA_ERR_TIMEOUT",
+          -6: "QLORA_ERR_SCRATCH_LIMIT"}
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -80,6 +82,7 @@ def load():
         "qlora_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
         "qlora_selftest_wait_timeout": (I, [P]),
         "qlora_status_string": (ctypes.c_char_p, [I]),
+        "qlora_quantize_nf4_noalloc": (I, [P, I64, I64, P, P, P, P, P]),
         "qlora_timing_enable": (I, [I]),
         "qlora_timing_reset": (None, []),
         "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -182,6 +185,18 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, workspace=None) 
     _check(load().qlora_quantize_nf4(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2),
                                      _ptr(w.mean), _ptr(ws), ws.numel() if ws is not None else 0,
                                      _stream()), "qlora_quantize_nf4")
+    return w
+
+
+def quantize_nf4_noalloc(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
+    """As quantize_nf4, but the library uses its own fixed device scratch
+    (at most 2**22 blocks of 64 weights) instead of a caller workspace."""
+    _need(W, torch.float32, "W")
+    rows, cols = W.shape
+    w = out if out is not None else alloc_nf4(rows, cols, W.device)
+    _check(load().qlora_quantize_nf4_noalloc(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8),
+                                             _ptr(w.step2), _ptr(w.mean), _stream()),
+           "qlora_quantize_nf4_noalloc")
     return w
 
 

@@ -555,8 +555,58 @@ const char* qlora_status_string(int status) {
     case QLORA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_TIMEOUT: return "a device-side wait timed out";
+    case QLORA_ERR_SCRATCH_LIMIT: return "size exceeds the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
 
 }  // extern "C"
+
+// ============================================================================
+// No-allocation quantizer: the scratch of qlora_quantize_nf4 in a fixed
+// device array of this library instead of a caller workspace.
+namespace {
+
+constexpr int64_t kNoAllocMaxBlocks = QLORA_NOALLOC_MAX_BLOCKS;
+constexpr size_t kNoAllocScratchBytes =
+    ((static_cast<size_t>(kNoAllocMaxBlocks) * 4 + 255) & ~static_cast<size_t>(255)) +
+    ((static_cast<size_t>(kNoAllocMaxBlocks / qnf4::kTreeChunk + 1) * 8 + 255) & ~static_cast<size_t>(255));
+
+// One copy per device that loads the library.  In host code this name is a
+// host-side stand-in, never a device address: the address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current).
+void* noalloc_scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int qlora_quantize_nf4_noalloc(const float* W, int64_t rows, int64_t cols, uint8_t* codes,
+                                          int8_t* q8, float* step2, float* mean, void* stream) {
+  if (!W || !codes || !q8 || !step2 || !mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(q8, 16) || !aligned(step2, 16) || !aligned(mean, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 64 || cols % 64 != 0 || rows * cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (rows * cols / 64 > kNoAllocMaxBlocks) return QLORA_ERR_SCRATCH_LIMIT;
+  if (quant_ws(rows, cols).total > kNoAllocScratchBytes) return QLORA_ERR_SCRATCH_LIMIT;
+  void* scratch = noalloc_scratch_for_current_device();
+  if (scratch == nullptr) return QLORA_ERR_CUDA;
+  return launch_quantize(W, rows, cols, codes, q8, step2, mean, scratch, static_cast<cudaStream_t>(stream));
+}
+

@@ -63,7 +63,9 @@ enum {
   QLORA_ERR_UNSUPPORTED_SHAPE = -2,/* a size rule below is violated               */
   QLORA_ERR_WORKSPACE = -3,        /* workspace missing or smaller than required  */
   QLORA_ERR_CUDA = -4,             /* a CUDA runtime/driver call failed           */
-  QLORA_ERR_TIMEOUT = -5           /* a device-side wait gave up (see below)      */
+  QLORA_ERR_TIMEOUT = -5,          /* a device-side wait gave up (see below)      */
+  QLORA_ERR_SCRATCH_LIMIT = -6     /* size beyond the built-in scratch of a
+                                      no-allocation entry point               */
 };
 
 /* Operation selector of qlora_workspace_size. */
@@ -245,6 +247,39 @@ int qlora_selftest_wait_timeout(void* stream);
 int qlora_timing_enable(int on);
 void qlora_timing_reset(void);
 int qlora_timing_collect(const char* kernel, double* total_ms, int64_t* launches);
+
+/*
+ * qlora_quantize_nf4_noalloc -- qlora_quantize_nf4 without a caller workspace.
+ *
+ * The pages describe no such variant; it exists for callers that cannot
+ * obtain device memory at the moment they quantize: a host that forbids
+ * cudaMalloc after start-up (an allocation can synchronize the device and
+ * break a memory budget planned in advance), or a plugin that has no access
+ * to its host framework's allocator and so cannot size and pass the
+ * workspace that qlora_quantize_nf4 needs.  It computes exactly what
+ * qlora_quantize_nf4 computes (same kernels, bit-identical outputs); its
+ * scratch (block absmaxes and the partial sums of the scale-mean tree) lives
+ * in a fixed device array inside the library, QLORA_NOALLOC_MAX_BLOCKS blocks
+ * of 64 weights large (16 MiB + 8 KiB), which every GPU that loads the
+ * library holds until the process exits.  The call itself allocates nothing.
+ *
+ * The first call on a device looks up that array's device address (once per
+ * device, with the device current); make that first call before any stream
+ * capture begins.  Every call shares the one array: calls that can overlap on
+ * the GPU (different streams, or different host threads) race on it and must
+ * be ordered by the caller.  The array keeps the previous call's contents;
+ * each call overwrites every scratch value before reading it, so nothing has
+ * to start at zero.
+ *
+ * Arguments and size rules as qlora_quantize_nf4, without the workspace.
+ * Returns QLORA_ERR_SCRATCH_LIMIT (nothing launched) when
+ * rows*cols/64 > QLORA_NOALLOC_MAX_BLOCKS, QLORA_ERR_CUDA if the address
+ * lookup fails.
+ */
+#define QLORA_NOALLOC_MAX_BLOCKS (1LL << 22)
+int qlora_quantize_nf4_noalloc(const float* W, int64_t rows, int64_t cols,
+                               uint8_t* codes, int8_t* q8, float* step2, float* mean,
+                               void* stream);
 
 /* qlora_status_string -- static English description of a status code. */
 const char* qlora_status_string(int status);
