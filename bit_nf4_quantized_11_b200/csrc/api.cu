@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_pair_sm100.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
 #include "skinny.cuh"
@@ -170,16 +171,32 @@ GemvPlan gemv_plan(int64_t in, int64_t out) {
   return {static_cast<int>(splits), static_cast<int>(bps)};
 }
 
-size_t fwd_ws(int64_t M, int64_t in, int64_t out) {
+// K splits of the row-wise rank-r product: only when there are too few
+// 16-row tiles to fill the GPU (few-token calls); each split keeps at least
+// one 32-wide chunk per warp.
+int rowwise_splits(int64_t M, int64_t K) {
+  const int64_t row_tiles = cdiv(M, 16);
+  if (row_tiles >= 128) return 1;
+  const int64_t max_splits = std::max<int64_t>(1, K / 32 / 8);
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, cdiv(2 * device_sm_count(), row_tiles))));
+}
+
+size_t rowwise_ws(int64_t M, int64_t K, int r) {
+  const int ks = rowwise_splits(M, K);
+  return ks > 1 ? round256(static_cast<size_t>(ks) * M * r * 4) : 0;
+}
+
+size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
+  size_t b = rowwise_ws(M, in, r);
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
-    return round256(static_cast<size_t>(p.splits) * 16 * out * 4);
+    b += round256(static_cast<size_t>(p.splits) * 16 * out * 4);
   }
-  return 0;
+  return b;
 }
 
 struct BwdWs {
-  size_t du_off, bt_off, dbp_off, dap_off, total;
+  size_t du_off, row_off, dbp_off, dap_off, total;
   int chunks;
 };
 
@@ -187,8 +204,8 @@ BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
   BwdWs w{};
   w.chunks = static_cast<int>(cdiv(M, qnf4::kColChunk));
   w.du_off = 0;
-  w.bt_off = w.du_off + round256(static_cast<size_t>(M) * r * 2);
-  w.dbp_off = w.bt_off + round256(static_cast<size_t>(r) * out * 2);
+  w.row_off = w.du_off + round256(static_cast<size_t>(M) * r * 2);
+  w.dbp_off = w.row_off + rowwise_ws(M, out, r);
   w.dap_off = w.dbp_off + round256(static_cast<size_t>(w.chunks) * out * r * 4);
   w.total = w.dap_off + round256(static_cast<size_t>(w.chunks) * in * r * 4);
   return w;
@@ -250,8 +267,9 @@ int gemm_tile_m(int64_t M) {
     const char* e = std::getenv("QLORA_NF4_GEMM_TILE_M");
     return e ? std::atoi(e) : 0;
   }();
-  if (forced == 128 || forced == 256) return forced;
-  return M >= 1024 ? 256 : 128;
+  if (forced == 128 || forced == 256 || forced == 512) return forced;
+  if (M > 384) return 512;       // CTA-pair tile (cta_group::2)
+  return M > 128 ? 256 : 128;
 }
 
 template <int MS, bool kDx, int kStages>
@@ -264,6 +282,21 @@ int launch_gemm_t(const qnf4::GemmArgs& args, const CUtensorMap& tm_act, const C
   {
     LaunchTimer lt_(kDx ? "gemm_dx" : "gemm_fwd", st);
     kern<<<static_cast<unsigned>(tiles), Cfg::THREADS, Cfg::SMEM, st>>>(tm_act, tm_lora, args);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+template <bool kDx>
+int launch_gemm_pair(const qnf4::GemmArgs& args, const CUtensorMap& tm_act, const CUtensorMap& tm_lora,
+                     cudaStream_t st) {
+  using Cfg = qnf4::PairCfg;
+  auto kern = qnf4::qlora_gemm_pair_kernel<kDx>;
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+  const int64_t pairs = cdiv(args.M, Cfg::BM) * cdiv(args.N, Cfg::BN);
+  {
+    LaunchTimer lt_(kDx ? "gemm_dx" : "gemm_fwd", st);
+    kern<<<static_cast<unsigned>(2 * pairs), Cfg::THREADS, Cfg::SMEM, st>>>(tm_act, tm_lora, args);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
@@ -291,6 +324,7 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
   a.L = tables().L;
   a.timeout_ns = g_timeout_ns.load();
   const int tm = gemm_tile_m(M);
+  if (tm == 512) return dx ? launch_gemm_pair<true>(a, tm_act, tm_lora, st) : launch_gemm_pair<false>(a, tm_act, tm_lora, st);
   if (!dx) {
     return tm == 256 ? launch_gemm_t<2, false, 3>(a, tm_act, tm_lora, st)
                      : launch_gemm_t<1, false, 4>(a, tm_act, tm_lora, st);
@@ -299,32 +333,59 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
                    : launch_gemm_t<1, true, 4>(a, tm_act, tm_lora, st);
 }
 
-int launch_rowwise(const uint16_t* act, const uint16_t* Wt, uint16_t* out, int64_t M, int64_t K, int R,
-                   float scale, cudaStream_t st) {
+template <int NT, bool kKR>
+int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int ks, int64_t M,
+                     int64_t K, int R, float scale, cudaStream_t st) {
+  const int n_chunks = static_cast<int>(K / 32);
+  const int cps = static_cast<int>(cdiv(n_chunks, ks));
+  dim3 grid(static_cast<unsigned>(cdiv(M, 16)), static_cast<unsigned>(ks));
   {
     LaunchTimer lt_("lora_rowwise", st);
-    qnf4::rowwise_skinny_kernel<<<static_cast<unsigned>(cdiv(M, 16)), qnf4::kRowThreads, 0, st>>>(
-      act, Wt, out, static_cast<int>(M), static_cast<int>(K), R, scale);
+    qnf4::rowwise_skinny_kernel<NT, kKR><<<grid, qnf4::kRowThreads, 0, st>>>(
+        act, W, out, ks > 1 ? part : nullptr, static_cast<int>(M), static_cast<int>(K), R, scale, cps);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  if (ks > 1) {
+    LaunchTimer lt_("lora_rowwise_finalize", st);
+    qnf4::rowwise_finalize_kernel<<<static_cast<unsigned>(cdiv(M * R, 256)), 256, 0, st>>>(
+        part, ks, static_cast<int>(M), R, scale, out);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
 }
 
-int launch_colwise_sum(const uint16_t* act, const uint16_t* u, float* part, int64_t M, int64_t P, int R,
-                       float* out, bool transpose, cudaStream_t st) {
-  const int chunks = static_cast<int>(cdiv(M, qnf4::kColChunk));
-  dim3 grid(static_cast<unsigned>(cdiv(P, 128)), static_cast<unsigned>(chunks));
+// out[M, R] = bf16(scale * act[M, K] . W^T) with W given as [R, K] (kKR =
+// false) or as [K, R] (kKR = true); part: fp32 workspace of rowwise_ws bytes.
+template <bool kKR>
+int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int64_t M, int64_t K,
+                   int R, float scale, cudaStream_t st) {
+  const int ks = rowwise_splits(M, K);
+  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, part, ks, M, K, R, scale, st);
+  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, part, ks, M, K, R, scale, st);
+  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, part, ks, M, K, R, scale, st);
+  return launch_rowwise_t<8, kKR>(act, W, out, part, ks, M, K, R, scale, st);
+}
+
+// dB = dh^T us -> [out, r] and dA = du^T x -> [r, in], one launch each for the
+// partials and for the fixed-order chunk sum.
+int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
+                      int64_t in, int64_t out, int R, float* dBp, float* dAp, int chunks, float* dB, float* dA,
+                      cudaStream_t st) {
+  const qnf4::ColProblem pb{dh, us, dBp, static_cast<int>(out), 0};
+  const qnf4::ColProblem pa{x, du, dAp, static_cast<int>(in), 1};
+  const int smem = qnf4::kColStages * qnf4::kColStageBytes;
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::colwise_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  dim3 grid(static_cast<unsigned>(cdiv(std::max(in, out), 128)), static_cast<unsigned>(chunks), 2);
   {
     LaunchTimer lt_("lora_colwise", st);
-    qnf4::colwise_skinny_kernel<<<grid, qnf4::kColThreads, 0, st>>>(act, u, part, static_cast<int>(M),
-                                                                  static_cast<int>(P), R);
+    qnf4::colwise_skinny_kernel<<<grid, qnf4::kColThreads, smem, st>>>(pb, pa, static_cast<int>(M), R);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
-  const int64_t n_el = P * R;
-  const int grid2 = static_cast<int>(std::min<int64_t>(cdiv(n_el, 256), 4096));
+  const int64_t n_b = out * R, n_a = in * R;
+  dim3 g2(static_cast<unsigned>(std::min<int64_t>(cdiv(std::max(n_a, n_b) / 4, 256), 1024)), 2);
   {
     LaunchTimer lt_("sum_chunks", st);
-    qnf4::sum_chunks_kernel<<<grid2, 256, 0, st>>>(part, chunks, static_cast<int>(P), R, out, transpose ? 1 : 0);
+    qnf4::sum_chunks_kernel<<<g2, 256, 0, st>>>(dBp, dB, n_b, dAp, dA, n_a, chunks);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
@@ -369,7 +430,7 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t in_features, int64_t out_
       return 0;
     case QLORA_OP_LINEAR_FWD:
       if (M < 1) return 0;
-      return fwd_ws(M, in_features, out_features);
+      return fwd_ws(M, in_features, out_features, r);
     case QLORA_OP_LINEAR_BWD:
       if (M < 1 || r < 1) return 0;
       return bwd_ws(M, in_features, out_features, r).total;
@@ -415,13 +476,14 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   const int sc = check_linear_shapes(M, w, r);
   if (sc != QLORA_OK) return sc;
   const int64_t in = w->cols, out = w->rows;
-  const size_t need = fwd_ws(M, in, out);
+  const size_t need = fwd_ws(M, in, out, r);
   if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
     return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float s = alpha / static_cast<float>(r);
 
-  int rc = launch_rowwise(x, A, us_out, M, in, r, s, st);           // us = bf16(s x A^T)
+  float* row_part = static_cast<float*>(workspace);
+  int rc = launch_rowwise<false>(x, A, us_out, row_part, M, in, r, s, st);   // us = bf16(s x A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
@@ -431,7 +493,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
     g.step2 = w->step2;
     g.mean = w->mean;
     g.x = x;
-    g.part = static_cast<float*>(workspace);
+    g.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rowwise_ws(M, in, r));
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
@@ -474,24 +536,16 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
-  uint16_t* Bt = reinterpret_cast<uint16_t*>(base + ws.bt_off);
+  float* row_part = reinterpret_cast<float*>(base + ws.row_off);
   float* dBp = reinterpret_cast<float*>(base + ws.dbp_off);
   float* dAp = reinterpret_cast<float*>(base + ws.dap_off);
   const float s = alpha / static_cast<float>(r);
 
-  dim3 tg(static_cast<unsigned>(cdiv(r, 32)), static_cast<unsigned>(cdiv(out, 32)));
-  {
-    LaunchTimer lt_("transpose", st);
-    qnf4::transpose_bf16_kernel<<<tg, 256, 0, st>>>(B, static_cast<int>(out), r, Bt);     // B^T [r, out]
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  int rc = launch_rowwise(dh, Bt, du, M, out, r, s, st);                             // du = bf16(s dh B)
+  int rc = launch_rowwise<true>(dh, B, du, row_part, M, out, r, s, st);               // du = bf16(s dh B)
   if (rc != QLORA_OK) return rc;
   rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
   if (rc != QLORA_OK) return rc;
-  rc = launch_colwise_sum(dh, us, dBp, M, out, r, dB, false, st);                     // dB = dh^T us
-  if (rc != QLORA_OK) return rc;
-  return launch_colwise_sum(x, du, dAp, M, in, r, dA, true, st);                      // dA = du^T x
+  return launch_lora_grads(dh, us, x, du, M, in, out, r, dBp, dAp, ws.chunks, dB, dA, st);  // dB, dA
 }
 
 int qlora_last_device_status(void* stream) {

@@ -11,7 +11,7 @@
 // glossary page: NF4 -> 16-bit per layer, on the fly).  The LoRA branch is the
 // extra rank-r K-slice appended after the main K loop.
 //
-// Tiling (per CTA, one output tile, 320 threads):
+// Tiling (per CTA, one output tile, 576 threads):
 //   BM = 128*MS token rows (A operand: x or dh, TMA-loaded, 128B swizzle)
 //   BN = 256 output columns (B operand: dequantized W0 written to shared
 //        memory by 8 dequant warps, in the UMMA 128B-swizzled layout;
@@ -22,7 +22,9 @@
 //   fp32 accumulators in TMEM (MS x 256 columns), UMMA 128x256x16 issued by
 //   one thread, kStages-deep shared-memory ring with mbarriers.
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + UMMA issuer,
-// warps 2..9 dequant producers and then the epilogue (TMEM -> bf16 -> HBM).
+// warps 2..17 dequant producers in two groups of 8 that take alternate
+// stages (so each thread has two stages of time to hide its global loads),
+// then all 16 run the epilogue (TMEM -> bf16 -> HBM).
 //
 // Every mbarrier wait is bounded: after the timeout the CTA sets the device
 // error flag, stops waiting, lets every role run to the end of its fixed trip
@@ -61,7 +63,7 @@ struct GemmCfg {
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = RING + BAR_BYTES + 1024;       // + alignment slack
   static constexpr uint32_t TMEM_COLS = MS * 256;            // 256 or 512
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 576;                         // 2 + 16 warps
 };
 
 // Bounded wait shared by all roles of a CTA; after the first timeout every
@@ -76,7 +78,7 @@ __device__ __forceinline__ void pipe_wait(uint64_t* bar, uint32_t parity, uint64
 }
 
 template <int MS, bool kDx, int kStages>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
 qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
                   const __grid_constant__ CUtensorMap tm_lora,
                   const GemmArgs args) {
@@ -180,7 +182,8 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     }
   } else {
     // -------------------------------------------------- dequant producers
-    const int t = threadIdx.x - 64;                       // 0..255
+    const int group = (warp - 2) >> 3;                    // stages it = group, group+2, ...
+    const int t = (threadIdx.x - 64) & 255;               // 0..255 within the group
     const int64_t w_row_bytes = args.w_cols / 2;
     const int64_t w_row_blocks = args.w_cols / 64;
     const float mu = __ldg(args.mean);
@@ -217,25 +220,31 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       lora_row = k;
     }
 
-    auto load_codes = [&](int it, uint4& c0, uint4& c1, int& qv) {
+    // everything one stage needs from global memory, loaded ahead of use
+    struct StageIn {
+      uint4 c0, c1;
+      int q;
+      float st;
+    };
+    auto load_stage = [&](int it, StageIn& d) {
       if (col_valid && it < n_main) {
         const uint8_t* p = code_ptr + it * code_step;
-        c0 = ld_nc_v4(p);
-        c1 = ld_nc_v4(p + 16);
-        qv = __ldg(args.q8 + q8_idx + it * q8_step);
+        const int64_t blk = q8_idx + it * q8_step;
+        d.c0 = ld_nc_v4(p);
+        d.c1 = ld_nc_v4(p + 16);
+        d.q = __ldg(args.q8 + blk);
+        d.st = __ldg(args.step2 + blk / 256);
       }
     };
 
-    uint4 ca0 = make_uint4(0, 0, 0, 0), ca1 = ca0, cb0 = ca0, cb1 = ca0;
-    int qa = 0, qb = 0;
-    load_codes(0, ca0, ca1, qa);
-    load_codes(1, cb0, cb1, qb);
+    StageIn na{}, nb{};
+    load_stage(group, na);
+    load_stage(group + 2, nb);
 
-    for (int it = 0; it < n_iter; ++it) {
-      const uint4 c0 = ca0, c1 = ca1;
-      const int qc = qa;
-      ca0 = cb0; ca1 = cb1; qa = qb;
-      load_codes(it + 2, cb0, cb1, qb);
+    for (int it = group; it < n_iter; it += 2) {
+      const StageIn cur = na;
+      na = nb;
+      load_stage(it + 4, nb);
 
       const int s = it % kStages;
       const uint32_t ph = (it / kStages) & 1u;
@@ -244,10 +253,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
 
       if (it < n_main) {
         if (col_valid) {
-          const int64_t blk = q8_idx + it * q8_step;
-          const float c_hat = block_scale(qc, __ldg(args.step2 + blk / 256), mu);
+          const float c_hat = block_scale(cur.q, cur.st, mu);
           const Nf4Table tb = make_table(args.L, c_hat);
-          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          const uint32_t w[8] = {cur.c0.x, cur.c0.y, cur.c0.z, cur.c0.w, cur.c1.x, cur.c1.y, cur.c1.z, cur.c1.w};
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             uint32_t o[4];
@@ -287,13 +295,15 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     }
 
     // ------------------------------------------------------------ epilogue
+    // 16 warps: 4 per TMEM lane quadrant, each takes a quarter of the
+    // quadrant's accumulator columns.
     pipe_wait(acc_full, 0, tmo, abort_flag);
     tc_fence_after_sync();
     const int q = warp & 3;                       // TMEM lane quadrant of this warp
-    const int half = (warp - 2) >> 2;             // 0: warps 2-5, 1: warps 6-9
-    const int sub = (MS == 2) ? half : 0;
-    const int c_begin = (MS == 2) ? 0 : half * 128;
-    const int c_count = (MS == 2) ? 256 : 128;
+    const int part = (warp - 2) >> 2;             // 0..3
+    const int sub = (MS == 2) ? (part >> 1) : 0;
+    const int c_count = (MS == 2) ? 128 : 64;
+    const int c_begin = (MS == 2) ? (part & 1) * 128 : part * 64;
     const int m = m0 + sub * 128 + q * 32 + lane;
     for (int cc = 0; cc < c_count; cc += 32) {
       const int col = c_begin + cc;
@@ -301,7 +311,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + sub * 256 + col, v);
       tmem_ld_wait();
       if (m < args.M && n0 + col < args.N) {
-        uint16_t* dst = args.out + static_cast<int64_t>(m) * args.N + n0 + col;
+        uint16_t* dstp = args.out + static_cast<int64_t>(m) * args.N + n0 + col;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint4 o = make_uint4(
@@ -309,7 +319,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
               pack_bf16x2_rn(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
               pack_bf16x2_rn(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
               pack_bf16x2_rn(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
-          st_v4(dst + 8 * i, o);
+          st_v4(dstp + 8 * i, o);
         }
       }
     }
