@@ -158,39 +158,45 @@ QuantWs quant_ws(int64_t rows, int64_t cols) {
 }
 
 struct GemvPlan {
-  int splits, blocks_per_split;
+  int splits, stages_per_split, smem;
 };
 
-GemvPlan gemv_plan(int64_t in, int64_t out) {
-  const int64_t nb = in / 64;
-  const int64_t row_ctas = cdiv(out, qnf4::kGemvRowsPerCta);
+// Split K so that ~4 CTAs per SM stream the weight, each over at most
+// kGvMaxStages stages of 128 columns (its activation slice fits in shared memory).
+GemvPlan gemv_plan(int64_t M, int64_t in, int64_t out) {
+  const int64_t n_st = cdiv(in, qnf4::kGvStageK);
+  const int64_t row_ctas = cdiv(out, qnf4::kGvRows);
   const int64_t target = 4 * static_cast<int64_t>(device_sm_count());
-  int64_t splits = std::max<int64_t>(1, std::min<int64_t>(nb, cdiv(target, row_ctas)));
-  const int64_t bps = cdiv(nb, splits);
-  splits = cdiv(nb, bps);
-  return {static_cast<int>(splits), static_cast<int>(bps)};
+  int64_t splits = std::max<int64_t>(cdiv(target, row_ctas), cdiv(n_st, qnf4::kGvMaxStages));
+  splits = std::max<int64_t>(1, std::min<int64_t>(splits, n_st));
+  const int64_t sps = cdiv(n_st, splits);
+  splits = cdiv(n_st, sps);
+  return {static_cast<int>(splits), static_cast<int>(sps),
+          qnf4::gemv_smem_bytes(static_cast<int>(M), static_cast<int>(sps))};
 }
 
-// K splits of the row-wise rank-r product: only when there are too few
-// 16-row tiles to fill the GPU (few-token calls); each split keeps at least
-// one 32-wide chunk per warp.
-int rowwise_splits(int64_t M, int64_t K) {
-  const int64_t row_tiles = cdiv(M, 16);
-  if (row_tiles >= 128) return 1;
-  const int64_t max_splits = std::max<int64_t>(1, K / 32 / 8);
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(max_splits, cdiv(2 * device_sm_count(), row_tiles))));
+// K splits of the row-wise rank-r product: enough CTAs (64 rows x one
+// 64-wide rank chunk x one K range each) to keep ~2 per SM streaming, with at
+// least 4 K stages (256 columns) per range.
+int rowwise_splits(int64_t M, int64_t K, int r) {
+  const int64_t tiles = cdiv(M, 64) * cdiv(r, 64);
+  const int64_t n_st = K / 64;
+  const int64_t want = cdiv(2 * device_sm_count(), tiles);
+  int64_t ks = std::max<int64_t>(1, std::min<int64_t>(want, n_st / 4));
+  ks = cdiv(n_st, cdiv(n_st, ks));                     // no empty split
+  return static_cast<int>(ks);
 }
 
 size_t rowwise_ws(int64_t M, int64_t K, int r) {
-  const int ks = rowwise_splits(M, K);
+  const int ks = rowwise_splits(M, K, r);
   return ks > 1 ? round256(static_cast<size_t>(ks) * M * r * 4) : 0;
 }
 
 size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
   size_t b = rowwise_ws(M, in, r);
   if (M <= 16) {
-    const GemvPlan p = gemv_plan(in, out);
-    b += round256(static_cast<size_t>(p.splits) * 16 * out * 4);
+    const GemvPlan p = gemv_plan(M, in, out);
+    b += round256(static_cast<size_t>(p.splits) * M * out * 4);
   }
   return b;
 }
@@ -221,7 +227,7 @@ int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, 
   double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + w.tree_off);
 
   const int sms = device_sm_count();
-  const int64_t want = cdiv(n_blocks, 16);
+  const int64_t want = cdiv(n_blocks, 16 * qnf4::kQRounds);
   const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
   {
     LaunchTimer lt_("quantize_blocks", st);
@@ -336,18 +342,21 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
 template <int NT, bool kKR>
 int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int ks, int64_t M,
                      int64_t K, int R, float scale, cudaStream_t st) {
-  const int n_chunks = static_cast<int>(K / 32);
-  const int cps = static_cast<int>(cdiv(n_chunks, ks));
-  dim3 grid(static_cast<unsigned>(cdiv(M, 16)), static_cast<unsigned>(ks));
+  using C = qnf4::RowCfg<NT, kKR>;
+  auto kern = qnf4::rowwise_skinny_kernel<NT, kKR>;
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  const int n_st = static_cast<int>(K / 64);
+  const int sps = static_cast<int>(cdiv(n_st, ks));
+  dim3 grid(static_cast<unsigned>(cdiv(M, 64)), static_cast<unsigned>(ks), static_cast<unsigned>(cdiv(R, C::RC)));
   {
-    LaunchTimer lt_("lora_rowwise", st);
-    qnf4::rowwise_skinny_kernel<NT, kKR><<<grid, qnf4::kRowThreads, 0, st>>>(
-        act, W, out, ks > 1 ? part : nullptr, static_cast<int>(M), static_cast<int>(K), R, scale, cps);
+    LaunchTimer lt_(kKR ? "lora_rowwise_du" : "lora_rowwise", st);
+    kern<<<grid, qnf4::kRowThreads, C::SMEM, st>>>(act, W, out, ks > 1 ? part : nullptr, static_cast<int>(M),
+                                                 static_cast<int>(K), R, scale, sps);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   if (ks > 1) {
     LaunchTimer lt_("lora_rowwise_finalize", st);
-    qnf4::rowwise_finalize_kernel<<<static_cast<unsigned>(cdiv(M * R, 256)), 256, 0, st>>>(
+    qnf4::rowwise_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(M * R / 4, 256), 2048)), 256, 0, st>>>(
         part, ks, static_cast<int>(M), R, scale, out);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
@@ -359,7 +368,7 @@ int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, floa
 template <bool kKR>
 int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int64_t M, int64_t K,
                    int R, float scale, cudaStream_t st) {
-  const int ks = rowwise_splits(M, K);
+  const int ks = rowwise_splits(M, K, R);
   if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, part, ks, M, K, R, scale, st);
   if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, part, ks, M, K, R, scale, st);
   if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, part, ks, M, K, R, scale, st);
@@ -486,7 +495,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   int rc = launch_rowwise<false>(x, A, us_out, row_part, M, in, r, s, st);   // us = bf16(s x A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
-    const GemvPlan p = gemv_plan(in, out);
+    const GemvPlan p = gemv_plan(M, in, out);
     qnf4::GemvArgs g{};
     g.codes = w->codes;
     g.q8 = w->q8;
@@ -497,21 +506,21 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
-    g.blocks_per_split = p.blocks_per_split;
+    g.stages_per_split = p.stages_per_split;
+    g.x_pitch = qnf4::gemv_x_pitch(p.stages_per_split);
     g.L = tables().L;
-    const int smem = 256 * 32 * 4;
     QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::nf4_gemv_splitk_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    dim3 grid(static_cast<unsigned>(cdiv(out, qnf4::kGemvRowsPerCta)), static_cast<unsigned>(p.splits));
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem));
+    dim3 grid(static_cast<unsigned>(cdiv(out, qnf4::kGvRows)), static_cast<unsigned>(p.splits));
     {
-    LaunchTimer lt_("gemv", st);
-    qnf4::nf4_gemv_splitk_kernel<<<grid, qnf4::kGemvThreads, smem, st>>>(g);
-  }
+      LaunchTimer lt_("gemv", st);
+      qnf4::nf4_gemv_splitk_kernel<<<grid, qnf4::kGvThreads, p.smem, st>>>(g);
+    }
     QLORA_CUDA_TRY(cudaGetLastError());
     const int64_t n_el = M * out;
     {
     LaunchTimer lt_("gemv_finalize", st);
-    qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(cdiv(n_el, 256)), 256, 0, st>>>(
+    qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
         g.part, p.splits, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
   }
     QLORA_CUDA_TRY(cudaGetLastError());

@@ -25,13 +25,19 @@ constexpr int kTreeChunk = 4096;  // leaves summed by one CTA of the scale-mean 
 // One half-warp per 64-weight block: each lane loads 4 fp32 (16 B), the
 // absmax is reduced over the 16 lanes, and each lane packs its 4 codes into
 // 2 bytes, so a block's 32 code bytes are written by one coalesced store.
+// A warp takes 2*kQRounds consecutive blocks per iteration and issues all
+// their loads before any arithmetic, keeping 64 B per lane in flight.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t nearest_code(float v, const float* s_thr) {
-  // number of thresholds strictly below v, by binary search over the 15
-  // ascending thresholds (thresholds in shared memory: every lane may read a
-  // different one without serialising)
-  uint32_t c = (v > s_thr[7]) ? 8u : 0u;
-  c += (v > s_thr[c + 3]) ? 4u : 0u;
+constexpr int kQRounds = 4;
+
+// Number of thresholds strictly below v (= nearest level, ties to the lower
+// index).  Binary search over the 15 ascending thresholds: the first two
+// levels compare with register copies of thresholds 7, 3 and 11, the last two
+// read shared memory (every lane may read a different entry without
+// serialising).
+__device__ __forceinline__ uint32_t nearest_code(float v, float t3, float t7, float t11, const float* s_thr) {
+  uint32_t c = (v > t7) ? 8u : 0u;
+  c += (v > (c ? t11 : t3)) ? 4u : 0u;
   c += (v > s_thr[c + 1]) ? 2u : 0u;
   c += (v > s_thr[c]) ? 1u : 0u;
   return c;
@@ -43,37 +49,45 @@ __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
   __shared__ float s_thr[16];
   if (threadIdx.x < 15) s_thr[threadIdx.x] = thr.v[threadIdx.x];
   __syncthreads();
+  const float t3 = thr.v[3], t7 = thr.v[7], t11 = thr.v[11];
 
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;          // which of the warp's two blocks
+  const int half = lane >> 4;          // which block of a pair
   const int l16 = lane & 15;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
 
-  for (int64_t pair = warp; pair * 2 < n_blocks; pair += n_warps) {
-    const int64_t b = pair * 2 + half;
-    const bool valid = b < n_blocks;
-    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (valid) {
-      const uint4 u = ld_stream_v4(W + b * kBlock + l16 * 4);
-      w = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
-    }
-    float m = fmaxf(fmaxf(fabsf(w.x), fabsf(w.y)), fmaxf(fabsf(w.z), fabsf(w.w)));
+  for (int64_t base = warp * 2 * kQRounds; base < n_blocks; base += n_warps * 2 * kQRounds) {
+    float4 w[kQRounds];
 #pragma unroll
-    for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    // m is now the exact absmax of this half-warp's block
-    uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
-    if (m > 0.f) {
-      const float r = __frcp_rn(m);
-      c0 = nearest_code(__fmul_rn(w.x, r), s_thr);
-      c1 = nearest_code(__fmul_rn(w.y, r), s_thr);
-      c2 = nearest_code(__fmul_rn(w.z, r), s_thr);
-      c3 = nearest_code(__fmul_rn(w.w, r), s_thr);
+    for (int rd = 0; rd < kQRounds; ++rd) {
+      const int64_t b = base + 2 * rd + half;
+      w[rd] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b < n_blocks) {
+        const uint4 u = ld_stream_v4(W + b * kBlock + l16 * 4);
+        w[rd] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+      }
     }
-    if (valid) {
-      const uint16_t packed = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
-      reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = packed;
-      if (l16 == 0) absmax[b] = m;
+#pragma unroll
+    for (int rd = 0; rd < kQRounds; ++rd) {
+      const int64_t b = base + 2 * rd + half;
+      float m = fmaxf(fmaxf(fabsf(w[rd].x), fabsf(w[rd].y)), fmaxf(fabsf(w[rd].z), fabsf(w[rd].w)));
+#pragma unroll
+      for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      // m is now the exact absmax of this half-warp's block
+      uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
+      if (m > 0.f) {
+        const float r = __frcp_rn(m);
+        c0 = nearest_code(__fmul_rn(w[rd].x, r), t3, t7, t11, s_thr);
+        c1 = nearest_code(__fmul_rn(w[rd].y, r), t3, t7, t11, s_thr);
+        c2 = nearest_code(__fmul_rn(w[rd].z, r), t3, t7, t11, s_thr);
+        c3 = nearest_code(__fmul_rn(w[rd].w, r), t3, t7, t11, s_thr);
+      }
+      if (b < n_blocks) {
+        const uint16_t packed = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
+        reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = packed;
+        if (l16 == 0) absmax[b] = m;
+      }
     }
   }
 }
@@ -160,27 +174,44 @@ __global__ void __launch_bounds__(256) dq_scales_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// K4: dequantize to bf16.  One thread per 32 codes (16 bytes, half a block):
-// it forms the block scale, the block's 16-entry bf16 table, decodes with
-// prmt and writes 64 bytes of bf16.
+// K4: dequantize to bf16.  A thread handles 32 codes (16 bytes, half a block)
+// at a time -- block scale, the block's 16-entry bf16 table, prmt decode,
+// 64 bytes of bf16 out -- and loads kDqRounds such halves before decoding.
 // ---------------------------------------------------------------------------
+constexpr int kDqRounds = 4;
+
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
     const uint8_t* __restrict__ codes, const int8_t* __restrict__ q8,
     const float* __restrict__ step2, const float* __restrict__ mean_ptr,
     int64_t n_halves, uint16_t* __restrict__ out, Levels L) {
   const float mu = *mean_ptr;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_halves; i += stride) {
-    const int64_t b = i >> 1;
-    const uint4 cw = ld_stream_v4(codes + i * 16);
-    const float c_hat = block_scale(q8[b], step2[b / kGroup], mu);
-    const Nf4Table t = make_table(L, c_hat);
-    uint32_t o[4];
-    uint16_t* dst = out + i * 32;
-    decode8(t, cw.x, o); st_v4(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
-    decode8(t, cw.y, o); st_v4(dst + 8, make_uint4(o[0], o[1], o[2], o[3]));
-    decode8(t, cw.z, o); st_v4(dst + 16, make_uint4(o[0], o[1], o[2], o[3]));
-    decode8(t, cw.w, o); st_v4(dst + 24, make_uint4(o[0], o[1], o[2], o[3]));
+  const int64_t n_thr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i0 = tid; i0 < n_halves; i0 += n_thr * kDqRounds) {
+    uint4 cw[kDqRounds];
+    float ch[kDqRounds];
+#pragma unroll
+    for (int rd = 0; rd < kDqRounds; ++rd) {
+      const int64_t i = i0 + rd * n_thr;
+      if (i < n_halves) {
+        const int64_t b = i >> 1;
+        cw[rd] = ld_stream_v4(codes + i * 16);
+        ch[rd] = block_scale(q8[b], step2[b / kGroup], mu);
+      }
+    }
+#pragma unroll
+    for (int rd = 0; rd < kDqRounds; ++rd) {
+      const int64_t i = i0 + rd * n_thr;
+      if (i < n_halves) {
+        const Nf4Table t = make_table(L, ch[rd]);
+        uint32_t o[4];
+        uint16_t* dst = out + i * 32;
+        decode8(t, cw[rd].x, o); st_v4(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
+        decode8(t, cw[rd].y, o); st_v4(dst + 8, make_uint4(o[0], o[1], o[2], o[3]));
+        decode8(t, cw[rd].z, o); st_v4(dst + 16, make_uint4(o[0], o[1], o[2], o[3]));
+        decode8(t, cw[rd].w, o); st_v4(dst + 24, make_uint4(o[0], o[1], o[2], o[3]));
+      }
+    }
   }
 }
 

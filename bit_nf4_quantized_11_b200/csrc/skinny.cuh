@@ -21,119 +21,166 @@
 namespace qnf4 {
 
 // ---------------------------------------------------------------------------
-// row-wise skinny GEMM.  CTA = 8 warps on 16 token rows and one K range
-// (blockIdx.y splits K when there are few rows); the K range is cut into
-// 32-wide chunks dealt round-robin to the warps, which load a batch of chunks
-// before issuing its MMAs so that several loads are in flight per thread.
-// The MMA's K order is permuted consistently for both operands (thread q of a
-// quad owns physical k = 8q..8q+7 of every 32-chunk), so each activation
-// fragment is one 16-byte load.  The second operand is either Wt [R][K]
-// (k contiguous: one 16-byte load per n-tile) or W [K][R] (n contiguous:
-// element loads that stay in L1, so no transposed copy is needed).
-// Warp partials are reduced through shared memory in a fixed order; with
-// one K range the result is scaled and rounded to bf16, otherwise fp32
-// partials go to part[split][row][n] for rowwise_finalize_kernel.
-// Output columns are processed 8*NT at a time.
+// row-wise skinny GEMM: out[m][n] = scale * sum_k act[m][k] * W[n][k] for n in
+// one 64-wide chunk of the rank (grid.z), over one K range (grid.y).
+// CTA = 4 warps on 64 token rows; K is streamed in 64-wide stages through a
+// kRowStages-deep cp.async ring (the activation tile and the matching W tile),
+// consumed with ldmatrix + mma.sync (each warp owns 16 rows x 8*NT columns).
+// W is either [R][K] (k contiguous, ldmatrix) or [K][R] (n contiguous,
+// ldmatrix.trans), so neither orientation needs a transposed copy.
+// Activation rows are 128 B in shared memory with the 16-byte chunk index
+// XOR-ed by (row & 7), so every ldmatrix phase hits 8 different bank groups.
+// With one K range the result is scaled and rounded to bf16 in place;
+// otherwise fp32 partials go to part[split][row][n] for the finalize kernel.
 // ---------------------------------------------------------------------------
-constexpr int kRowThreads = 256;
+constexpr int kRowThreads = 128;
+constexpr int kRowStages = 4;
+constexpr int kRowActBytes = 64 * 128;                  // 64 rows x 64 k bf16
 
 template <int NT, bool kKR>
-__device__ __forceinline__ void rowwise_b_frag(const uint16_t* __restrict__ W, int K, int R, int nb, int j,
-                                               int g, int q, int k0, uint4& b) {
-  if (!kKR) {
-    b = ld_nc_v4(W + static_cast<int64_t>(nb + 8 * j + g) * K + k0 + 8 * q);
-  } else {
-    const uint16_t* p = W + static_cast<int64_t>(k0 + 8 * q) * R + nb + 8 * j + g;
-    uint32_t e[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) e[i] = __ldg(p + static_cast<int64_t>(i) * R);
-    b = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
-  }
-}
+struct RowCfg {
+  static constexpr int RC = 8 * NT;                     // rank columns per CTA
+  // The tile always spans at least 16 rank columns (an x4 ldmatrix reads two
+  // 8-column tiles); columns past the rank are zero-filled.
+  static constexpr int RCA = RC < 16 ? 16 : RC;
+  static constexpr int NTA = RCA / 8;
+  // W tile: [RCA rows x 64 k] (128 B rows, swizzled) or [64 k rows x RCA n] (padded rows)
+  static constexpr int W_PITCH = kKR ? (RCA * 2 + ((RCA * 2 / 16) % 2 == 0 ? 16 : 0)) : 128;
+  static constexpr int W_BYTES = kKR ? 64 * W_PITCH : RCA * 128;
+  static constexpr int STAGE = kRowActBytes + ((W_BYTES + 127) / 128) * 128;
+  static constexpr int SMEM = kRowStages * STAGE;
+};
 
 template <int NT, bool kKR>
 __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
     const uint16_t* __restrict__ act, const uint16_t* __restrict__ W,
     uint16_t* __restrict__ out, float* __restrict__ part, int M, int K, int R, float scale,
-    int chunks_per_split) {
-  constexpr int kBatch = NT <= 2 ? 4 : (NT == 4 ? 2 : 1);
-  __shared__ float s_red[8][16][8 * NT + 1];
+    int stages_per_split) {
+  using C = RowCfg<NT, kKR>;
+  extern __shared__ __align__(128) uint8_t s_row[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, q = lane & 3;
-  const int m0 = blockIdx.x * 16;
-  const int c_begin = blockIdx.y * chunks_per_split;
-  const int c_end = min(K / 32, c_begin + chunks_per_split);
-  const bool row0 = (m0 + g) < M, row1 = (m0 + g + 8) < M;
-  const uint16_t* a_row0 = act + static_cast<int64_t>(row0 ? m0 + g : 0) * K + 8 * q;
-  const uint16_t* a_row1 = act + static_cast<int64_t>(row1 ? m0 + g + 8 : 0) * K + 8 * q;
-  const uint4 z = make_uint4(0, 0, 0, 0);
+  const int m0 = blockIdx.x * 64;
+  const int nb = blockIdx.z * C::RC;
+  const int nt = min(NT, (R - nb) / 8);
+  const int kst_begin = blockIdx.y * stages_per_split;
+  const int kst_end = min(K / 64, kst_begin + stages_per_split);
+  const int n_st = kst_end - kst_begin;
 
-  for (int nb = 0; nb < R; nb += 8 * NT) {
-    const int nt = min(NT, (R - nb) / 8);
-    float acc[NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  auto stage = [&](int i) {
+    uint8_t* sa = s_row + (i % kRowStages) * C::STAGE;
+    uint8_t* sw = sa + kRowActBytes;
+    const int k0 = (kst_begin + i) * 64;
+    for (int e = threadIdx.x; e < 64 * 8; e += kRowThreads) {       // activation 64 x 64
+      const int row = e >> 3, ch = e & 7;
+      const bool ok = m0 + row < M;
+      const uint16_t* src = act + static_cast<int64_t>(ok ? m0 + row : 0) * K + k0 + ch * 8;
+      cp_async_16(smem_u32(sa + row * 128 + ((ch ^ (row & 7)) << 4)), src, ok);
+    }
+    if (!kKR) {
+      for (int e = threadIdx.x; e < C::RCA * 8; e += kRowThreads) {  // W rows n, 64 k
+        const int row = e >> 3, ch = e & 7;
+        const bool ok = row < C::RC && nb + row < R;
+        const uint16_t* src = W + static_cast<int64_t>(ok ? nb + row : 0) * K + k0 + ch * 8;
+        cp_async_16(smem_u32(sw + row * 128 + ((ch ^ (row & 7)) << 4)), src, ok);
+      }
+    } else {
+      for (int e = threadIdx.x; e < 64 * C::NTA; e += kRowThreads) { // W rows k, RCA n
+        const int row = e / C::NTA, ch = e % C::NTA;
+        const bool ok = ch < NT && nb + ch * 8 < R;
+        const uint16_t* src = W + static_cast<int64_t>(k0 + row) * R + (ok ? nb + ch * 8 : 0);
+        cp_async_16(smem_u32(sw + row * C::W_PITCH + ch * 16), src, ok);
+      }
+    }
+  };
 
-    for (int c = c_begin + warp; c < c_end; c += 8 * kBatch) {
-      uint4 u0[kBatch], u1[kBatch], b[kBatch][NT];
+  float acc[NT][4];
 #pragma unroll
-      for (int bi = 0; bi < kBatch; ++bi) {
-        const int cc = c + 8 * bi;
-        const bool ok = cc < c_end;
-        const int k0 = cc * 32;
-        u0[bi] = (ok && row0) ? ld_nc_v4(a_row0 + k0) : z;
-        u1[bi] = (ok && row1) ? ld_nc_v4(a_row1 + k0) : z;
+  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          b[bi][j] = z;
-          if (ok && j < nt) rowwise_b_frag<NT, kKR>(W, K, R, nb, j, g, q, k0, b[bi][j]);
-        }
+  for (int i = 0; i < kRowStages - 1; ++i) {
+    if (i < n_st) stage(i);
+    cp_async_commit();
+  }
+  for (int i = 0; i < n_st; ++i) {
+    cp_async_wait<kRowStages - 2>();
+    __syncthreads();
+    if (i + kRowStages - 1 < n_st) stage(i + kRowStages - 1);
+    cp_async_commit();
+    const uint32_t sa = smem_u32(s_row + (i % kRowStages) * C::STAGE);
+    const uint32_t sw = sa + kRowActBytes;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      {
+        const int row = warp * 16 + (lane & 15);
+        const int ch = 2 * kk + (lane >> 4);
+        ldsm_x4(sa + row * 128 + ((ch ^ (row & 7)) << 4), a0, a1, a2, a3);
       }
 #pragma unroll
-      for (int bi = 0; bi < kBatch; ++bi) {
+      for (int jp = 0; jp < NT; jp += 2) {
+        if (jp < nt) {
+          uint32_t b0, b1, b2, b3;
+          if (!kKR) {
+            // matrices: (n jp*8.., k lo), (n jp*8.., k hi), (n jp*8+8.., k lo), (n jp*8+8.., k hi)
+            const int mi = lane >> 3;
+            const int row = jp * 8 + ((mi >> 1) << 3) + (lane & 7);
+            const int ch = 2 * kk + (mi & 1);
+            ldsm_x4(sw + row * 128 + ((ch ^ (row & 7)) << 4), b0, b1, b2, b3);
+          } else {
+            // matrices: (k lo, n jp*8..), (k hi, n jp*8..), (k lo, n jp*8+8..), (k hi, n jp*8+8..)
+            const int mi = lane >> 3;
+            const int krow = kk * 16 + ((mi & 1) << 3) + (lane & 7);
+            const int ncol = jp * 8 + ((mi >> 1) << 3);
+            ldsm_x4_trans(sw + krow * C::W_PITCH + ncol * 2, b0, b1, b2, b3);
+          }
+          mma_bf16_16816(acc[jp], a0, a1, a2, a3, b0, b1);
+          if (jp + 1 < nt) mma_bf16_16816(acc[jp + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+
+  const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j < nt) {
-            mma_bf16_16816(acc[j], u0[bi].x, u1[bi].x, u0[bi].y, u1[bi].y, b[bi][j].x, b[bi][j].y);
-            mma_bf16_16816(acc[j], u0[bi].z, u1[bi].z, u0[bi].w, u1[bi].w, b[bi][j].z, b[bi][j].w);
+  for (int j = 0; j < NT; ++j) {
+    if (j < nt) {
+      const int n = nb + 8 * j + 2 * q;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int m = m0 + warp * 16 + g + 8 * h;
+        if (m < M) {
+          const float v0 = acc[j][2 * h], v1 = acc[j][2 * h + 1];
+          if (part == nullptr) {
+            *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(m) * R + n) =
+                pack_bf16x2_rn(v0 * scale, v1 * scale);
+          } else {
+            *reinterpret_cast<float2*>(part + (static_cast<int64_t>(blockIdx.y) * M + m) * R + n) =
+                make_float2(v0, v1);
           }
         }
       }
     }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      s_red[warp][g][8 * j + 2 * q] = acc[j][0];
-      s_red[warp][g][8 * j + 2 * q + 1] = acc[j][1];
-      s_red[warp][g + 8][8 * j + 2 * q] = acc[j][2];
-      s_red[warp][g + 8][8 * j + 2 * q + 1] = acc[j][3];
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < 16 * 8 * NT; e += kRowThreads) {
-      const int rr = e / (8 * NT), cc = e % (8 * NT);
-      if (cc < nt * 8 && m0 + rr < M) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) v += s_red[w][rr][cc];
-        if (part == nullptr) {
-          out[static_cast<int64_t>(m0 + rr) * R + nb + cc] = __bfloat16_as_ushort(__float2bfloat16_rn(v * scale));
-        } else {
-          part[(static_cast<int64_t>(blockIdx.y) * M + m0 + rr) * R + nb + cc] = v;
-        }
-      }
-    }
-    __syncthreads();
   }
 }
 
-// out[m][n] = bf16(scale * sum_{s < splits} part[s][m][n]), splits added in order.
+// out[m][n] = bf16(scale * sum_{s < splits} part[s][m][n]), splits added in
+// order; four outputs per thread (M*R is a multiple of 8).
 __global__ void __launch_bounds__(256) rowwise_finalize_kernel(
     const float* __restrict__ part, int splits, int M, int R, float scale, uint16_t* __restrict__ out) {
-  const int64_t n_el = static_cast<int64_t>(M) * R;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_el;
+  const int64_t n4 = static_cast<int64_t>(M) * R / 4;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float v = 0.f;
-    for (int s = 0; s < splits; ++s) v += part[static_cast<int64_t>(s) * n_el + e];
-    out[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v * scale));
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* p = reinterpret_cast<const float4*>(part) + e;
+#pragma unroll 4
+    for (int s = 0; s < splits; ++s) {
+      const float4 t = __ldg(p + static_cast<int64_t>(s) * n4);
+      v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
+    }
+    reinterpret_cast<uint2*>(out)[e] =
+        make_uint2(pack_bf16x2_rn(v.x * scale, v.y * scale), pack_bf16x2_rn(v.z * scale, v.w * scale));
   }
 }
 
@@ -286,6 +333,7 @@ __global__ void __launch_bounds__(256) sum_chunks_kernel(
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
     for (int c = 0; c < C; ++c) {
       const float4 t = __ldg(reinterpret_cast<const float4*>(part) + c * stride + e);
       v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;

@@ -65,7 +65,9 @@ def test_workspace_sizes(lib):
     n = q.workspace_size(q.OP_QUANTIZE, 0, 4096, 4096, 0)
     assert n >= 4096 * 4096 // 64 * 4
     assert q.workspace_size(q.OP_DEQUANTIZE, 0, 512, 512, 0) == 0
-    assert q.workspace_size(q.OP_LINEAR_FWD, 4096, 4096, 4096, 16) == 0     # fused GEMM path
+    # forward: at most the split-K partials of the rank-r down-projection
+    assert q.workspace_size(q.OP_LINEAR_FWD, 4096, 4096, 4096, 16) <= 4096 * 16 * 4 * 64
+    assert q.workspace_size(q.OP_LINEAR_FWD, 64, 128, 128, 8) == 0           # one K range
     assert q.workspace_size(q.OP_LINEAR_FWD, 4, 8192, 28672, 16) > 0        # split-K GEMV partials
     nb = q.workspace_size(q.OP_LINEAR_BWD, 4096, 4096, 4096, 16)
     assert nb >= 4096 * 16 * 2
