@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["quantize", "gemv", "workloads"], default=None,
+                    help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
 
 
@@ -422,16 +424,10 @@ def run_reference(args, world, rank):
 
 
 # ---------------------------------------------------------------------------- components
-def components(q, dev):
-    """Extra measurements outside the timed region: quantizer and dequantizer
-    HBM throughput, the few-token GEMV, and the other fwd+bwd workloads."""
-    out = {}
-    peaks, src = load_peaks()
+def comp_quantize(q, dev, peaks, src, reps=3):
+    """Quantizer and dequantizer on the 65B decoder layer's seven weights (3.2 GB fp32 > L2)."""
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-
-    # quantizer + dequantizer on the 65B decoder layer's seven weights (3.2 GB fp32 > L2)
-    quant_res = []
-    ws = None
+    out = {}
     weights = []
     for i, (label, n_in, n_out) in enumerate(workloads.LAYER_65B.projections):
         W = synth.weight(n_out, n_in, workloads.LAYER_65B.w_std, seed=i).to(dev)
@@ -445,7 +441,6 @@ def components(q, dev):
     q.timing_reset()
     q.timing_enable(True)
     a, b = ev(), ev()
-    reps = 3
     a.record()
     for _ in range(reps):
         for _, W, w in weights:
@@ -461,7 +456,6 @@ def components(q, dev):
         "frac_hbm": qbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "quantize_blocks_ms": kq / reps if nq else None,
         "peak_source": f"hbm_gbs of {src}"}
-    # dequantizer (0.52 B/weight in, 2 B/weight out)
     deq_out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _, _, w in weights]
     for (_, _, w), o in zip(weights, deq_out):
         q.dequantize_nf4(w, out=o)
@@ -478,13 +472,18 @@ def components(q, dev):
                                    "frac_hbm": dbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"]}
     del deq_out, weights, ws
     torch.cuda.empty_cache()
+    return out
 
-    # few-token GEMV on the 70B MLP shapes
+
+def comp_gemv(q, dev, peaks, n=60):
+    """Few-token forward on the 70B MLP shapes; 3 weight copies (3 x 121 MB > L2)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    a, b = ev(), ev()
     g = workloads.GEMV_70B
     gres = {}
     for (label, n_in, n_out) in g.projections:
         ws_list = []
-        for i in range(3):              # 3 weight copies: 3 x 121 MB > L2
+        for i in range(3):
             W = synth.weight(n_out, n_in, g.w_std, seed=10 + i).to(dev)
             ws_list.append(q.quantize_nf4(W))
             del W
@@ -497,7 +496,6 @@ def components(q, dev):
             torch.cuda.synchronize()
             q.timing_reset()
             q.timing_enable(True)
-            n = 60
             a.record()
             for i in range(n):
                 q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha)
@@ -514,9 +512,14 @@ def components(q, dev):
                 "frac_hbm_kernel": (wbytes / (kms / kn * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kn else None}
         del ws_list
         torch.cuda.empty_cache()
-    out["gemv_70b"] = gres
+    return {"gemv_70b": gres}
 
-    # other fwd+bwd workloads: 7B MLP (3 projections) and 65B decoder layer (7 projections)
+
+def comp_workloads(q, dev, peaks):
+    """fwd+bwd of the 7B MLP (3 projections) and the 65B decoder layer (7 projections)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    a, b = ev(), ev()
+    out = {}
     for wl in (workloads.MLP_7B, workloads.LAYER_65B):
         M = wl.M[0]
         tot_ms, tot_flops = 0.0, 0.0
@@ -545,11 +548,32 @@ def components(q, dev):
     return out
 
 
+def components(q, dev, only=None):
+    """Extra measurements outside the timed region: quantizer and dequantizer
+    HBM throughput, the few-token GEMV, and the other fwd+bwd workloads."""
+    peaks, src = load_peaks()
+    out = {}
+    if only in (None, "quantize"):
+        out.update(comp_quantize(q, dev, peaks, src))
+    if only in (None, "gemv"):
+        out.update(comp_gemv(q, dev, peaks))
+    if only in (None, "workloads"):
+        out.update(comp_workloads(q, dev, peaks))
+    return out
+
+
 # ---------------------------------------------------------------------------- main
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
+        if args.only is not None:
+            import bit_nf4_quantized_11_b200 as q
+            q.load()
+            if rank == 0:
+                print(json.dumps({"only": args.only,
+                                  "components": components(q, torch.device("cuda", local), args.only)}), flush=True)
+            return
         if args.impl == "reference":
             line = run_reference(args, world, rank)
             if line is not None:

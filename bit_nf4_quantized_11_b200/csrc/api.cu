@@ -36,12 +36,34 @@ std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 struct Tables {
   Levels L;
   Thresholds T;
+  qnf4::CodeTable C;
 };
+
+// Cell table of nearest_code: cell n covers 16 v in [n - 16.5, n - 15.5);
+// below[n] = thresholds under the cell, inside[n] = the (at most one)
+// threshold in it or +inf.
+void build_code_table(const Thresholds& T, qnf4::CodeTable* c) {
+  for (int n = 0; n < qnf4::kCodeCells; ++n) {
+    const double lo = (n - 16.5) / 16.0, hi = (n - 15.5) / 16.0;
+    uint32_t below = 0;
+    float inside = INFINITY;
+    for (int j = 0; j < 15; ++j) {
+      const double t = T.v[j];
+      if (t < lo) ++below;
+      else if (t < hi) inside = T.v[j];
+    }
+    c->below[n] = below;
+    c->inside[n] = inside;
+  }
+}
 
 const Tables& tables() {
   static Tables t;
   static std::once_flag once;
-  std::call_once(once, [] { qnf4_host::build_codebook(t.L.v, t.T.v); });
+  std::call_once(once, [] {
+    qnf4_host::build_codebook(t.L.v, t.T.v);
+    build_code_table(t.T, &t.C);
+  });
   return t;
 }
 
@@ -158,21 +180,36 @@ QuantWs quant_ws(int64_t rows, int64_t cols) {
 }
 
 struct GemvPlan {
-  int splits, stages_per_split, smem;
+  int ctas, local_tiles, n_st;
+  int64_t n_units;
 };
 
-// Split K so that ~4 CTAs per SM stream the weight, each over at most
-// kGvMaxStages stages of 128 columns (its activation slice fits in shared memory).
-GemvPlan gemv_plan(int64_t M, int64_t in, int64_t out) {
-  const int64_t n_st = cdiv(in, qnf4::kGvStageK);
-  const int64_t row_ctas = cdiv(out, qnf4::kGvRows);
-  const int64_t target = 4 * static_cast<int64_t>(device_sm_count());
-  int64_t splits = std::max<int64_t>(cdiv(target, row_ctas), cdiv(n_st, qnf4::kGvMaxStages));
-  splits = std::max<int64_t>(1, std::min<int64_t>(splits, n_st));
-  const int64_t sps = cdiv(n_st, splits);
-  splits = cdiv(n_st, sps);
-  return {static_cast<int>(splits), static_cast<int>(sps),
-          qnf4::gemv_smem_bytes(static_cast<int>(M), static_cast<int>(sps))};
+int gemv_ctas_per_sm() {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel, qnf4::kGvThreads, qnf4::kGvSmem) !=
+          cudaSuccess ||
+      n < 1)
+    n = 2;
+  return n;
+}
+
+// Persistent grid (every CTA resident at once) splitting the (128-row tile x
+// 128-column unit) sequence evenly; local_tiles bounds the tiles one CTA's
+// range touches.
+GemvPlan gemv_plan(int64_t in, int64_t out) {
+  GemvPlan p{};
+  p.n_st = static_cast<int>(cdiv(in, qnf4::kGvStageK));
+  p.n_units = cdiv(out, qnf4::kGvRows) * p.n_st;
+  const int64_t resident = static_cast<int64_t>(gemv_ctas_per_sm()) * device_sm_count();
+  p.ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(resident, p.n_units)));
+  const int64_t per_cta = cdiv(p.n_units, p.ctas);
+  p.local_tiles = static_cast<int>(cdiv(per_cta, p.n_st) + 1);
+  return p;
+}
+
+size_t gemv_ws(int64_t M, int64_t in, int64_t out) {
+  const GemvPlan p = gemv_plan(in, out);
+  return round256(static_cast<size_t>(p.ctas) * p.local_tiles * M * qnf4::kGvRows * 4);
 }
 
 // K splits of the row-wise rank-r product: enough CTAs (64 rows x one
@@ -194,10 +231,7 @@ size_t rowwise_ws(int64_t M, int64_t K, int r) {
 
 size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
   size_t b = rowwise_ws(M, in, r);
-  if (M <= 16) {
-    const GemvPlan p = gemv_plan(M, in, out);
-    b += round256(static_cast<size_t>(p.splits) * M * out * 4);
-  }
+  if (M <= 16) b += gemv_ws(M, in, out);
   return b;
 }
 
@@ -231,7 +265,7 @@ int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, 
   const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
   {
     LaunchTimer lt_("quantize_blocks", st);
-    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.T);
+    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
 
@@ -495,7 +529,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   int rc = launch_rowwise<false>(x, A, us_out, row_part, M, in, r, s, st);   // us = bf16(s x A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
-    const GemvPlan p = gemv_plan(M, in, out);
+    const GemvPlan p = gemv_plan(in, out);
     qnf4::GemvArgs g{};
     g.codes = w->codes;
     g.q8 = w->q8;
@@ -506,23 +540,23 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
-    g.stages_per_split = p.stages_per_split;
-    g.x_pitch = qnf4::gemv_x_pitch(p.stages_per_split);
+    g.n_st = p.n_st;
+    g.n_units = p.n_units;
+    g.local_tiles = p.local_tiles;
     g.L = tables().L;
-    QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::nf4_gemv_splitk_kernel,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize, p.smem));
-    dim3 grid(static_cast<unsigned>(cdiv(out, qnf4::kGvRows)), static_cast<unsigned>(p.splits));
+    QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::nf4_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        qnf4::kGvSmem));
     {
       LaunchTimer lt_("gemv", st);
-      qnf4::nf4_gemv_splitk_kernel<<<grid, qnf4::kGvThreads, p.smem, st>>>(g);
+      qnf4::nf4_gemv_kernel<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(g);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
     const int64_t n_el = M * out;
     {
-    LaunchTimer lt_("gemv_finalize", st);
-    qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
-        g.part, p.splits, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
-  }
+      LaunchTimer lt_("gemv_finalize", st);
+      qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
+          g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
+    }
     QLORA_CUDA_TRY(cudaGetLastError());
     return QLORA_OK;
   }

@@ -21,39 +21,53 @@ constexpr int kGroup = 256;       // blocks per second-level group
 constexpr int kTreeChunk = 4096;  // leaves summed by one CTA of the scale-mean tree
 
 // ---------------------------------------------------------------------------
+// K1 and its code table
+// ---------------------------------------------------------------------------
+constexpr int kQRounds = 4;
+
+// Exact nearest level without a search.  [-1, 1] (slightly widened: a block's
+// normalised values can exceed 1 by an ulp) is cut into 33 cells by
+// n = round(16 v) + 16; every cell contains at most one threshold and every
+// threshold lies more than 4e-3 from a cell edge, so for any fp32 v
+//   #{j : v > thr_j} = below[n] + (v > inside[n])
+// where below[n] counts the thresholds under the cell and inside[n] is the
+// threshold inside it (+inf if none).  The host builds the table from the
+// fp32 thresholds; n comes from one fused multiply-add whose single rounding
+// to an integer (magnitude 1.5 * 2^23) yields round(16 v) in the low bits.
+constexpr int kCodeCells = 33;
+constexpr float kCellMagic = 12582928.0f;          // 1.5 * 2^23 + 16
+struct CodeTable { uint32_t below[kCodeCells]; float inside[kCodeCells]; };
+
+__device__ __forceinline__ uint32_t nearest_code(float v, uint32_t tab_lane) {
+  const float y = __fmaf_rn(v, 16.0f, kCellMagic);
+  // finite |v| <= 1 + 2^-22 gives n in 0..32; the clamp keeps any input in the table
+  const uint32_t n = min(static_cast<uint32_t>(__float_as_int(y) - __float_as_int(kCellMagic) + 16),
+                         static_cast<uint32_t>(kCodeCells - 1));
+  uint32_t below, inside_bits;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(inside_bits) : "r"(tab_lane + n * 256));
+  return below + (v > __uint_as_float(inside_bits) ? 1u : 0u);
+}
+
 // K1: per-block absmax, nearest-level code, nibble packing.
 // One half-warp per 64-weight block: each lane loads 4 fp32 (16 B), the
 // absmax is reduced over the 16 lanes, and each lane packs its 4 codes into
 // 2 bytes, so a block's 32 code bytes are written by one coalesced store.
 // A warp takes 2*kQRounds consecutive blocks per iteration and issues all
 // their loads before any arithmetic, keeping 64 B per lane in flight.
-// ---------------------------------------------------------------------------
-constexpr int kQRounds = 4;
-
-// Number of thresholds strictly below v (= nearest level, ties to the lower
-// index).  Binary search over the 15 ascending thresholds: the first two
-// levels compare with register copies of thresholds 7, 3 and 11, the last two
-// read shared memory (every lane may read a different entry without
-// serialising).
-__device__ __forceinline__ uint32_t nearest_code(float v, float t3, float t7, float t11, const float* s_thr) {
-  uint32_t c = (v > t7) ? 8u : 0u;
-  c += (v > (c ? t11 : t3)) ? 4u : 0u;
-  c += (v > s_thr[c + 1]) ? 2u : 0u;
-  c += (v > s_thr[c]) ? 1u : 0u;
-  return c;
-}
-
+// The cell table sits in shared memory with one copy per lane (entry n of
+// lane l at (n*32 + l)*8), so lookups never conflict.
 __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
     const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
-    float* __restrict__ absmax, Thresholds thr) {
-  __shared__ float s_thr[16];
-  if (threadIdx.x < 15) s_thr[threadIdx.x] = thr.v[threadIdx.x];
+    float* __restrict__ absmax, CodeTable tab) {
+  __shared__ __align__(16) uint2 s_tab[kCodeCells * 32];
+  for (int e = threadIdx.x; e < kCodeCells * 32; e += blockDim.x)
+    s_tab[e] = make_uint2(tab.below[e >> 5], __float_as_uint(tab.inside[e >> 5]));
   __syncthreads();
-  const float t3 = thr.v[3], t7 = thr.v[7], t11 = thr.v[11];
 
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;          // which block of a pair
   const int l16 = lane & 15;
+  const uint32_t tab_lane = smem_u32(s_tab) + lane * 8;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
 
@@ -75,17 +89,22 @@ __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
 #pragma unroll
       for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       // m is now the exact absmax of this half-warp's block
-      uint32_t c0 = 7, c1 = 7, c2 = 7, c3 = 7;
-      if (m > 0.f) {
-        const float r = __frcp_rn(m);
-        c0 = nearest_code(__fmul_rn(w[rd].x, r), t3, t7, t11, s_thr);
-        c1 = nearest_code(__fmul_rn(w[rd].y, r), t3, t7, t11, s_thr);
-        c2 = nearest_code(__fmul_rn(w[rd].z, r), t3, t7, t11, s_thr);
-        c3 = nearest_code(__fmul_rn(w[rd].w, r), t3, t7, t11, s_thr);
+      uint32_t packed = 0x7777u;
+      const float r = __frcp_rn(m);
+      if (m > 0.f && isinf(r)) {
+        // absmax so small that 1/absmax overflows: v = w * inf is +inf (code
+        // 15), -inf (code 0), or NaN for a zero weight (the zero level, 7)
+        auto sat = [](float x) -> uint32_t { return x > 0.f ? 15u : (x < 0.f ? 0u : 7u); };
+        packed = sat(w[rd].x) | (sat(w[rd].y) << 4) | (sat(w[rd].z) << 8) | (sat(w[rd].w) << 12);
+      } else if (m > 0.f) {
+        const uint32_t c0 = nearest_code(__fmul_rn(w[rd].x, r), tab_lane);
+        const uint32_t c1 = nearest_code(__fmul_rn(w[rd].y, r), tab_lane);
+        const uint32_t c2 = nearest_code(__fmul_rn(w[rd].z, r), tab_lane);
+        const uint32_t c3 = nearest_code(__fmul_rn(w[rd].w, r), tab_lane);
+        packed = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
       }
       if (b < n_blocks) {
-        const uint16_t packed = static_cast<uint16_t>(c0 | (c1 << 4) | (c2 << 8) | (c3 << 12));
-        reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = packed;
+        reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = static_cast<uint16_t>(packed);
         if (l16 == 0) absmax[b] = m;
       }
     }

@@ -122,7 +122,9 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t in_features,
  * qlora_quantize_nf4 -- blockwise NF4 quantization with double quantization.
  *
  * Per block b of 64 weights: c_b = max|w| (exact); if c_b = 0 every code is 7;
- * otherwise v = fp32(w * fp32(1/c_b)) and code = #{j : v > thresholds[j]}.
+ * otherwise v = fp32(w * fp32(1/c_b)) and code = #{j : v > thresholds[j]},
+ * except that a NaN v (a zero weight in a block whose 1/c_b overflows to
+ * infinity) is code 7.
  * Second level: mean = fp32(T / n_blocks) where T is the fp64 sum of all c_b
  * in a fixed binary tree (zero-padded to a power of two, adjacent pairs added
  * level by level) and the division is done in fp64; d_b = fp32(c_b - mean);

@@ -29,7 +29,10 @@ R2 Nearest level, ties to the lower index; implemented as a comparison with the
    exact fp64 midpoints of consecutive fp32 levels.
 R3 Normalisation ``v = fl32(w * fl32(1/c))`` (reciprocal then multiply) rather
    than a division; an all-zero block (c = 0) encodes every weight as the zero
-   level (index 7).
+   level (index 7).  When 1/c overflows fp32 (c below ~2.9e-39), v is +inf or
+   -inf (codes 15 and 0 by the count rule) and a zero weight gives NaN, which
+   is encoded as the zero level (7): a zero weight always maps to the exact
+   zero level.
 R4 Packing: element 2i of a row goes to the low nibble of byte i, 2i+1 to the
    high nibble; blocks are 64 consecutive weights in row-major order.
 R5 Double quantization: one fp32 mean per tensor (pairwise fp64 sum of all
@@ -160,9 +163,12 @@ def encode(W: np.ndarray, c: np.ndarray) -> np.ndarray:
     blocks = W.reshape(-1, BLOCK)
     codes = np.full(blocks.shape, ZERO_INDEX, dtype=np.uint8)
     nz = c > 0
-    recip = fl32(1.0 / c[nz])                       # fl32(1 / c_b)
-    v = fl32(blocks[nz] * recip[:, None])           # fl32(w * r_b)
-    codes[nz] = nearest_level(v)
+    with np.errstate(over="ignore", invalid="ignore"):
+        recip = fl32(1.0 / c[nz])                   # fl32(1 / c_b), inf for tiny c_b
+        v = fl32(blocks[nz] * recip[:, None])       # fl32(w * r_b)
+    enc = nearest_level(v)
+    enc[np.isnan(v)] = ZERO_INDEX                   # 0 * inf: a zero weight
+    codes[nz] = enc
     return codes.reshape(rows, cols)
 
 

@@ -56,6 +56,8 @@ def test_degenerate_blocks_bit_exact(cuda_lib):
     W[2, 64:128] = np.float32(1e-40)                 # subnormal block
     W[3, 128:192] = np.linspace(-1e-38, 1e-38, 64, dtype=np.float32)
     W[4, :64] = 1e4 * np.sign(W[4, :64])             # large magnitude
+    W[6, :64] = 0.0                                  # absmax whose reciprocal overflows
+    W[6, :5] = [2e-39, -2e-39, 0.0, -0.0, 1e-39]
     W[5, 3] = -0.0
     w = _check_quant(cuda_lib, torch.from_numpy(W))
     codes = w.codes.cpu().numpy()

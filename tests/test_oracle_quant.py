@@ -243,3 +243,16 @@ def test_quantize_rows_equals_full_quantize_rows():
     d_full = nf4.dequantize(full["codes"], full["q8"], full["step2"], full["mean"])
     d_sub = nf4.dequantize(sub["codes"], sub["q8"], sub["step2"], sub["mean"], blocks=sub["blocks"])
     assert np.array_equal(d_sub, d_full[rows])
+
+
+def test_reciprocal_overflow_block():
+    """Absmax below ~2.9e-39: 1/c overflows to inf; nonzero weights saturate to
+    the extreme levels by sign and zero weights stay at the zero level."""
+    W = np.zeros((1, 64), dtype=np.float32)
+    W[0, :4] = [2e-39, -2e-39, 0.0, -0.0]
+    W[0, 4] = 1e-39
+    q = nf4.quantize(W)
+    assert q["absmax"][0] == np.float32(2e-39)
+    assert list(q["codes"][0, :5]) == [15, 0, 7, 7, 15]
+    assert np.all(q["codes"][0, 5:] == 7)
+
