@@ -139,14 +139,29 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D bf16 row-major [rows, cols] tensor, box {64 cols, 128 rows}, 128B swizzle,
 // out-of-range elements read as zero.
-bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows = 128) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D byte tensor [rows, cols] (packed NF4 codes, cols = in / 2), box
+// {128 bytes, 256 rows}, 128B swizzle, out-of-range bytes read as zero.
+bool make_tmap_codes(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(qnf4::kGvStageK / 2), static_cast<cuuint32_t>(qnf4::kGvRows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -186,15 +201,17 @@ struct GemvPlan {
 
 int gemv_ctas_per_sm() {
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel, qnf4::kGvThreads, qnf4::kGvSmem) !=
-          cudaSuccess ||
+  cudaFuncSetAttribute(qnf4::nf4_gemv_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       qnf4::kGvSmem);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel<true, true>, qnf4::kGvThreads,
+                                                    qnf4::kGvSmem) != cudaSuccess ||
       n < 1)
-    n = 2;
+    n = 1;
   return n;
 }
 
-// Persistent grid (every CTA resident at once) splitting the (128-row tile x
-// 128-column unit) sequence evenly; local_tiles bounds the tiles one CTA's
+// Persistent grid (every CTA resident at once) splitting the (256-row tile x
+// 256-column unit) sequence evenly; local_tiles bounds the tiles one CTA's
 // range touches.
 GemvPlan gemv_plan(int64_t in, int64_t out) {
   GemvPlan p{};
@@ -531,11 +548,9 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
     qnf4::GemvArgs g{};
-    g.codes = w->codes;
     g.q8 = w->q8;
     g.step2 = w->step2;
     g.mean = w->mean;
-    g.x = x;
     g.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rowwise_ws(M, in, r));
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
@@ -543,12 +558,19 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
     g.n_st = p.n_st;
     g.n_units = p.n_units;
     g.local_tiles = p.local_tiles;
+    g.timeout_ns = g_timeout_ns.load();
     g.L = tables().L;
-    QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::nf4_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        qnf4::kGvSmem));
+    CUtensorMap tm_codes, tm_x;
+    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)) ||
+        !make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(M), static_cast<uint64_t>(in), M > 8 ? 16 : 8))
+      return QLORA_ERR_CUDA;
     {
       LaunchTimer lt_("gemv", st);
-      qnf4::nf4_gemv_kernel<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(g);
+      const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
+      auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
+                         : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
+      QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qnf4::kGvSmem));
+      kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
     const int64_t n_el = M * out;

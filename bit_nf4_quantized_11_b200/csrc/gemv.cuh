@@ -1,51 +1,69 @@
 // gemv.cuh -- few-token (M <= 16) QLoRA forward: streaming NF4 GEMV.
 //
 // With 1..16 tokens the layer is bound by streaming the packed weight from
-// HBM (0.52 byte per weight), so the kernel is organised around that stream.
-// The work is (row tile of 128 weight rows) x (stage of 128 K columns)
-// units, ordered tile-major; a persistent grid sized to the resident capacity
-// splits the unit sequence evenly, so every CTA streams the same number of
-// bytes whatever the shape.  Each warp owns 16 rows of the current tile (the
-// 16-row operand of a warp-level bf16 MMA); per unit a thread holds, for rows
-// g and g+8, 32 consecutive codes (16 bytes, always inside one 64-weight
-// block) and keeps kGvPF units in flight in registers, across tile
-// boundaries.  Nibble pairs are decoded through a 256-entry table of bf16
-// level pairs in shared memory (one copy per lane, so lookups never conflict)
-// and scaled by the block's double-quantized scale with one packed bf16
-// multiply; activations are read through L1.  The MMA's K order is permuted
-// consistently for both operands: step i of a unit takes physical columns
-// 32q + 4i .. 32q + 4i + 3 for quad lane q.  Where a CTA's range starts or
-// ends inside a tile it writes an fp32 partial of that tile; the finalize
-// kernel adds a tile's partials in CTA order and the LoRA branch us . B^T
-// ("QLoRA", llm-compass, 方法与公式: h = dequant(W0) x + (alpha/r) B A x).
+// HBM (0.52 byte per weight), so the kernel is organised around that stream
+// and around the issue and load/store-unit budget per weight it leaves.  The
+// work is (row tile of 256 weight rows) x (unit of 256 K columns = four
+// 64-weight blocks) units, ordered tile-major; a persistent grid of one CTA
+// per SM splits the unit sequence evenly, so every CTA streams the same
+// number of bytes whatever the shape.
 //
-// The weight operand here is bf16(bf16(level) * bf16(c_hat)) rather than the
-// exactly rounded bf16(level * c_hat) of the GEMM path: a relative difference
-// of a few 2^-9 per weight, far inside the output tolerance, bought to keep
-// the decode at ~2 instructions per weight.
+// Per unit, one thread issues two TMA loads into a ring of shared-memory
+// stages: the 256 x 128-byte code tile and the 8- (or 16-) token x 256-column
+// activation tile, both with 128-byte swizzle so that the reads below are
+// bank-conflict free.  16 warps own 16 rows each (the 16-row operand of a
+// warp-level bf16 MMA); per unit a thread reads, for rows g and g+8, 16
+// consecutive codes of each of the four blocks, and its warp releases the
+// code part of the stage as soon as they are in registers.  Second-level
+// scale codes (four per row and unit) are fetched one unit ahead, group
+// steps are cached.
+//
+// Each MMA step covers 16 columns of ONE block for all four quad lanes: step
+// s of block j takes columns 64j + 16q + 4s .. +3 for quad lane q, in the
+// same permuted K order for weights and activations.  A block's four steps
+// accumulate into a fresh fp32 tile that is then added to the running sum
+// times the block's exact fp32 scale c_hat (rows g and g+8 each with their
+// own), so the MMA's weight operand is bf16(level) -- the exactly rounded
+// level -- and the scale costs nothing per weight.  (The GEMM path instead
+// rounds bf16(level * c_hat) per weight; the two differ by at most 2^-9
+// relative per weight, far inside the output tolerance.)
+//
+// Decoding is one byte permute and one shared load per nibble pair: the
+// 256-entry table of bf16 level pairs has one 256-byte row per byte value,
+// with one 4-byte copy per lane in its first 128 bytes (so lookups never
+// conflict), and sits on a 64 KB boundary of the shared window, so that a
+// single prmt assembles (window bits 16-17 | byte << 8 | lane * 4), the
+// complete shared address.  Where a CTA's range starts or ends inside a tile
+// it writes an fp32 partial of that tile; the finalize kernel adds a tile's
+// partials in CTA order and the LoRA branch us . B^T ("QLoRA", llm-compass,
+// 方法与公式: h = dequant(W0) x + (alpha/r) B A x).
 #pragma once
 
 #include "common.cuh"
 
 namespace qnf4 {
 
-constexpr int kGvThreads = 256;          // 8 warps x 16 rows
-constexpr int kGvRows = 128;             // weight rows per tile
-constexpr int kGvStageK = 128;           // K columns per unit
-constexpr int kGvPF = 4;                 // units of codes in flight per thread
-constexpr int kGvSmem = 256 * 32 * 4;    // level-pair table, one copy per lane
+constexpr int kGvWarps = 16;
+constexpr int kGvThreads = 32 * kGvWarps;
+constexpr int kGvRows = 16 * kGvWarps;                    // weight rows per tile (256)
+constexpr int kGvStageK = 256;                            // K columns per unit (four blocks)
+constexpr int kGvStages = 3;                              // ring of unit tiles (2 in flight)
+constexpr int kGvCodeBytes = kGvRows * kGvStageK / 2;     // 32 KB
+constexpr int kGvXBox = 64;                               // activation box: 64 columns x tokens
+constexpr int kGvStageBytes = kGvCodeBytes + 16 * kGvStageK * 2;   // + up to 16 tokens x 256 columns
+constexpr int kGvLutBytes = 256 * 256;                    // 256 rows of 256 bytes
+constexpr int kGvSmem = 220 * 1024;                       // table on a 64 KB boundary + stages around it
 
 struct GemvArgs {
-  const uint8_t* codes;
   const int8_t* q8;
   const float* step2;
   const float* mean;
-  const uint16_t* x;       // [M, in]
   float* part;             // [ctas][local_tiles][M][kGvRows]
   int M, in, out;
-  int n_st;                // units per tile = ceil(in / 128)
+  int n_st;                // units per tile = ceil(in / 256)
   int64_t n_units;         // tiles * n_st
   int local_tiles;         // partial tiles reserved per CTA
+  uint64_t timeout_ns;     // bound of every pipeline wait
   Levels L;
 };
 
@@ -54,130 +72,283 @@ __host__ __device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t n
   return c * n / p;
 }
 
-struct GvStage {
-  uint4 c[2];        // codes of rows g and g+8
-  int q[2];          // second-level codes of their blocks
-  float st[2];       // steps of their groups
-};
+// Register-only MMAs and table loads without `volatile`, so that the
+// compiler may interleave the lookups of one step with the MMA of the
+// previous one.  Every table address derives from a value produced after the
+// barrier that publishes the table (a volatile move).
+__device__ __forceinline__ void gv_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-__global__ void __launch_bounds__(kGvThreads) nf4_gemv_kernel(const GemvArgs a) {
-  extern __shared__ __align__(16) uint32_t s_lut[];                 // [256][32]
+// d = A B with a zero accumulator input.
+__device__ __forceinline__ void gv_mma_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
+__device__ __forceinline__ uint32_t gv_lds(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Stage reads: volatile, so they stay after the pipeline wait.
+__device__ __forceinline__ uint2 gv_lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint4 gv_lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+// Byte offset, in a tile of 128-byte rows written with 128-byte swizzle, of
+// the 16-byte chunk c of row `row` (chunk index XOR row % 8) plus `half` * 8.
+__device__ __forceinline__ uint32_t gv_swz128(int row, int c, int half) {
+  return static_cast<uint32_t>(row * 128 + (((c ^ row) & 7) << 4) + half * 8);
+}
+
+// kPaired: in % 256 == 0, so every unit holds four whole blocks whose index
+// run starts at a multiple of 4 (one aligned 32-bit load of their q8 codes,
+// one group step for all four).  kTwoTok: 9..16 tokens, a second 8-token MMA
+// tile.
+template <bool kPaired, bool kTwoTok>
+__global__ void __launch_bounds__(kGvThreads, 1)
+    nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                    const GemvArgs a) {
+  constexpr int XR = kTwoTok ? 16 : 8;                               // token rows of the activation box
+  constexpr uint32_t kTxBytes = kGvCodeBytes + 4 * kGvXBox * 2 * XR;
+  extern __shared__ __align__(1024) uint8_t s_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kGvStages], empty_bar[kGvStages];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, q = lane & 3;
-  const int n_tok_tiles = (a.M + 7) / 8;                            // 1 or 2
   const int64_t u_begin = gemv_unit_begin(blockIdx.x, a.n_units, gridDim.x);
   const int64_t u_end = gemv_unit_begin(blockIdx.x + 1, a.n_units, gridDim.x);
   if (u_begin >= u_end) return;                                     // CTA-uniform
+  const int n_local = static_cast<int>(u_end - u_begin);
   const int t_first = static_cast<int>(u_begin / a.n_st);
+  const int st_first = static_cast<int>(u_begin - static_cast<int64_t>(t_first) * a.n_st);
 
+  // table on the first 64 KB boundary inside s_raw; stages (1024-aligned)
+  // in the room below it first, then above it
+  const uint32_t raw = smem_u32(s_raw), raw_end = raw + kGvSmem;
+  const uint32_t lut = (raw + 0xFFFFu) & ~0xFFFFu;
+  const uint32_t low = (raw + 1023u) & ~1023u;
+  const int n_low = lut >= low + kGvStageBytes ? static_cast<int>((lut - low) / kGvStageBytes) : 0;
+  const uint32_t high = lut + kGvLutBytes;
+  if (lut + kGvLutBytes > raw_end || lut >= (1u << 24) ||
+      (n_low < kGvStages && high + (kGvStages - n_low) * kGvStageBytes > raw_end)) {   // CTA-uniform
+    if (threadIdx.x == 0) raise_device_error(3);
+    return;
+  }
+  auto stage_addr = [&](int s) -> uint32_t {
+    return s < n_low ? low + s * kGvStageBytes : high + (s - n_low) * kGvStageBytes;
+  };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGvStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kGvWarps);
+    }
+    fence_mbar_init();
+  }
   for (int e = threadIdx.x; e < 256 * 32; e += kGvThreads) {
-    const int b = e >> 5;
-    s_lut[e] = pack_bf16x2_rn(a.L.v[b & 15], a.L.v[b >> 4]);
+    const int b = e >> 5, l = e & 31;
+    const uint32_t v = pack_bf16x2_rn(a.L.v[b & 15], a.L.v[b >> 4]);
+    asm volatile("st.shared.u32 [%0], %1;" :: "r"(lut + b * 256 + l * 4), "r"(v) : "memory");
   }
   __syncthreads();
 
-  const int64_t row_bytes = a.in / 2;
-  const int64_t row_blocks = a.in / 64;
-  const float mu = __ldg(a.mean);
-  const int row_in_tile0 = warp * 16 + g;
-
-  // (tile, unit-in-tile) of the next unit to load, advanced one unit per load
-  int64_t u_ld = u_begin;
-  int t_ld = t_first;
-  int st_ld = static_cast<int>(u_begin - static_cast<int64_t>(t_first) * a.n_st);
-  auto load = [&](GvStage& d) {
-    d.c[0] = d.c[1] = make_uint4(0, 0, 0, 0);
-    d.q[0] = d.q[1] = 0;
-    d.st[0] = d.st[1] = 0.f;
-    const bool live = u_ld < u_end;
-    const int t = t_ld, st = st_ld;
-    ++u_ld;
-    if (++st_ld == a.n_st) { st_ld = 0; ++t_ld; }
-    if (!live) return;
-    const int col = st * kGvStageK + 32 * q;
-    if (col >= a.in) return;                                         // half unit (in % 128 == 64)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = t * kGvRows + row_in_tile0 + 8 * h;
-      if (r < a.out) {
-        d.c[h] = ld_stream_v4(a.codes + static_cast<int64_t>(r) * row_bytes + col / 2);
-        const int64_t b = static_cast<int64_t>(r) * row_blocks + col / 64;
-        d.q[h] = __ldg(a.q8 + b);
-        d.st[h] = __ldg(a.step2 + b / 256);
+  // Unit tiles: thread 0 issues unit i's loads into stage i % kGvStages once
+  // every warp has released the unit that used that stage before.
+  const bool producer = threadIdx.x == 0;
+  int p_issued = 0, p_st = st_first, p_t = t_first;
+  bool p_ok = true;
+  auto produce_until = [&](int limit) {                            // issue loads of units < limit
+    for (; p_ok && p_issued < limit && p_issued < n_local; ++p_issued) {
+      const int s = p_issued % kGvStages;
+      if (p_issued >= kGvStages &&
+          !mbar_wait_bounded(&empty_bar[s], ((p_issued / kGvStages) + 1) & 1, a.timeout_ns)) {
+        raise_device_error(1);
+        p_ok = false;
+        break;
       }
+      const uint32_t dst = stage_addr(s);
+      mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
+      tma_load_2d(dst, &tm_codes, &full_bar[s], p_st * (kGvStageK / 2), p_t * kGvRows);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        tma_load_2d(dst + kGvCodeBytes + j * (kGvXBox * 2 * XR), &tm_x, &full_bar[s],
+                    p_st * kGvStageK + j * kGvXBox, 0);
+      if (++p_st == a.n_st) { p_st = 0; ++p_t; }
     }
   };
+  if (producer) {
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_x);
+    produce_until(kGvStages - 1);
+  }
 
-  GvStage ring[kGvPF];
+  const int g = lane >> 2, q = lane & 3;
+  uint32_t lane_key;                                                 // bytes 0 and 2 of every table address
+  asm volatile("mov.b32 %0, %1;" : "=r"(lane_key) : "r"(lut | static_cast<uint32_t>(lane * 4)) : "memory");
+  const int row_in_tile0 = warp * 16 + g;
+  const bool tok0 = g < a.M, tok1 = kTwoTok && g + 8 < a.M;
+
+  const int64_t row_blocks = a.in / 64;
+  const float mu = __ldg(a.mean);
+
+  // scale cursor: block index of row g's first block in the current unit
+  int r0 = t_first * kGvRows + row_in_tile0;                        // row g of the current tile
+  int64_t b0 = static_cast<int64_t>(r0) * row_blocks + 4 * st_first;
+  const int64_t b_wrap = kGvRows * row_blocks - 4 * static_cast<int64_t>(a.n_st);
+  const int64_t b8 = 8 * row_blocks;
+  // paired: q8 codes of the current and the next unit, cached group steps
+  uint32_t qc[2] = {0u, 0u}, qn[2] = {0u, 0u};
+  int64_t gi[2] = {-1, -1};
+  float sv[2] = {0.f, 0.f};
+  if (kPaired) {
 #pragma unroll
-  for (int i = 0; i < kGvPF; ++i) load(ring[i]);
+    for (int h = 0; h < 2; ++h)
+      if (r0 + 8 * h < a.out) qn[h] = __ldg(reinterpret_cast<const uint32_t*>(a.q8 + b0 + h * b8));
+  }
 
   float acc[2][4];
 #pragma unroll
   for (int j = 0; j < 2; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  const uint32_t lut_lane = smem_u32(s_lut) + lane * 4;
-  const bool tok0 = g < a.M, tok1 = g + 8 < a.M;
-  const uint16_t* x0 = a.x + static_cast<int64_t>(tok0 ? g : 0) * a.in + 32 * q;
-  const uint16_t* x1 = a.x + static_cast<int64_t>(tok1 ? g + 8 : 0) * a.in + 32 * q;
 
-  int t = t_first;                                                  // tile / unit of the unit computed
-  int st = static_cast<int>(u_begin - static_cast<int64_t>(t_first) * a.n_st);
-  for (int64_t u0 = u_begin; u0 < u_end; u0 += kGvPF) {
+  int t = t_first, st = st_first;
+  for (int i = 0; i < n_local; ++i) {
+    const int s = i % kGvStages;
+    const uint32_t sb = stage_addr(s);
+    const bool ok = mbar_wait_bounded(&full_bar[s], (i / kGvStages) & 1, a.timeout_ns);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {                              // warp-uniform give-up
+      if (lane == 0) raise_device_error(1);
+      break;
+    }
+    uint2 cg[4], ch[4];
 #pragma unroll
-    for (int k = 0; k < kGvPF; ++k) {
-      const int64_t u = u0 + k;
-      if (u < u_end) {
-        const GvStage cur = ring[k];
-        load(ring[k]);
-        const int col = st * kGvStageK;
-        const __nv_bfloat162 s0 = __float2bfloat162_rn(block_scale(cur.q[0], cur.st[0], mu));
-        const __nv_bfloat162 s1 = __float2bfloat162_rn(block_scale(cur.q[1], cur.st[1], mu));
-        const bool colv = col + 32 * q < a.in;
-        const uint32_t w0[4] = {cur.c[0].x, cur.c[0].y, cur.c[0].z, cur.c[0].w};
-        const uint32_t w1[4] = {cur.c[1].x, cur.c[1].y, cur.c[1].z, cur.c[1].w};
+    for (int j = 0; j < 4; ++j) {
+      cg[j] = gv_lds64(sb + gv_swz128(row_in_tile0, 2 * j + (q >> 1), q & 1));
+      ch[j] = gv_lds64(sb + gv_swz128(row_in_tile0 + 8, 2 * j + (q >> 1), q & 1));
+    }
+
+    const int col0 = st * kGvStageK;
+    const bool last_in_tile = st == a.n_st - 1;
+
+    // block scales of rows g and g+8; the next unit's q8 codes
+    float sc[2][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {          // k16 steps: physical columns 32q + 4i .. +3
-          // activations of this step: 4 consecutive columns per token row (L1 hits)
-          uint2 xa = make_uint2(0, 0), xb = make_uint2(0, 0);
-          if (tok0 && colv) xa = __ldg(reinterpret_cast<const uint2*>(x0 + col + 4 * i));
-          if (tok1 && colv) xb = __ldg(reinterpret_cast<const uint2*>(x1 + col + 4 * i));
-          const int word = i >> 1, sh = (i & 1) * 16;
-          uint32_t e0, e1, e2, e3;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e0) : "r"(lut_lane + ((w0[word] >> sh) & 0xFFu) * 128));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e1) : "r"(lut_lane + ((w0[word] >> (sh + 8)) & 0xFFu) * 128));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e2) : "r"(lut_lane + ((w1[word] >> sh) & 0xFFu) * 128));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(e3) : "r"(lut_lane + ((w1[word] >> (sh + 8)) & 0xFFu) * 128));
-          __nv_bfloat162 p0 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&e0), s0);
-          __nv_bfloat162 p1 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&e2), s1);
-          __nv_bfloat162 p2 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&e1), s0);
-          __nv_bfloat162 p3 = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&e3), s1);
-          const uint32_t a0 = *reinterpret_cast<uint32_t*>(&p0);   // row g,   columns 4i, 4i+1
-          const uint32_t a1 = *reinterpret_cast<uint32_t*>(&p1);   // row g+8, columns 4i, 4i+1
-          const uint32_t a2 = *reinterpret_cast<uint32_t*>(&p2);   // row g,   columns 4i+2, 4i+3
-          const uint32_t a3 = *reinterpret_cast<uint32_t*>(&p3);   // row g+8, columns 4i+2, 4i+3
-          mma_bf16_16816(acc[0], a0, a1, a2, a3, xa.x, xa.y);
-          if (n_tok_tiles > 1) mma_bf16_16816(acc[1], a0, a1, a2, a3, xb.x, xb.y);
+    for (int h = 0; h < 2; ++h) {
+      const int64_t b = b0 + h * b8;
+      const bool row_ok = r0 + 8 * h < a.out;
+      if (kPaired) {
+        qc[h] = qn[h];
+        const int64_t b_next = last_in_tile ? b + b_wrap + 4 : b + 4;
+        const bool next_ok = last_in_tile ? r0 + kGvRows + 8 * h < a.out : row_ok;
+        if (next_ok && i + 1 < n_local) qn[h] = __ldg(reinterpret_cast<const uint32_t*>(a.q8 + b_next));
+        const int64_t gidx = b >> 8;
+        if (row_ok && gidx != gi[h]) {
+          sv[h] = __ldg(a.step2 + gidx);
+          gi[h] = gidx;
         }
-        // end of this CTA's part of tile t: write the partial and restart
-        if (st == a.n_st - 1 || u == u_end - 1) {
-          float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * a.local_tiles + (t - t_first)) * a.M) * kGvRows;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
+        for (int j = 0; j < 4; ++j)
+          sc[h][j] = block_scale(static_cast<int8_t>((qc[h] >> (8 * j)) & 0xFFu), sv[h], mu);
+      } else {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int tk = 8 * j + 2 * q + hh;
-              if (tk < a.M) {
-                dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0] = acc[j][hh];
-                dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0 + 8] = acc[j][2 + hh];
-              }
-            }
-            acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-          }
+        for (int j = 0; j < 4; ++j) {
+          const bool live = row_ok && col0 + 64 * j < a.in;
+          const int qv = live ? __ldg(a.q8 + b + j) : 0;
+          const float sj = live ? __ldg(a.step2 + ((b + j) >> 8)) : 0.f;
+          sc[h][j] = block_scale(qv, sj, mu);
         }
-        if (++st == a.n_st) { st = 0; ++t; }
       }
     }
+
+    const uint32_t xs = sb + kGvCodeBytes;
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      if (kPaired || blk == 0 || col0 + 64 * blk < a.in) {
+        // activations: 16 consecutive columns 64 blk + 16q .. +15 of token rows g, g+8
+        const uint32_t xb_ = xs + blk * (kGvXBox * 2 * XR);
+        uint4 xa0 = make_uint4(0, 0, 0, 0), xa1 = xa0, xc0 = xa0, xc1 = xa0;
+        if (tok0) {
+          xa0 = gv_lds128(xb_ + gv_swz128(g, 2 * q, 0));
+          xa1 = gv_lds128(xb_ + gv_swz128(g, 2 * q + 1, 0));
+        }
+        if (tok1) {
+          xc0 = gv_lds128(xb_ + gv_swz128(g + 8, 2 * q, 0));
+          xc1 = gv_lds128(xb_ + gv_swz128(g + 8, 2 * q + 1, 0));
+        }
+        const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+        const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
+        const uint32_t wg[2] = {cg[blk].x, cg[blk].y}, wh[2] = {ch[blk].x, ch[blk].y};
+        float pb[2][4];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {     // columns 64 blk + 16q + 4 s4 .. +3: bytes 2 s4, 2 s4 + 1
+          const uint32_t sel_lo = 0x7604u | ((2 * (s4 & 1)) << 4);
+          const uint32_t sel_hi = 0x7604u | ((2 * (s4 & 1) + 1) << 4);
+          const uint32_t e0 = gv_lds(prmt(wg[s4 >> 1], lane_key, sel_lo));
+          const uint32_t e1 = gv_lds(prmt(wh[s4 >> 1], lane_key, sel_lo));
+          const uint32_t e2 = gv_lds(prmt(wg[s4 >> 1], lane_key, sel_hi));
+          const uint32_t e3 = gv_lds(prmt(wh[s4 >> 1], lane_key, sel_hi));
+          // a0: row g columns +0,+1; a1: row g+8 same; a2, a3: columns +2,+3
+          if (s4 == 0) {
+            gv_mma_z(pb[0], e0, e1, e2, e3, xa[0], xa[1]);
+            if (kTwoTok) gv_mma_z(pb[1], e0, e1, e2, e3, xc[0], xc[1]);
+          } else {
+            gv_mma(pb[0], e0, e1, e2, e3, xa[2 * s4], xa[2 * s4 + 1]);
+            if (kTwoTok) gv_mma(pb[1], e0, e1, e2, e3, xc[2 * s4], xc[2 * s4 + 1]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < (kTwoTok ? 2 : 1); ++j) {
+          acc[j][0] = fmaf(pb[j][0], sc[0][blk], acc[j][0]);
+          acc[j][1] = fmaf(pb[j][1], sc[0][blk], acc[j][1]);
+          acc[j][2] = fmaf(pb[j][2], sc[1][blk], acc[j][2]);
+          acc[j][3] = fmaf(pb[j][3], sc[1][blk], acc[j][3]);
+        }
+      }
+    }
+    // the stage (codes and activations) is no longer read by this warp
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if (producer) produce_until(i + kGvStages);                     // refill the stage of unit i - 1
+
+    // end of this CTA's part of tile t: write the partial and restart
+    if (last_in_tile || i == n_local - 1) {
+      float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * a.local_tiles + (t - t_first)) * a.M) * kGvRows;
+#pragma unroll
+      for (int j = 0; j < (kTwoTok ? 2 : 1); ++j) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int tk = 8 * j + 2 * q + hh;
+          if (tk < a.M) {
+            dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0] = acc[j][hh];
+            dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0 + 8] = acc[j][2 + hh];
+          }
+        }
+        acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      }
+    }
+    b0 += 4;
+    if (++st == a.n_st) { st = 0; ++t; r0 += kGvRows; b0 += b_wrap; }
   }
+  // leave no copy in flight when the CTA exits (only on a give-up path can
+  // issued loads still be unconsumed): wait, bounded, for the last ones
+  if (producer)
+    for (int j = p_issued > kGvStages ? p_issued - kGvStages : 0; j < p_issued; ++j)
+      if (!mbar_wait_bounded(&full_bar[j % kGvStages], (j / kGvStages) & 1, a.timeout_ns)) raise_device_error(1);
 }
 
 // h[m][o] = bf16( sum of the partials of o's tile, in CTA order

@@ -75,6 +75,14 @@ def test_few_token_gemv(cuda_lib, M):
     _run(cuda_lib, M, 1024, 768, 16, 32.0, seed=M, backward=True)
 
 
+@pytest.mark.parametrize("M,n_in,n_out", [(3, 576, 320), (12, 192, 448), (1, 64, 64), (16, 64, 1088),
+                                           (7, 4160, 576)])
+def test_few_token_ragged(cuda_lib, M, n_in, n_out):
+    # K with a half 128-column unit (in % 128 == 64), a partial last row tile,
+    # a single unit, and more row tiles than a CTA range spans
+    _run(cuda_lib, M, n_in, n_out, 8, 16.0, seed=100 + M, backward=False)
+
+
 def test_zero_adapter_is_plain_quantized_matmul(cuda_lib):
     """B = 0: h equals x dequant(W0)^T, dA = 0 exactly."""
     q = cuda_lib
