@@ -34,7 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from bit_nf4_quantized_11_b200 import synth, workloads  # noqa: E402
+from bit_nf4_quantized_11_b200 import dp, synth, workloads  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 quant/GEMV GB/s, % of B200 roofline"
 L2_BYTES = 126 * 2 ** 20
@@ -199,8 +199,7 @@ def run_ours(args, world, rank, local):
     h = torch.empty(M, n_out, dtype=torch.bfloat16, device=dev)
     us = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
     dx = torch.empty(M, n_in, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(r, n_in, dtype=torch.float32, device=dev)
-    dB = torch.empty(n_out, r, dtype=torch.float32, device=dev)
+    grads, dA, dB = dp.adapter_grad_buffers(r, n_in, n_out, dev)
     ws_f = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_FWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_BWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
 
@@ -208,9 +207,8 @@ def run_ours(args, world, rank, local):
         c = copies[i % len(copies)]
         q.linear_fwd(c["x"], c["w"], c["A"], c["B"], alpha, h=h, us=us, workspace=ws_f)
         q.linear_bwd(c["dh"], c["x"], us, c["w"], c["A"], c["B"], alpha, dx=dx, dA=dA, dB=dB, workspace=ws_b)
-        if world > 1:                       # data-parallel adapter-gradient sync
-            torch.distributed.all_reduce(dA)
-            torch.distributed.all_reduce(dB)
+        if world > 1:                       # data-parallel adapter-gradient sum
+            dp.allreduce_adapter_grads(grads)
 
     for i in range(args.warmup):
         step(i)
@@ -309,15 +307,15 @@ def measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev):
     dA_host = torch.empty(r, n_in, dtype=torch.float32).pin_memory()
     dB_host = torch.empty(n_out, r, dtype=torch.float32).pin_memory()
     n = max(10, min(100, args.steps // 10))
+    grads, dA, dB = dp.adapter_grad_buffers(r, n_in, n_out, dev)
 
     def step():
         x.copy_(xh, non_blocking=True)
         dh.copy_(dhh, non_blocking=True)
         h, us = q.linear_fwd(x, c["w"], c["A"], c["B"], alpha)
-        dx, dA, dB = q.linear_bwd(dh, x, us, c["w"], c["A"], c["B"], alpha)
+        dx, _, _ = q.linear_bwd(dh, x, us, c["w"], c["A"], c["B"], alpha, dA=dA, dB=dB)
         if world > 1:
-            torch.distributed.all_reduce(dA)
-            torch.distributed.all_reduce(dB)
+            dp.allreduce_adapter_grads(grads)
         h_host.copy_(h, non_blocking=True)
         dx_host.copy_(dx, non_blocking=True)
         dA_host.copy_(dA, non_blocking=True)

@@ -52,7 +52,7 @@ constexpr int kGvCodeBytes = kGvRows * kGvStageK / 2;     // 32 KB
 constexpr int kGvXBox = 64;                               // activation box: 64 columns x tokens
 constexpr int kGvStageBytes = kGvCodeBytes + 16 * kGvStageK * 2;   // + up to 16 tokens x 256 columns
 constexpr int kGvLutBytes = 256 * 256;                    // 256 rows of 256 bytes
-constexpr int kGvSmem = 220 * 1024;                       // table on a 64 KB boundary + stages around it
+constexpr int kGvSmem = 192 * 1024;                       // stages, then the table on the next 64 KB boundary
 
 struct GemvArgs {
   const int8_t* q8;
@@ -139,21 +139,15 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int t_first = static_cast<int>(u_begin / a.n_st);
   const int st_first = static_cast<int>(u_begin - static_cast<int64_t>(t_first) * a.n_st);
 
-  // table on the first 64 KB boundary inside s_raw; stages (1024-aligned)
-  // in the room below it first, then above it
-  const uint32_t raw = smem_u32(s_raw), raw_end = raw + kGvSmem;
-  const uint32_t lut = (raw + 0xFFFFu) & ~0xFFFFu;
-  const uint32_t low = (raw + 1023u) & ~1023u;
-  const int n_low = lut >= low + kGvStageBytes ? static_cast<int>((lut - low) / kGvStageBytes) : 0;
-  const uint32_t high = lut + kGvLutBytes;
-  if (lut + kGvLutBytes > raw_end || lut >= (1u << 24) ||
-      (n_low < kGvStages && high + (kGvStages - n_low) * kGvStageBytes > raw_end)) {   // CTA-uniform
+  // contiguous 1024-aligned stages at the start of s_raw, the table on the
+  // next 64 KB boundary of the window after them
+  const uint32_t raw = smem_u32(s_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const uint32_t lut = (sbase + kGvStages * kGvStageBytes + 0xFFFFu) & ~0xFFFFu;
+  if (lut + kGvLutBytes > raw + kGvSmem || lut >= (1u << 24)) {     // cannot place them (CTA-uniform)
     if (threadIdx.x == 0) raise_device_error(3);
     return;
   }
-  auto stage_addr = [&](int s) -> uint32_t {
-    return s < n_low ? low + s * kGvStageBytes : high + (s - n_low) * kGvStageBytes;
-  };
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGvStages; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -182,7 +176,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         p_ok = false;
         break;
       }
-      const uint32_t dst = stage_addr(s);
+      const uint32_t dst = sbase + s * kGvStageBytes;
       mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
       tma_load_2d(dst, &tm_codes, &full_bar[s], p_st * (kGvStageK / 2), p_t * kGvRows);
 #pragma unroll
@@ -203,34 +197,45 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   asm volatile("mov.b32 %0, %1;" : "=r"(lane_key) : "r"(lut | static_cast<uint32_t>(lane * 4)) : "memory");
   const int row_in_tile0 = warp * 16 + g;
   const bool tok0 = g < a.M, tok1 = kTwoTok && g + 8 < a.M;
+  // stage-relative read offsets: codes of row g, block j (row g+8: + 1024);
+  // activation chunks 2q, 2q+1 of token g (token g+8: + 1024)
+  uint32_t coff[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) coff[j] = gv_swz128(row_in_tile0, 2 * j + (q >> 1), q & 1);
+  const uint32_t xoff0 = kGvCodeBytes + gv_swz128(g, 2 * q, 0);
+  const uint32_t xoff1 = kGvCodeBytes + gv_swz128(g, 2 * q + 1, 0);
+  constexpr uint32_t kXBlk = kGvXBox * 2 * XR;                       // bytes per activation box
 
   const int64_t row_blocks = a.in / 64;
   const float mu = __ldg(a.mean);
 
-  // scale cursor: block index of row g's first block in the current unit
-  int r0 = t_first * kGvRows + row_in_tile0;                        // row g of the current tile
-  int64_t b0 = static_cast<int64_t>(r0) * row_blocks + 4 * st_first;
+  // Block scales are computed once per (row, block) and shared through the
+  // free upper half of the table's rows: lane l of a warp handles row
+  // (l % 16) of the warp's 16 and blocks 2 (l / 16), 2 (l / 16) + 1 of the
+  // unit, writes them to its warp's 256-byte slot (rows 0-7 in table row
+  // 2 warp, rows 8-15 in 2 warp + 1, 16 bytes per row) and reads back the
+  // four scales of rows g and g+8.
+  const int srow = lane & 15, spair = lane >> 4;
+  const uint32_t s_st = lut + (2 * warp + (srow >> 3)) * 256 + 128 + (srow & 7) * 16 + spair * 8;
+  const uint32_t s_ld = lut + 2 * warp * 256 + 128 + g * 16;         // row g; row g+8: + 256
+  int rs = t_first * kGvRows + warp * 16 + srow;                    // this lane's scale row
+  const int8_t* qp = a.q8 + static_cast<int64_t>(rs) * row_blocks + 4 * st_first + 2 * spair;
   const int64_t b_wrap = kGvRows * row_blocks - 4 * static_cast<int64_t>(a.n_st);
-  const int64_t b8 = 8 * row_blocks;
-  // paired: q8 codes of the current and the next unit, cached group steps
-  uint32_t qc[2] = {0u, 0u}, qn[2] = {0u, 0u};
-  int64_t gi[2] = {-1, -1};
-  float sv[2] = {0.f, 0.f};
-  if (kPaired) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      if (r0 + 8 * h < a.out) qn[h] = __ldg(reinterpret_cast<const uint32_t*>(a.q8 + b0 + h * b8));
-  }
+  // paired: the two q8 codes of the next unit (each byte XOR 0x80), cached group step
+  uint32_t qn = 0x8080u;
+  float sv = 0.f;
+  if (kPaired && rs < a.out) qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(qp))) ^ 0x8080u;
 
   float acc[2][4];
 #pragma unroll
   for (int j = 0; j < 2; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
   int t = t_first, st = st_first;
+  int s = 0;
+  uint32_t phase = 0, sb = sbase;
+  bool new_row = true;                                               // group steps to (re)load
   for (int i = 0; i < n_local; ++i) {
-    const int s = i % kGvStages;
-    const uint32_t sb = stage_addr(s);
-    const bool ok = mbar_wait_bounded(&full_bar[s], (i / kGvStages) & 1, a.timeout_ns);
+    const bool ok = mbar_wait_bounded(&full_bar[s], phase, a.timeout_ns);
     if (!__all_sync(0xFFFFFFFFu, ok)) {                              // warp-uniform give-up
       if (lane == 0) raise_device_error(1);
       break;
@@ -238,57 +243,60 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     uint2 cg[4], ch[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      cg[j] = gv_lds64(sb + gv_swz128(row_in_tile0, 2 * j + (q >> 1), q & 1));
-      ch[j] = gv_lds64(sb + gv_swz128(row_in_tile0 + 8, 2 * j + (q >> 1), q & 1));
+      cg[j] = gv_lds64(sb + coff[j]);
+      ch[j] = gv_lds64(sb + coff[j] + 1024);
     }
 
     const int col0 = st * kGvStageK;
     const bool last_in_tile = st == a.n_st - 1;
 
-    // block scales of rows g and g+8; the next unit's q8 codes
-    float sc[2][4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t b = b0 + h * b8;
-      const bool row_ok = r0 + 8 * h < a.out;
+    // this lane's two block scales, then the eight of rows g and g+8
+    {
+      const bool row_ok = rs < a.out;
+      float s0, s1;
       if (kPaired) {
-        qc[h] = qn[h];
-        const int64_t b_next = last_in_tile ? b + b_wrap + 4 : b + 4;
-        const bool next_ok = last_in_tile ? r0 + kGvRows + 8 * h < a.out : row_ok;
-        if (next_ok && i + 1 < n_local) qn[h] = __ldg(reinterpret_cast<const uint32_t*>(a.q8 + b_next));
-        const int64_t gidx = b >> 8;
-        if (row_ok && gidx != gi[h]) {
-          sv[h] = __ldg(a.step2 + gidx);
-          gi[h] = gidx;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          sc[h][j] = block_scale(static_cast<int8_t>((qc[h] >> (8 * j)) & 0xFFu), sv[h], mu);
+        const uint32_t qc = qn;
+        const int8_t* q_next = last_in_tile ? qp + b_wrap + 4 : qp + 4;
+        const bool next_ok = last_in_tile ? rs + kGvRows < a.out : row_ok;
+        if (next_ok && i + 1 < n_local)
+          qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(q_next))) ^ 0x8080u;
+        // a unit's four blocks share one group; a group starts at a multiple of 256 blocks
+        const int64_t b_unit = (qp - a.q8) - 2 * spair;
+        if (row_ok && (new_row || (static_cast<uint32_t>(b_unit) & 255u) == 0)) sv = __ldg(a.step2 + (b_unit >> 8));
+        // exact floats of the signed codes: 2^23 + (q + 128) - (2^23 + 128)
+        const float q0 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7650u)), -8388736.0f);
+        const float q1 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7651u)), -8388736.0f);
+        s0 = __fadd_rn(__fmul_rn(q0, sv), mu);
+        s1 = __fadd_rn(__fmul_rn(q1, sv), mu);
       } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const bool live = row_ok && col0 + 64 * j < a.in;
-          const int qv = live ? __ldg(a.q8 + b + j) : 0;
-          const float sj = live ? __ldg(a.step2 + ((b + j) >> 8)) : 0.f;
-          sc[h][j] = block_scale(qv, sj, mu);
-        }
+        const int c0 = col0 + 128 * spair;
+        const bool l0 = row_ok && c0 < a.in, l1 = row_ok && c0 + 64 < a.in;
+        const int64_t b = qp - a.q8;
+        s0 = block_scale(l0 ? __ldg(qp) : 0, l0 ? __ldg(a.step2 + (b >> 8)) : 0.f, mu);
+        s1 = block_scale(l1 ? __ldg(qp + 1) : 0, l1 ? __ldg(a.step2 + ((b + 1) >> 8)) : 0.f, mu);
       }
+      asm volatile("st.shared.v2.f32 [%0], {%1, %2};" :: "r"(s_st), "f"(s0), "f"(s1) : "memory");
     }
+    __syncwarp();
+    float sc[2][4];
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(sc[0][0]), "=f"(sc[0][1]), "=f"(sc[0][2]), "=f"(sc[0][3]) : "r"(s_ld) : "memory");
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(sc[1][0]), "=f"(sc[1][1]), "=f"(sc[1][2]), "=f"(sc[1][3]) : "r"(s_ld + 256) : "memory");
+    new_row = false;
 
-    const uint32_t xs = sb + kGvCodeBytes;
 #pragma unroll
     for (int blk = 0; blk < 4; ++blk) {
       if (kPaired || blk == 0 || col0 + 64 * blk < a.in) {
         // activations: 16 consecutive columns 64 blk + 16q .. +15 of token rows g, g+8
-        const uint32_t xb_ = xs + blk * (kGvXBox * 2 * XR);
         uint4 xa0 = make_uint4(0, 0, 0, 0), xa1 = xa0, xc0 = xa0, xc1 = xa0;
         if (tok0) {
-          xa0 = gv_lds128(xb_ + gv_swz128(g, 2 * q, 0));
-          xa1 = gv_lds128(xb_ + gv_swz128(g, 2 * q + 1, 0));
+          xa0 = gv_lds128(sb + xoff0 + blk * kXBlk);
+          xa1 = gv_lds128(sb + xoff1 + blk * kXBlk);
         }
         if (tok1) {
-          xc0 = gv_lds128(xb_ + gv_swz128(g + 8, 2 * q, 0));
-          xc1 = gv_lds128(xb_ + gv_swz128(g + 8, 2 * q + 1, 0));
+          xc0 = gv_lds128(sb + xoff0 + blk * kXBlk + 1024);
+          xc1 = gv_lds128(sb + xoff1 + blk * kXBlk + 1024);
         }
         const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
         const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
@@ -341,8 +349,10 @@ __global__ void __launch_bounds__(kGvThreads, 1)
         acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
       }
     }
-    b0 += 4;
-    if (++st == a.n_st) { st = 0; ++t; r0 += kGvRows; b0 += b_wrap; }
+    qp += 4;
+    if (++st == a.n_st) { st = 0; ++t; rs += kGvRows; qp += b_wrap; new_row = true; }
+    sb += kGvStageBytes;
+    if (++s == kGvStages) { s = 0; phase ^= 1u; sb = sbase; }
   }
   // leave no copy in flight when the CTA exits (only on a give-up path can
   // issued loads still be unconsumed): wait, bounded, for the last ones
