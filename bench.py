@@ -68,10 +68,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash():
+# sources of the fused dequant GEMM kernels (the dominant kernel of the step)
+GEMM_SOURCES = ("common.cuh", "gemm_pair_sm100.cuh", "gemm_sm100.cuh")
+
+
+def source_hash(names=GEMM_SOURCES):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_nf4_quantized_11_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
