@@ -231,40 +231,39 @@ size_t gemv_ws(int64_t M, int64_t in, int64_t out) {
 
 // K splits of the row-wise rank-r product: enough CTAs (64 rows x one
 // 64-wide rank chunk x one K range each) to keep ~2 per SM streaming, with at
-// least 4 K stages (256 columns) per range.
+// least 4 K stages (256 columns) per range.  The splits of a row tile form one
+// cluster (reduced over distributed shared memory), so there are at most 8.
 int rowwise_splits(int64_t M, int64_t K, int r) {
   const int64_t tiles = cdiv(M, 64) * cdiv(r, 64);
   const int64_t n_st = K / 64;
   const int64_t want = cdiv(2 * device_sm_count(), tiles);
-  int64_t ks = std::max<int64_t>(1, std::min<int64_t>(want, n_st / 4));
+  int64_t ks = std::max<int64_t>(1, std::min<int64_t>({want, n_st / 4, 8}));
   ks = cdiv(n_st, cdiv(n_st, ks));                     // no empty split
   return static_cast<int>(ks);
 }
 
-size_t rowwise_ws(int64_t M, int64_t K, int r) {
-  const int ks = rowwise_splits(M, K, r);
-  return ks > 1 ? round256(static_cast<size_t>(ks) * M * r * 4) : 0;
+// Token chunks of the column-wise products: one cluster of at most 8 chunks
+// per 128-wide column tile, each chunk a multiple of 32 tokens.
+int col_chunk_tokens(int64_t M) {
+  const int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(qnf4::kColMaxChunks, cdiv(M, 256)));
+  return static_cast<int>(cdiv(cdiv(M, chunks), 32) * 32);
 }
 
 size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
-  size_t b = rowwise_ws(M, in, r);
-  if (M <= 16) b += gemv_ws(M, in, out);
-  return b;
+  (void)r;
+  return M <= 16 ? gemv_ws(M, in, out) : 0;
 }
 
 struct BwdWs {
-  size_t du_off, row_off, dbp_off, dap_off, total;
-  int chunks;
+  size_t du_off, total;
 };
 
 BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
+  (void)in;
+  (void)out;
   BwdWs w{};
-  w.chunks = static_cast<int>(cdiv(M, qnf4::kColChunk));
   w.du_off = 0;
-  w.row_off = w.du_off + round256(static_cast<size_t>(M) * r * 2);
-  w.dbp_off = w.row_off + rowwise_ws(M, out, r);
-  w.dap_off = w.dbp_off + round256(static_cast<size_t>(w.chunks) * out * r * 4);
-  w.total = w.dap_off + round256(static_cast<size_t>(w.chunks) * in * r * 4);
+  w.total = round256(static_cast<size_t>(M) * r * 2);
   return w;
 }
 
@@ -391,61 +390,70 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
 }
 
 template <int NT, bool kKR>
-int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int ks, int64_t M,
-                     int64_t K, int R, float scale, cudaStream_t st) {
+int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int ks, int64_t M, int64_t K, int R,
+                     float scale, cudaStream_t st) {
   using C = qnf4::RowCfg<NT, kKR>;
   auto kern = qnf4::rowwise_skinny_kernel<NT, kKR>;
   QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
   const int n_st = static_cast<int>(K / 64);
   const int sps = static_cast<int>(cdiv(n_st, ks));
-  dim3 grid(static_cast<unsigned>(cdiv(M, 64)), static_cast<unsigned>(ks), static_cast<unsigned>(cdiv(R, C::RC)));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(cdiv(M, 64)), static_cast<unsigned>(ks), static_cast<unsigned>(cdiv(R, C::RC)));
+  cfg.blockDim = dim3(qnf4::kRowThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(ks);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ks > 1 ? 1 : 0;
   {
     LaunchTimer lt_(kKR ? "lora_rowwise_du" : "lora_rowwise", st);
-    kern<<<grid, qnf4::kRowThreads, C::SMEM, st>>>(act, W, out, ks > 1 ? part : nullptr, static_cast<int>(M),
-                                                 static_cast<int>(K), R, scale, sps);
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  if (ks > 1) {
-    LaunchTimer lt_("lora_rowwise_finalize", st);
-    qnf4::rowwise_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(M * R / 4, 256), 2048)), 256, 0, st>>>(
-        part, ks, static_cast<int>(M), R, scale, out);
+    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, act, W, out, static_cast<int>(M), static_cast<int>(K), R, scale, sps));
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
 }
 
 // out[M, R] = bf16(scale * act[M, K] . W^T) with W given as [R, K] (kKR =
-// false) or as [K, R] (kKR = true); part: fp32 workspace of rowwise_ws bytes.
+// false) or as [K, R] (kKR = true).
 template <bool kKR>
-int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, float* part, int64_t M, int64_t K,
-                   int R, float scale, cudaStream_t st) {
+int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_t M, int64_t K, int R, float scale,
+                   cudaStream_t st) {
   const int ks = rowwise_splits(M, K, R);
-  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, part, ks, M, K, R, scale, st);
-  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, part, ks, M, K, R, scale, st);
-  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, part, ks, M, K, R, scale, st);
-  return launch_rowwise_t<8, kKR>(act, W, out, part, ks, M, K, R, scale, st);
+  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, ks, M, K, R, scale, st);
+  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, ks, M, K, R, scale, st);
+  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, ks, M, K, R, scale, st);
+  return launch_rowwise_t<8, kKR>(act, W, out, ks, M, K, R, scale, st);
 }
 
-// dB = dh^T us -> [out, r] and dA = du^T x -> [r, in], one launch each for the
-// partials and for the fixed-order chunk sum.
+// dB = dh^T us -> [out, r] and dA = du^T x -> [r, in] in one launch: column
+// tiles x token chunks x the two problems, chunks of a tile in one cluster.
 int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
-                      int64_t in, int64_t out, int R, float* dBp, float* dAp, int chunks, float* dB, float* dA,
-                      cudaStream_t st) {
-  const qnf4::ColProblem pb{dh, us, dBp, static_cast<int>(out), 0};
-  const qnf4::ColProblem pa{x, du, dAp, static_cast<int>(in), 1};
+                      int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st) {
+  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0};
+  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1};
   const int smem = qnf4::kColStages * qnf4::kColStageBytes;
   QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::colwise_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  dim3 grid(static_cast<unsigned>(cdiv(std::max(in, out), 128)), static_cast<unsigned>(chunks), 2);
+  const int chunk_tokens = col_chunk_tokens(M);
+  const unsigned chunks = static_cast<unsigned>(cdiv(M, chunk_tokens));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(cdiv(std::max(in, out), 128)), chunks, 2);
+  cfg.blockDim = dim3(qnf4::kColThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = chunks;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   {
     LaunchTimer lt_("lora_colwise", st);
-    qnf4::colwise_skinny_kernel<<<grid, qnf4::kColThreads, smem, st>>>(pb, pa, static_cast<int>(M), R);
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  const int64_t n_b = out * R, n_a = in * R;
-  dim3 g2(static_cast<unsigned>(std::min<int64_t>(cdiv(std::max(n_a, n_b) / 4, 256), 1024)), 2);
-  {
-    LaunchTimer lt_("sum_chunks", st);
-    qnf4::sum_chunks_kernel<<<g2, 256, 0, st>>>(dBp, dB, n_b, dAp, dA, n_a, chunks);
+    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, qnf4::colwise_skinny_kernel, pb, pa, static_cast<int>(M), R, chunk_tokens));
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
@@ -542,8 +550,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float s = alpha / static_cast<float>(r);
 
-  float* row_part = static_cast<float*>(workspace);
-  int rc = launch_rowwise<false>(x, A, us_out, row_part, M, in, r, s, st);   // us = bf16(s x A^T)
+  int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s, st);             // us = bf16(s x A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
@@ -551,7 +558,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
     g.q8 = w->q8;
     g.step2 = w->step2;
     g.mean = w->mean;
-    g.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + rowwise_ws(M, in, r));
+    g.part = static_cast<float*>(workspace);
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
@@ -601,16 +608,13 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
-  float* row_part = reinterpret_cast<float*>(base + ws.row_off);
-  float* dBp = reinterpret_cast<float*>(base + ws.dbp_off);
-  float* dAp = reinterpret_cast<float*>(base + ws.dap_off);
   const float s = alpha / static_cast<float>(r);
 
-  int rc = launch_rowwise<true>(dh, B, du, row_part, M, out, r, s, st);               // du = bf16(s dh B)
+  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                         // du = bf16(s dh B)
   if (rc != QLORA_OK) return rc;
   rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
   if (rc != QLORA_OK) return rc;
-  return launch_lora_grads(dh, us, x, du, M, in, out, r, dBp, dAp, ws.chunks, dB, dA, st);  // dB, dA
+  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st);                // dB, dA
 }
 
 int qlora_last_device_status(void* stream) {

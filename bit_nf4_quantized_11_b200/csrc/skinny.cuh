@@ -30,9 +30,34 @@ namespace qnf4 {
 // ldmatrix.trans), so neither orientation needs a transposed copy.
 // Activation rows are 128 B in shared memory with the 16-byte chunk index
 // XOR-ed by (row & 7), so every ldmatrix phase hits 8 different bank groups.
-// With one K range the result is scaled and rounded to bf16 in place;
-// otherwise fp32 partials go to part[split][row][n] for the finalize kernel.
+// With one K range the result is scaled and rounded to bf16 in place.  With
+// several, the K ranges of a row tile form one thread-block cluster along y:
+// each CTA leaves its fp32 partial tile in its own shared memory, then every
+// CTA adds up its share of the tile over distributed shared memory, partials
+// in rank order (deterministic), and scales, rounds and stores it.
 // ---------------------------------------------------------------------------
+// Sum over the CTAs of this cluster, in rank order, of the float4 at local
+// shared address `addr` of each (all loads issued before the first add).
+__device__ __forceinline__ float4 cluster_sum_f4(uint32_t addr, int ranks) {
+  float4 t[8];
+#pragma unroll
+  for (int rk = 0; rk < 8; ++rk) {
+    t[rk] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rk < ranks)
+      asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                   : "=f"(t[rk].x), "=f"(t[rk].y), "=f"(t[rk].z), "=f"(t[rk].w)
+                   : "r"(mapa_shared(addr, rk)) : "memory");
+  }
+  float4 v = t[0];
+#pragma unroll
+  for (int rk = 1; rk < 8; ++rk) {
+    if (rk < ranks) {
+      v.x += t[rk].x; v.y += t[rk].y; v.z += t[rk].z; v.w += t[rk].w;
+    }
+  }
+  return v;
+}
+
 constexpr int kRowThreads = 128;
 constexpr int kRowStages = 4;
 constexpr int kRowActBytes = 64 * 128;                  // 64 rows x 64 k bf16
@@ -49,13 +74,13 @@ struct RowCfg {
   static constexpr int W_BYTES = kKR ? 64 * W_PITCH : RCA * 128;
   static constexpr int STAGE = kRowActBytes + ((W_BYTES + 127) / 128) * 128;
   static constexpr int SMEM = kRowStages * STAGE;
+  static_assert(64 * RC * 4 <= SMEM, "partial tile must fit the stage ring");
 };
 
 template <int NT, bool kKR>
 __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
     const uint16_t* __restrict__ act, const uint16_t* __restrict__ W,
-    uint16_t* __restrict__ out, float* __restrict__ part, int M, int K, int R, float scale,
-    int stages_per_split) {
+    uint16_t* __restrict__ out, int M, int K, int R, float scale, int stages_per_split) {
   using C = RowCfg<NT, kKR>;
   extern __shared__ __align__(128) uint8_t s_row[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,84 +168,92 @@ __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
   cp_async_wait<0>();
 
   const int g = lane >> 2, q = lane & 3;
+  if (gridDim.y == 1) {
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    if (j < nt) {
-      const int n = nb + 8 * j + 2 * q;
+    for (int j = 0; j < NT; ++j) {
+      if (j < nt) {
+        const int n = nb + 8 * j + 2 * q;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int m = m0 + warp * 16 + g + 8 * h;
-        if (m < M) {
-          const float v0 = acc[j][2 * h], v1 = acc[j][2 * h + 1];
-          if (part == nullptr) {
+        for (int h = 0; h < 2; ++h) {
+          const int m = m0 + warp * 16 + g + 8 * h;
+          if (m < M)
             *reinterpret_cast<uint32_t*>(out + static_cast<int64_t>(m) * R + n) =
-                pack_bf16x2_rn(v0 * scale, v1 * scale);
-          } else {
-            *reinterpret_cast<float2*>(part + (static_cast<int64_t>(blockIdx.y) * M + m) * R + n) =
-                make_float2(v0, v1);
-          }
+                pack_bf16x2_rn(acc[j][2 * h] * scale, acc[j][2 * h + 1] * scale);
         }
       }
     }
+    return;
   }
-}
 
-// out[m][n] = bf16(scale * sum_{s < splits} part[s][m][n]), splits added in
-// order; four outputs per thread (M*R is a multiple of 8).
-__global__ void __launch_bounds__(256) rowwise_finalize_kernel(
-    const float* __restrict__ part, int splits, int M, int R, float scale, uint16_t* __restrict__ out) {
-  const int64_t n4 = static_cast<int64_t>(M) * R / 4;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* p = reinterpret_cast<const float4*>(part) + e;
-#pragma unroll 4
-    for (int s = 0; s < splits; ++s) {
-      const float4 t = __ldg(p + static_cast<int64_t>(s) * n4);
-      v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
+  // cluster of the row tile's K ranges: partial tile [64 rows][RC] in shared memory
+  __syncthreads();                                                   // every warp is done with the stages
+  float* red = reinterpret_cast<float*>(s_row);
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      *reinterpret_cast<float2*>(red + (warp * 16 + g + 8 * h) * C::RC + 8 * j + 2 * q) =
+          make_float2(acc[j][2 * h], acc[j][2 * h + 1]);
+  cluster_sync_all();
+  {
+    // every CTA of the cluster reduces and stores its share of the tile
+    const int ks = static_cast<int>(gridDim.y), rank = static_cast<int>(cluster_ctarank());
+    constexpr int n4 = 64 * C::RC / 4;
+    const uint32_t red_addr = smem_u32(red);
+    for (int e = rank * n4 / ks + threadIdx.x; e < (rank + 1) * n4 / ks; e += kRowThreads) {
+      const int row = e / (C::RC / 4), c4 = e % (C::RC / 4);
+      const float4 v = cluster_sum_f4(red_addr + e * 16, ks);
+      const int m = m0 + row, n = nb + 4 * c4;
+      if (m < M && n < R)
+        *reinterpret_cast<uint2*>(out + static_cast<int64_t>(m) * R + n) =
+            make_uint2(pack_bf16x2_rn(v.x * scale, v.y * scale), pack_bf16x2_rn(v.z * scale, v.w * scale));
     }
-    reinterpret_cast<uint2*>(out)[e] =
-        make_uint2(pack_bf16x2_rn(v.x * scale, v.y * scale), pack_bf16x2_rn(v.z * scale, v.w * scale));
   }
+  cluster_sync_all();                                                // partials stay until all are read
 }
 
 // ---------------------------------------------------------------------------
 // col-wise skinny GEMM (reduction over tokens), both backward problems in one
-// launch (blockIdx.z): dB = dh^T us and dA^T = x^T du.  CTA = 4 warps on a
-// 128-wide p tile and a chunk of kColChunk tokens; 32-token steps are staged
-// in shared memory with cp.async in a kColStages-deep ring (rows padded to an
-// odd number of 16-byte units so ldmatrix.trans is conflict free) and consumed
-// with ldmatrix.trans + mma.  Each warp owns 32 p rows x 64 n columns.
-// Partials are written in the orientation of the final output: [c][p][n] for
-// dB (out, r) and [c][n][p] for dA (r, in), so the chunk sum is elementwise.
+// launch (blockIdx.z): dB = dh^T us and dA = du^T x.  CTA = 4 warps on a
+// 128-wide p tile and one token chunk; 32-token steps are staged in shared
+// memory with cp.async in a kColStages-deep ring (rows padded to an odd number
+// of 16-byte units so ldmatrix.trans is conflict free) and consumed with
+// ldmatrix.trans + mma.  Each warp owns 32 p rows x 64 n columns.  The token
+// chunks of a p tile form one thread-block cluster along y (at most 8): each
+// CTA leaves its fp32 partial tile in shared memory, in the orientation of the
+// output ([p][n] for dB [out, r], [n][p] for dA [r, in]), then every CTA adds
+// up its share of the tile over distributed shared memory, partials in rank
+// order (deterministic), and stores it.
 // ---------------------------------------------------------------------------
-constexpr int kColChunk = 512;
+constexpr int kColMaxChunks = 8;
 constexpr int kColThreads = 128;
 constexpr int kColStages = 4;
 constexpr int kActStride = 128 * 2 + 16;   // bytes per staged act row (17 x 16 B)
 constexpr int kUStride = 64 * 2 + 16;      // bytes per staged u row   (9 x 16 B)
 constexpr int kColStageBytes = 32 * kActStride + 32 * kUStride;
+static_assert(128 * 64 * 4 <= kColStages * kColStageBytes, "partial tile must fit the stage ring");
 
 struct ColProblem {
   const uint16_t* act;   // [M, P]
   const uint16_t* u;     // [M, R]
-  float* part;           // [chunks][P][R] or [chunks][R][P]
+  float* out;            // [P][R] (dB) or [R][P] (dA)
   int P;
-  int n_major;           // 1: partial layout [c][n][p]
+  int n_major;           // 1: output layout [n][p]
 };
 
 __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem prob0, ColProblem prob1,
-                                                                     int M, int R) {
+                                                                     int M, int R, int chunk_tokens) {
   extern __shared__ __align__(128) uint8_t s_col[];
   const ColProblem pr = blockIdx.z == 0 ? prob0 : prob1;
   const int P = pr.P;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int p0 = blockIdx.x * 128;
-  if (p0 >= P) return;                                   // CTA-uniform
+  // a p tile past P still takes part in its cluster's barriers (with no work)
+  const bool p_live = p0 < P;
   const int chunk = blockIdx.y;
-  const int mb = chunk * kColChunk;
-  const int m_end = min(M, mb + kColChunk);
-  const int n_steps = (m_end - mb + 31) / 32;
+  const int mb = chunk * chunk_tokens;
+  const int m_end = min(M, mb + chunk_tokens);
+  const int n_steps = p_live && m_end > mb ? (m_end - mb + 31) / 32 : 0;
   const int mi = lane >> 3, ri = lane & 7;
 
   for (int nb = 0; nb < R; nb += 64) {
@@ -292,53 +325,46 @@ __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem 
     }
     cp_async_wait<0>();
     __syncthreads();
-    // write the partial tile
+    // partial tile [128 p][64 n] (dB) or [64 n][128 p] (dA) in shared memory
     const int g = lane >> 2, q = lane & 3;
-    float* dst = pr.part + static_cast<int64_t>(chunk) * P * R;
+    float* red = reinterpret_cast<float*>(s_col);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      const int pa = p0 + warp * 32 + i * 16 + g;
+      const int pl = warp * 32 + i * 16 + g;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        if (j < nt) {
-          const int n = nb + 8 * j + 2 * q;
+        const int nl = 8 * j + 2 * q;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int pp = pa + 8 * h;
-            if (pp < P) {
-              if (pr.n_major) {
-                dst[static_cast<int64_t>(n) * P + pp] = acc[i][j][2 * h];
-                dst[static_cast<int64_t>(n + 1) * P + pp] = acc[i][j][2 * h + 1];
-              } else {
-                *reinterpret_cast<float2*>(dst + static_cast<int64_t>(pp) * R + n) =
-                    make_float2(acc[i][j][2 * h], acc[i][j][2 * h + 1]);
-              }
-            }
+        for (int h = 0; h < 2; ++h) {
+          if (pr.n_major) {
+            red[nl * 128 + pl + 8 * h] = acc[i][j][2 * h];
+            red[(nl + 1) * 128 + pl + 8 * h] = acc[i][j][2 * h + 1];
+          } else {
+            *reinterpret_cast<float2*>(red + (pl + 8 * h) * 64 + nl) = make_float2(acc[i][j][2 * h], acc[i][j][2 * h + 1]);
           }
         }
       }
     }
-  }
-}
-
-// out_z[e] = sum over chunks c = 0..C-1 of part_z[c][e], in chunk order, for
-// the two problems z = blockIdx.y (float4-vectorised; n_el % 4 == 0).
-__global__ void __launch_bounds__(256) sum_chunks_kernel(
-    const float* __restrict__ part0, float* __restrict__ out0, int64_t n_el0,
-    const float* __restrict__ part1, float* __restrict__ out1, int64_t n_el1, int C) {
-  const float* part = blockIdx.y == 0 ? part0 : part1;
-  float* out = blockIdx.y == 0 ? out0 : out1;
-  const int64_t n4 = (blockIdx.y == 0 ? n_el0 : n_el1) / 4;
-  const int64_t stride = n4;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n4;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int c = 0; c < C; ++c) {
-      const float4 t = __ldg(reinterpret_cast<const float4*>(part) + c * stride + e);
-      v.x += t.x; v.y += t.y; v.z += t.z; v.w += t.w;
+    cluster_sync_all();
+    if (p_live) {
+      // every CTA of the cluster reduces (chunks in rank order) and stores its share of the tile
+      const int ks = static_cast<int>(gridDim.y), rank = static_cast<int>(cluster_ctarank());
+      constexpr int n4 = 128 * 64 / 4;
+      const uint32_t red_addr = smem_u32(red);
+      for (int e = rank * n4 / ks + threadIdx.x; e < (rank + 1) * n4 / ks; e += kColThreads) {
+        const float4 v = cluster_sum_f4(red_addr + e * 16, ks);
+        if (pr.n_major) {                                            // red [n][p]: 4 consecutive p
+          const int nl = e / 32, pl = (e % 32) * 4;
+          if (nl < 8 * nt && p0 + pl < P)
+            *reinterpret_cast<float4*>(pr.out + static_cast<int64_t>(nb + nl) * P + p0 + pl) = v;
+        } else {                                                     // red [p][n]: 4 consecutive n
+          const int pl = e / 16, nl = (e % 16) * 4;
+          if (nl < 8 * nt && p0 + pl < P)
+            *reinterpret_cast<float4*>(pr.out + static_cast<int64_t>(p0 + pl) * R + nb + nl) = v;
+        }
+      }
     }
-    reinterpret_cast<float4*>(out)[e] = v;
+    cluster_sync_all();                                              // partials stay until all are read
   }
 }
 

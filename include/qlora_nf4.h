@@ -237,7 +237,7 @@ int qlora_selftest_wait_timeout(void* stream);
  * the number of launches since the last reset.  Names: "quantize_blocks",
  * "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
  * "gemv", "gemv_finalize", "lora_rowwise" (us), "lora_rowwise_du" (du),
- * "lora_rowwise_finalize", "lora_colwise", "sum_chunks".  Events are created by the library on first use (host-side
+ * "lora_colwise" (dA and dB).  Events are created by the library on first use (host-side
  * CUDA objects, no device memory).  Not for use during stream capture.
  *
  * qlora_timing_enable: on != 0 enables, 0 disables; returns the previous state.
