@@ -440,24 +440,31 @@ def comp_quantize(q, dev, peaks, src, reps=3):
         for _, W, w in weights:
             q.quantize_nf4(W, out=w, workspace=ws)
     torch.cuda.synchronize()
-    q.timing_reset()
-    q.timing_enable(True)
     a, b = ev(), ev()
-    a.record()
-    for _ in range(reps):
-        for _, W, w in weights:
-            q.quantize_nf4(W, out=w, workspace=ws)
-    b.record()
-    torch.cuda.synchronize()
-    q.timing_enable(False)
-    tot = a.elapsed_time(b) / reps
+
+    def region(per_kernel):
+        q.timing_reset()
+        q.timing_enable(per_kernel)
+        a.record()
+        for _ in range(reps):
+            for _, W, w in weights:
+                q.quantize_nf4(W, out=w, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        q.timing_enable(False)
+        return a.elapsed_time(b) / reps
+
+    tot = region(False)                       # clean: no per-kernel events
+    region(True)                              # same work, per-kernel split
     qbytes = sum(workloads.quant_bytes(*W.shape) for _, W, _ in weights)
-    kq, nq = q.timing_collect("quantize_blocks")
+    split = {}
+    for name in ("quantize_blocks", "scale_mean_tree", "dq_scales"):
+        t, n = q.timing_collect(name)
+        split[name + "_ms"] = t / reps if n else None
     out["quantize_65b_layer"] = {
         "weights": sum(W.numel() for _, W, _ in weights), "ms": tot, "GB/s": qbytes / (tot * 1e-3) / 1e9,
         "frac_hbm": qbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "quantize_blocks_ms": kq / reps if nq else None,
-        "peak_source": f"hbm_gbs of {src}"}
+        "kernels_with_events": split, "peak_source": f"hbm_gbs of {src}"}
     deq_out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _, _, w in weights]
     for (_, _, w), o in zip(weights, deq_out):
         q.dequantize_nf4(w, out=o)

@@ -175,7 +175,7 @@ int device_sm_count() {
 
 // ------------------------------------------------------------------ workspace
 struct QuantWs {
-  size_t absmax_off, tree_off, total;
+  size_t absmax_off, tree_off, ticket_off, total;
   int64_t tree_count;  // doubles reserved for all tree passes
 };
 
@@ -184,13 +184,16 @@ QuantWs quant_ws(int64_t rows, int64_t cols) {
   const int64_t n_blocks = rows * cols / 64;
   w.absmax_off = 0;
   w.tree_off = round256(static_cast<size_t>(n_blocks) * 4);
+  // chunk sums of every pass down to the one the last CTA finishes, then two
+  // ticket counters (one per pass parity)
   int64_t count = 0, n = n_blocks;
   do {
     n = cdiv(n, qnf4::kTreeChunk);
     count += n;
-  } while (n > 1);
+  } while (n > qnf4::kTreeTop);
   w.tree_count = count;
-  w.total = w.tree_off + round256(static_cast<size_t>(count) * 8);
+  w.ticket_off = w.tree_off + round256(static_cast<size_t>(count) * 8);
+  w.total = w.ticket_off + 256;
   return w;
 }
 
@@ -276,34 +279,40 @@ int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, 
   float* absmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.absmax_off);
   double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + w.tree_off);
 
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + w.ticket_off);
+
   const int sms = device_sm_count();
   const int64_t want = cdiv(n_blocks, 16 * qnf4::kQRounds);
   const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
   {
     LaunchTimer lt_("quantize_blocks", st);
-    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C);
+    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C, tickets);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
 
-  // fixed summation tree, one pass per 4096x reduction
+  // fixed summation tree: 4096x reductions; the pass that leaves at most
+  // kTreeTop sums is finished (and the mean written) by its last CTA.  Each
+  // pass resets the ticket of the pass after it (they alternate).
   int64_t n = n_blocks;
   int64_t parts = cdiv(n, qnf4::kTreeChunk);
+  int pass = 0;
   {
     LaunchTimer lt_("scale_mean_tree", st);
     qnf4::pairwise_tree_kernel<float><<<static_cast<unsigned>(parts), 256, 0, st>>>(
-      absmax, n, tree, n_blocks, parts == 1 ? mean : nullptr);
+        absmax, n, tree, parts <= qnf4::kTreeTop, tickets, n_blocks, mean, tickets + 1);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   double* prev = tree;
-  while (parts > 1) {
+  while (parts > qnf4::kTreeTop) {
     n = parts;
     parts = cdiv(n, qnf4::kTreeChunk);
     double* next = prev + n;
+    ++pass;
     {
-    LaunchTimer lt_("scale_mean_tree", st);
-    qnf4::pairwise_tree_kernel<double><<<static_cast<unsigned>(parts), 256, 0, st>>>(
-        prev, n, next, n_blocks, parts == 1 ? mean : nullptr);
-  }
+      LaunchTimer lt_("scale_mean_tree", st);
+      qnf4::pairwise_tree_kernel<double><<<static_cast<unsigned>(parts), 256, 0, st>>>(
+          prev, n, next, parts <= qnf4::kTreeTop, tickets + (pass & 1), n_blocks, mean, tickets + ((pass + 1) & 1));
+    }
     QLORA_CUDA_TRY(cudaGetLastError());
     prev = next;
   }
@@ -693,7 +702,7 @@ namespace {
 constexpr int64_t kNoAllocMaxBlocks = QLORA_NOALLOC_MAX_BLOCKS;
 constexpr size_t kNoAllocScratchBytes =
     ((static_cast<size_t>(kNoAllocMaxBlocks) * 4 + 255) & ~static_cast<size_t>(255)) +
-    ((static_cast<size_t>(kNoAllocMaxBlocks / qnf4::kTreeChunk + 1) * 8 + 255) & ~static_cast<size_t>(255));
+    ((static_cast<size_t>(kNoAllocMaxBlocks / qnf4::kTreeChunk + 1) * 8 + 255) & ~static_cast<size_t>(255)) + 256;
 
 // One copy per device that loads the library.  In host code this name is a
 // host-side stand-in, never a device address: the address comes from

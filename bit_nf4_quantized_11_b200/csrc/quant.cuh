@@ -19,6 +19,7 @@ namespace qnf4 {
 constexpr int kBlock = 64;        // weights per first-level block
 constexpr int kGroup = 256;       // blocks per second-level group
 constexpr int kTreeChunk = 4096;  // leaves summed by one CTA of the scale-mean tree
+constexpr int kTreeTop = 1024;    // most partial sums the last CTA of a pass finishes
 
 // ---------------------------------------------------------------------------
 // K1 and its code table
@@ -58,8 +59,9 @@ __device__ __forceinline__ uint32_t nearest_code(float v, uint32_t tab_lane) {
 // lane l at (n*32 + l)*8), so lookups never conflict.
 __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
     const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
-    float* __restrict__ absmax, CodeTable tab) {
+    float* __restrict__ absmax, CodeTable tab, unsigned int* __restrict__ ticket) {
   __shared__ __align__(16) uint2 s_tab[kCodeCells * 32];
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;            // for the tree pass after this kernel
   for (int e = threadIdx.x; e < kCodeCells * 32; e += blockDim.x)
     s_tab[e] = make_uint2(tab.below[e >> 5], __float_as_uint(tab.inside[e >> 5]));
   __syncthreads();
@@ -118,21 +120,20 @@ __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
 // chunk of 4096 leaves: 16 consecutive leaves per thread (in-register tree),
 // then a xor-butterfly across the warp (offset 1, 2, 4, ... adds adjacent
 // pairs), then the 8 warp sums pairwise.  Chunks are aligned subtrees, so
-// repeating the pass over the chunk sums reproduces the full tree exactly;
-// missing leaves are exact zeros.  The pass that leaves one value also writes
-// mean = fp32(T / n_leaves) with the division in fp64.
+// summing the chunk sums the same way reproduces the full tree exactly;
+// missing leaves are exact zeros.  With `finish` (at most kTreeTop chunks),
+// the CTA that completes last (a ticket counter, reset to 0 by the kernel
+// before) sums the chunk sums -- 4 per thread, butterfly, warp sums -- and
+// writes mean = fp32(T / n_leaves) with the division in fp64.  Otherwise the
+// host runs another pass over the chunk sums.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) pairwise_tree_kernel(
-    const T* __restrict__ in, int64_t n, double* __restrict__ out,
-    int64_t n_leaves_total, float* __restrict__ mean_out) {
-  __shared__ double s_warp[8];
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTreeChunk + threadIdx.x * 16;
-  double v[16];
+template <int kPer>
+__device__ __forceinline__ double tree_256(const double (&v0)[kPer], double* s_warp) {
+  double v[kPer];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = (base + i < n) ? static_cast<double>(in[base + i]) : 0.0;
+  for (int i = 0; i < kPer; ++i) v[i] = v0[i];
 #pragma unroll
-  for (int width = 8; width >= 1; width >>= 1) {
+  for (int width = kPer / 2; width >= 1; width >>= 1) {
 #pragma unroll
     for (int i = 0; i < width; ++i) v[i] = __dadd_rn(v[2 * i], v[2 * i + 1]);
   }
@@ -141,14 +142,43 @@ __global__ void __launch_bounds__(256) pairwise_tree_kernel(
   for (int off = 1; off < 32; off <<= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, off));
   if ((threadIdx.x & 31) == 0) s_warp[threadIdx.x >> 5] = s;
   __syncthreads();
+  const double a = __dadd_rn(__dadd_rn(s_warp[0], s_warp[1]), __dadd_rn(s_warp[2], s_warp[3]));
+  const double b = __dadd_rn(__dadd_rn(s_warp[4], s_warp[5]), __dadd_rn(s_warp[6], s_warp[7]));
+  return __dadd_rn(a, b);                                            // same value in every thread
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) pairwise_tree_kernel(
+    const T* __restrict__ in, int64_t n, double* __restrict__ out, int finish,
+    unsigned int* __restrict__ ticket, int64_t n_leaves_total, float* __restrict__ mean_out,
+    unsigned int* __restrict__ next_ticket) {
+  __shared__ double s_warp[8];
+  __shared__ int s_last;
+  if (blockIdx.x == 0 && threadIdx.x == 0 && next_ticket != nullptr) *next_ticket = 0u;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kTreeChunk + threadIdx.x * 16;
+  double v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = (base + i < n) ? static_cast<double>(in[base + i]) : 0.0;
+  const double t = tree_256<16>(v, s_warp);
   if (threadIdx.x == 0) {
-    const double a = __dadd_rn(__dadd_rn(s_warp[0], s_warp[1]), __dadd_rn(s_warp[2], s_warp[3]));
-    const double b = __dadd_rn(__dadd_rn(s_warp[4], s_warp[5]), __dadd_rn(s_warp[6], s_warp[7]));
-    const double t = __dadd_rn(a, b);
     out[blockIdx.x] = t;
-    if (mean_out != nullptr)   // single-chunk pass: t is the whole tree
-      *mean_out = __double2float_rn(__ddiv_rn(t, static_cast<double>(n_leaves_total)));
+    if (finish) {
+      __threadfence();
+      s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    }
   }
+  __syncthreads();
+  if (!finish || !s_last) return;                                    // CTA-uniform
+  __threadfence();
+  double w[kTreeTop / 256];
+#pragma unroll
+  for (int i = 0; i < kTreeTop / 256; ++i) {
+    const int idx = threadIdx.x * (kTreeTop / 256) + i;
+    w[i] = idx < static_cast<int>(gridDim.x) ? __ldcg(out + idx) : 0.0;
+  }
+  __syncthreads();                                                   // s_warp is reused
+  const double total = tree_256<kTreeTop / 256>(w, s_warp);
+  if (threadIdx.x == 0) *mean_out = __double2float_rn(__ddiv_rn(total, static_cast<double>(n_leaves_total)));
 }
 
 // ---------------------------------------------------------------------------
@@ -168,27 +198,38 @@ __global__ void __launch_bounds__(256) dq_scales_kernel(
   float d[8];
   float S = 0.f;
   const int64_t base = g * kGroup + lane * 8;
+  if (base + 8 <= n_blocks) {                                        // two 16-byte loads
+    const float4 a = __ldg(reinterpret_cast<const float4*>(absmax + base));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(absmax + base + 4));
+    const float c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t idx = base + i;
-    d[i] = (idx < n_blocks) ? __fsub_rn(absmax[idx], mu) : 0.f;
-    S = fmaxf(S, fabsf(d[i]));
+    for (int i = 0; i < 8; ++i) d[i] = __fsub_rn(c[i], mu);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = (base + i < n_blocks) ? __fsub_rn(absmax[base + i], mu) : 0.f;
   }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) S = fmaxf(S, fabsf(d[i]));
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) S = fmaxf(S, __shfl_xor_sync(0xffffffffu, S, off));
   const float st = __fdiv_rn(S, 127.0f);
   if (lane == 0) step2[g] = st;
   const float inv = (st != 0.f) ? __frcp_rn(st) : 0.f;
+  uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int64_t idx = base + i;
-    if (idx >= n_blocks) break;
     int q = 0;
     if (st != 0.f) {
       const float p = __fmul_rn(d[i], inv);
       if (p == p) q = min(127, max(-127, __float2int_rn(p)));
     }
-    q8[idx] = static_cast<int8_t>(q);
+    packed[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
+  }
+  if (base + 8 <= n_blocks) {
+    *reinterpret_cast<uint2*>(q8 + base) = make_uint2(packed[0], packed[1]);   // one 8-byte store
+  } else {
+    for (int i = 0; i < 8 && base + i < n_blocks; ++i)
+      q8[base + i] = static_cast<int8_t>((packed[i >> 2] >> (8 * (i & 3))) & 0xFFu);
   }
 }
 

@@ -262,7 +262,7 @@ int qlora_timing_collect(const char* kernel, double* total_ms, int64_t* launches
  * qlora_quantize_nf4 computes (same kernels, bit-identical outputs); its
  * scratch (block absmaxes and the partial sums of the scale-mean tree) lives
  * in a fixed device array inside the library, QLORA_NOALLOC_MAX_BLOCKS blocks
- * of 64 weights large (16 MiB + 8 KiB), which every GPU that loads the
+ * of 64 weights large (16 MiB + 8.5 KiB), which every GPU that loads the
  * library holds until the process exits.  The call itself allocates nothing.
  *
  * The first call on a device looks up that array's device address (once per

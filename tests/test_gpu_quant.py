@@ -43,7 +43,7 @@ def _check_quant(q, W_cpu, sample_rows=None):
     (300, 640, "normal", 0.02, 2),       # 3000 blocks: partial last group (3000 % 256 = 184)
     (512, 512, "normal", 0.02, 0),       # the small parity layer
     (257, 1088, "student_t5", 0.02, 3),  # heavy tails, odd row count
-    (1024, 1024, "normal", 0.015, 4),    # 16384 blocks: two-pass summation tree
+    (1024, 1024, "normal", 0.015, 4),    # 16384 blocks: 4 tree chunks finished by the last CTA
 ])
 def test_quantize_bit_exact(cuda_lib, rows, cols, dist, std, seed):
     _check_quant(cuda_lib, synth.weight(rows, cols, std, dist, seed))
@@ -87,6 +87,16 @@ def test_quantize_70b_65b_shapes_sampled_rows(cuda_lib, shape, std):
     rows = np.sort(rng.choice(shape[0], 48, replace=False))
     rows[0], rows[-1] = 0, shape[0] - 1
     _check_quant(cuda_lib, synth.weight(shape[0], shape[1], std, "normal", 0), sample_rows=rows)
+
+
+def test_quantize_extra_tree_pass_sampled_rows(cuda_lib):
+    """8200 x 32768: 4 198 400 blocks leave 1025 sums of 4096-leaf subtrees,
+    more than the 1024 that the last CTA of a tree pass finishes, so a second
+    pass over them runs (and its last CTA writes the mean)."""
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(8200, 16, replace=False))
+    rows[0], rows[-1] = 0, 8199
+    _check_quant(cuda_lib, synth.weight(8200, 32768, 0.02, "normal", 5), sample_rows=rows)
 
 
 def test_dequantize_matches_codebook_levels_exactly(cuda_lib):
