@@ -35,6 +35,7 @@ Modules:
             dequantize, nibble packing
   linear    QLoRA linear forward / backward in fp64
   overhead  storage arithmetic of the quantization constants
+  merge     adapter merge into a bf16 copy of the dequantized base
 """
 
-from . import nf4, linear, overhead  # noqa: F401
+from . import nf4, linear, overhead, merge  # noqa: F401

@@ -43,6 +43,12 @@ R5 Double quantization: one fp32 mean per tensor (pairwise fp64 sum of all
    first-level codes always use the exact block absmax.
 R6 Dequantization: ``c_hat = fl32(fl32(q8 * step2) + mean)`` and
    ``w_hat = bf16_rne(fl32(level[code] * c_hat))``.
+R7 16-bit input: weights loaded in bf16 (as a 16-bit checkpoint is loaded
+   before quantization; "QLoRA: Fine-Tuning on One Consumer GPU", skillbyai,
+   section "Merging the adapter for serving", which loads the base in
+   bfloat16) are quantized by the same steps applied to the exact fp32 value
+   of each bf16 number; bf16 -> fp32 widening is exact, so nothing else
+   changes.
 """
 
 from __future__ import annotations
@@ -258,6 +264,12 @@ def quantize(W: np.ndarray) -> dict:
     q8, step2, mean = double_quantize(c)
     return dict(codes=codes, packed=pack(codes), absmax=c, q8=q8,
                 step2=step2, mean=mean)
+
+
+def quantize_bf16(bits: np.ndarray) -> dict:
+    """Quantize a weight given as bf16 bit patterns [rows, cols] (reading R7):
+    :func:`quantize` of the exact values of the bf16 numbers."""
+    return quantize(bf16_to_f64(bits))
 
 
 def dequant_scales(q8: np.ndarray, step2: np.ndarray, mean: float) -> np.ndarray:
