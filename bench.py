@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["quantize", "gemv", "workloads"], default=None,
+    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge"], default=None,
                     help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -465,6 +465,24 @@ def comp_quantize(q, dev, peaks, src, reps=3):
         "weights": sum(W.numel() for _, W, _ in weights), "ms": tot, "GB/s": qbytes / (tot * 1e-3) / 1e9,
         "frac_hbm": qbytes / (tot * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "kernels_with_events": split, "peak_source": f"hbm_gbs of {src}"}
+    # the same seven weights loaded in bf16 (2 B read per weight)
+    wb = [(label, W.to(torch.bfloat16), w) for label, W, w in weights]
+    for _ in range(2):
+        for _, Wb, w in wb:
+            q.quantize_nf4(Wb, out=w, workspace=ws)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        for _, Wb, w in wb:
+            q.quantize_nf4(Wb, out=w, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    tb = a.elapsed_time(b) / reps
+    qbytes_b = sum(workloads.quant_bytes(*Wb.shape) - 2 * Wb.numel() for _, Wb, _ in wb)
+    out["quantize_bf16_65b_layer"] = {"ms": tb, "GB/s": qbytes_b / (tb * 1e-3) / 1e9,
+                                      "frac_hbm": qbytes_b / (tb * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                      "bytes_per_weight": 2.516}
+    del wb
     deq_out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _, _, w in weights]
     for (_, _, w), o in zip(weights, deq_out):
         q.dequantize_nf4(w, out=o)
@@ -482,6 +500,57 @@ def comp_quantize(q, dev, peaks, src, reps=3):
     del deq_out, weights, ws
     torch.cuda.empty_cache()
     return out
+
+
+def comp_merge(q, dev, peaks, src, reps=5):
+    """Adapter merge into a bf16 base and its lossy re-quantization to NF4, on
+    the 7B attention projection (r=16) and the 65B down projection (r=64).
+    Merge bytes: packed weight read + bf16 written (2.516 B/weight); the loss
+    is the relative Frobenius error of the re-quantized merged weight."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    a, b = ev(), ev()
+    res = {}
+    for label, n_out, n_in, r, alpha, std in (("llama7b-attn-4096x4096-r16", 4096, 4096, 16, 32.0, 0.02),
+                                              ("llama65b-down-22016x8192-r64", 8192, 22016, 64, 16.0, 0.01)):
+        W = synth.weight(n_out, n_in, std, seed=3).to(dev)
+        A = synth.lora_A(r, n_in).to(dev)
+        B = (synth.lora_B(n_out, r).float() * 10).to(torch.bfloat16).to(dev)   # a trained-size adapter
+        w = q.quantize_nf4(W)
+        merged = torch.empty(n_out, n_in, dtype=torch.bfloat16, device=dev)
+        w2 = q.alloc_nf4(n_out, n_in, dev)
+        for _ in range(2):
+            q.merge_adapter(w, A, B, alpha, out=merged)
+            q.quantize_nf4(merged, out=w2)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(reps):
+            q.merge_adapter(w, A, B, alpha, out=merged)
+        b.record()
+        torch.cuda.synchronize()
+        t_merge = a.elapsed_time(b) / reps
+        a.record()
+        for _ in range(reps):
+            q.quantize_nf4(merged, out=w2)
+        b.record()
+        torch.cuda.synchronize()
+        t_req = a.elapsed_time(b) / reps
+        mbytes = workloads.gemv_weight_bytes(n_out, n_in) + 2 * n_out * n_in
+        qbytes = n_out * n_in * (2 + 0.5 + 1 / 64) + 4 * (n_out * n_in // 64 // 256)
+        base_f = q.dequantize_nf4(w).float()
+        req_f = q.dequantize_nf4(w2).float()
+        mf = merged.float()
+        res[f"merge_{label}"] = {
+            "merge_ms": t_merge, "merge_GB/s": mbytes / (t_merge * 1e-3) / 1e9,
+            "merge_frac_hbm": mbytes / (t_merge * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "requantize_bf16_ms": t_req, "requantize_GB/s": qbytes / (t_req * 1e-3) / 1e9,
+            "requantize_frac_hbm": qbytes / (t_req * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "merge_into_4bit_rel_error": float((req_f - mf).norm() / mf.norm()),
+            "base_quantization_rel_error": float((base_f - W).norm() / W.norm()),
+            "adapter_update_rel_size": float((mf - base_f).norm() / base_f.norm()),
+            "peak_source": f"hbm_gbs of {src}"}
+        del W, w, w2, merged, base_f, req_f, mf
+        torch.cuda.empty_cache()
+    return res
 
 
 def comp_gemv(q, dev, peaks, n=60):
@@ -568,6 +637,8 @@ def components(q, dev, only=None):
         out.update(comp_gemv(q, dev, peaks))
     if only in (None, "workloads"):
         out.update(comp_workloads(q, dev, peaks))
+    if only in (None, "merge"):
+        out.update(comp_merge(q, dev, peaks, src))
     return out
 
 

@@ -30,7 +30,7 @@ __all__ = [
     "dequantize_nf4", "alloc_nf4",
     "linear_fwd", "linear_bwd", "workspace_size", "last_device_status",
     "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
-    "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES",
+    "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES", "merge_adapter",
     "OP_QUANTIZE", "OP_DEQUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD",
 ]
 
@@ -83,6 +83,8 @@ def load():
         "qlora_selftest_wait_timeout": (I, [P]),
         "qlora_status_string": (ctypes.c_char_p, [I]),
         "qlora_quantize_nf4_noalloc": (I, [P, I64, I64, P, P, P, P, P]),
+        "qlora_quantize_nf4_bf16": (I, [P, I64, I64, P, P, P, P, P, SZ, P]),
+        "qlora_merge_adapter": (I, [W, P, P, I, F, P, P]),
         "qlora_timing_enable": (I, [I]),
         "qlora_timing_reset": (None, []),
         "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -177,15 +179,35 @@ def alloc_nf4(rows: int, cols: int, device) -> NF4Weight:
 
 
 def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, workspace=None) -> NF4Weight:
-    """NF4 + double quantization of an fp32 weight [rows, cols] (cols % 64 == 0)."""
-    _need(W, torch.float32, "W")
+    """NF4 + double quantization of an fp32 or bf16 weight [rows, cols]
+    (cols % 64 == 0); a bf16 weight is quantized as its exact fp32 values."""
+    if not (isinstance(W, torch.Tensor) and W.dtype == torch.bfloat16):
+        _need(W, torch.float32, "W")
+    else:
+        _need(W, torch.bfloat16, "W")
     rows, cols = W.shape
     w = out if out is not None else alloc_nf4(rows, cols, W.device)
     ws = _workspace(workspace_size(OP_QUANTIZE, 0, cols, rows, 0), W.device, workspace)
-    _check(load().qlora_quantize_nf4(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2),
-                                     _ptr(w.mean), _ptr(ws), ws.numel() if ws is not None else 0,
-                                     _stream()), "qlora_quantize_nf4")
+    fn, name = ((load().qlora_quantize_nf4_bf16, "qlora_quantize_nf4_bf16") if W.dtype == torch.bfloat16
+                else (load().qlora_quantize_nf4, "qlora_quantize_nf4"))
+    _check(fn(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2), _ptr(w.mean), _ptr(ws),
+              ws.numel() if ws is not None else 0, _stream()), name)
     return w
+
+
+def merge_adapter(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                  out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [out, in] = dequant(W0) + (alpha/r) B A, the adapter merged into a
+    bf16 copy of the base (A bf16 [r, in], B bf16 [out, r])."""
+    r = A.shape[0]
+    _need(A, torch.bfloat16, "A", (r, w.cols))
+    _need(B, torch.bfloat16, "B", (w.rows, r))
+    o = out if out is not None else torch.empty((w.rows, w.cols), dtype=torch.bfloat16, device=A.device)
+    _need(o, torch.bfloat16, "out", (w.rows, w.cols))
+    cw = w._c()
+    _check(load().qlora_merge_adapter(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(o), _stream()),
+           "qlora_merge_adapter")
+    return o
 
 
 def quantize_nf4_noalloc(W: torch.Tensor, out: NF4Weight | None = None) -> NF4Weight:
@@ -263,7 +285,8 @@ def selftest_wait_timeout() -> int:
 
 
 KERNEL_NAMES = ("quantize_blocks", "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
-                "gemv", "gemv_finalize", "lora_rowwise", "lora_rowwise_du", "lora_colwise")
+                "gemv", "gemv_finalize", "lora_rowwise", "lora_rowwise_du", "lora_colwise",
+                "merge_adapter")
 
 
 def timing_enable(on: bool = True) -> bool:

@@ -19,6 +19,7 @@
 #include "gemm_sm100.cuh"
 #include "gemm_pair_sm100.cuh"
 #include "gemv.cuh"
+#include "merge.cuh"
 #include "quant.cuh"
 #include "skinny.cuh"
 
@@ -271,7 +272,8 @@ BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
 }
 
 // ------------------------------------------------------------------ launches
-int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
+template <typename Tin>
+int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
                     float* mean, void* ws, cudaStream_t st) {
   const Tables& tb = tables();
   const int64_t n_blocks = rows * cols / 64;
@@ -282,11 +284,12 @@ int launch_quantize(const float* W, int64_t rows, int64_t cols, uint8_t* codes, 
   unsigned int* tickets = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + w.ticket_off);
 
   const int sms = device_sm_count();
-  const int64_t want = cdiv(n_blocks, 16 * qnf4::kQRounds);
-  const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 8)));
+  const int64_t want = cdiv(n_blocks, 64 * qnf4::kQRounds);       // 8 warps x 8 blocks x rounds per CTA
+  // one wave: 4 CTAs of 256 threads fit an SM at the kernel's register count
+  const int grid1 = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * 4)));
   {
     LaunchTimer lt_("quantize_blocks", st);
-    qnf4::nf4_quantize_blocks_kernel<<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C, tickets);
+    qnf4::nf4_quantize_blocks_kernel<Tin><<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C, tickets);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
 
@@ -525,6 +528,37 @@ int qlora_quantize_nf4(const float* W, int64_t rows, int64_t cols, uint8_t* code
   const QuantWs w = quant_ws(rows, cols);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
   return launch_quantize(W, rows, cols, codes, q8, step2, mean, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int qlora_quantize_nf4_bf16(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
+                            float* mean, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!W || !codes || !q8 || !step2 || !mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(q8, 16) || !aligned(step2, 16) || !aligned(mean, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 64 || cols % 64 != 0 || rows * cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const QuantWs w = quant_ws(rows, cols);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
+  return launch_quantize(W, rows, cols, codes, q8, step2, mean, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                        uint16_t* W_out, void* stream) {
+  if (!weight_ok(w) || !A || !B || !W_out || !aligned(A, 16) || !aligned(B, 16) || !aligned(W_out, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || r > 256 || w->rows < 64 || w->cols < 64 || w->rows % 64 != 0 || w->cols % 64 != 0 ||
+      w->rows * w->cols > (1ll << 40))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const float s = alpha / static_cast<float>(r);
+  const int64_t units = (w->rows / qnf4::kMergeRows) * (w->cols / 8);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+  {
+    LaunchTimer lt_("merge_adapter", static_cast<cudaStream_t>(stream));
+    qnf4::merge_adapter_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        w->codes, w->q8, w->step2, w->mean, A, B, r, s, w->rows, w->cols, W_out, tables().L);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
 }
 
 int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {

@@ -24,7 +24,7 @@ constexpr int kTreeTop = 1024;    // most partial sums the last CTA of a pass fi
 // ---------------------------------------------------------------------------
 // K1 and its code table
 // ---------------------------------------------------------------------------
-constexpr int kQRounds = 4;
+constexpr int kQRounds = 2;
 
 // Exact nearest level without a search.  [-1, 1] (slightly widened: a block's
 // normalised values can exceed 1 by an ulp) is cut into 33 cells by
@@ -45,20 +45,38 @@ __device__ __forceinline__ uint32_t nearest_code(float v, uint32_t tab_lane) {
   const uint32_t n = min(static_cast<uint32_t>(__float_as_int(y) - __float_as_int(kCellMagic) + 16),
                          static_cast<uint32_t>(kCodeCells - 1));
   uint32_t below, inside_bits;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(inside_bits) : "r"(tab_lane + n * 256));
+  // not volatile: the table is written before the barrier that precedes every
+  // weight load, and each lookup depends on a loaded weight
+  asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(below), "=r"(inside_bits) : "r"(tab_lane + n * 256));
   return below + (v > __uint_as_float(inside_bits) ? 1u : 0u);
 }
 
-// K1: per-block absmax, nearest-level code, nibble packing.
-// One half-warp per 64-weight block: each lane loads 4 fp32 (16 B), the
-// absmax is reduced over the 16 lanes, and each lane packs its 4 codes into
-// 2 bytes, so a block's 32 code bytes are written by one coalesced store.
-// A warp takes 2*kQRounds consecutive blocks per iteration and issues all
-// their loads before any arithmetic, keeping 64 B per lane in flight.
+// K1: per-block absmax, nearest-level code, nibble packing (fp32 or bf16
+// weights; a bf16 weight is quantized as its exact fp32 value).
+// Four lanes per 64-weight block: lane q takes the 4-weight chunks q, q+4,
+// q+8, q+12, so each load instruction reads every block's 64 consecutive
+// bytes (fp32) in one piece; the absmax is reduced over the 4 lanes with two
+// shuffles, and lane q writes the 2 code bytes of each of its chunks.  A warp
+// takes 8 * kQRounds consecutive blocks per iteration and issues all their
+// loads before any arithmetic (64 B per lane per round in flight).
 // The cell table sits in shared memory with one copy per lane (entry n of
 // lane l at (n*32 + l)*8), so lookups never conflict.
-__global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
-    const float* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
+// Four consecutive weights as fp32: 16 bytes of fp32, or 8 bytes of bf16
+// widened exactly (a bf16 number is the top half of its fp32 pattern).
+__device__ __forceinline__ float4 load_w4(const float* W, int64_t i) {
+  const uint4 u = ld_stream_v4(W + i);
+  return make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+}
+__device__ __forceinline__ float4 load_w4(const uint16_t* W, int64_t i) {
+  uint32_t a, b;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "l"(W + i));
+  return make_float4(__uint_as_float(a << 16), __uint_as_float(a & 0xFFFF0000u), __uint_as_float(b << 16),
+                     __uint_as_float(b & 0xFFFF0000u));
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(256, 4) nf4_quantize_blocks_kernel(
+    const Tin* __restrict__ W, int64_t n_blocks, uint8_t* __restrict__ codes,
     float* __restrict__ absmax, CodeTable tab, unsigned int* __restrict__ ticket) {
   __shared__ __align__(16) uint2 s_tab[kCodeCells * 32];
   if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;            // for the tree pass after this kernel
@@ -67,47 +85,60 @@ __global__ void __launch_bounds__(256) nf4_quantize_blocks_kernel(
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;          // which block of a pair
-  const int l16 = lane & 15;
+  const int bl = lane >> 2;            // block of this lane among the warp's 8
+  const int q = lane & 3;              // chunks q + 4k, k = 0..3
   const uint32_t tab_lane = smem_u32(s_tab) + lane * 8;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
 
-  for (int64_t base = warp * 2 * kQRounds; base < n_blocks; base += n_warps * 2 * kQRounds) {
-    float4 w[kQRounds];
+  for (int64_t base = warp * 8 * kQRounds; base < n_blocks; base += n_warps * 8 * kQRounds) {
+    float4 w[kQRounds][4];
 #pragma unroll
     for (int rd = 0; rd < kQRounds; ++rd) {
-      const int64_t b = base + 2 * rd + half;
-      w[rd] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (b < n_blocks) {
-        const uint4 u = ld_stream_v4(W + b * kBlock + l16 * 4);
-        w[rd] = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+      const int64_t b = base + 8 * rd + bl;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        w[rd][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (b < n_blocks) w[rd][k] = load_w4(W, b * kBlock + (q + 4 * k) * 4);
       }
     }
 #pragma unroll
     for (int rd = 0; rd < kQRounds; ++rd) {
-      const int64_t b = base + 2 * rd + half;
-      float m = fmaxf(fmaxf(fabsf(w[rd].x), fabsf(w[rd].y)), fmaxf(fabsf(w[rd].z), fabsf(w[rd].w)));
+      const int64_t b = base + 8 * rd + bl;
+      float m = 0.f;
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      // m is now the exact absmax of this half-warp's block
-      uint32_t packed = 0x7777u;
+      for (int k = 0; k < 4; ++k)
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(w[rd][k].x), fabsf(w[rd][k].y)), fmaxf(fabsf(w[rd][k].z), fabsf(w[rd][k].w))));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      // m is now the exact absmax of this lane's block
       const float r = __frcp_rn(m);
+      uint32_t packed[4];
       if (m > 0.f && isinf(r)) {
         // absmax so small that 1/absmax overflows: v = w * inf is +inf (code
         // 15), -inf (code 0), or NaN for a zero weight (the zero level, 7)
         auto sat = [](float x) -> uint32_t { return x > 0.f ? 15u : (x < 0.f ? 0u : 7u); };
-        packed = sat(w[rd].x) | (sat(w[rd].y) << 4) | (sat(w[rd].z) << 8) | (sat(w[rd].w) << 12);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          packed[k] = sat(w[rd][k].x) | (sat(w[rd][k].y) << 4) | (sat(w[rd][k].z) << 8) | (sat(w[rd][k].w) << 12);
       } else if (m > 0.f) {
-        const uint32_t c0 = nearest_code(__fmul_rn(w[rd].x, r), tab_lane);
-        const uint32_t c1 = nearest_code(__fmul_rn(w[rd].y, r), tab_lane);
-        const uint32_t c2 = nearest_code(__fmul_rn(w[rd].z, r), tab_lane);
-        const uint32_t c3 = nearest_code(__fmul_rn(w[rd].w, r), tab_lane);
-        packed = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t c0 = nearest_code(__fmul_rn(w[rd][k].x, r), tab_lane);
+          const uint32_t c1 = nearest_code(__fmul_rn(w[rd][k].y, r), tab_lane);
+          const uint32_t c2 = nearest_code(__fmul_rn(w[rd][k].z, r), tab_lane);
+          const uint32_t c3 = nearest_code(__fmul_rn(w[rd][k].w, r), tab_lane);
+          packed[k] = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) packed[k] = 0x7777u;
       }
       if (b < n_blocks) {
-        reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2))[l16] = static_cast<uint16_t>(packed);
-        if (l16 == 0) absmax[b] = m;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(codes + b * (kBlock / 2));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst[q + 4 * k] = static_cast<uint16_t>(packed[k]);
+        if (q == 0) absmax[b] = m;
       }
     }
   }

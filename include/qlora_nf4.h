@@ -148,6 +148,46 @@ int qlora_quantize_nf4(const float* W, int64_t rows, int64_t cols,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qlora_quantize_nf4_bf16 -- qlora_quantize_nf4 for a weight loaded in bf16
+ * (the 16-bit checkpoint form; "QLoRA: Fine-Tuning on One Consumer GPU",
+ * skillbyai, Merging the adapter for serving, loads the base in bfloat16).
+ * Every step is that of qlora_quantize_nf4 applied to the exact fp32 value of
+ * each bf16 weight (bf16 -> fp32 widening is exact), so the outputs equal
+ * those of qlora_quantize_nf4 on the widened tensor, bit for bit.
+ *
+ * W       device bf16 (uint16 bit patterns) [rows, cols], 16-byte aligned,
+ *         finite values.  Other arguments, workspace, size rules and return
+ *         values as qlora_quantize_nf4 (same workspace size).
+ */
+int qlora_quantize_nf4_bf16(const uint16_t* W, int64_t rows, int64_t cols,
+                            uint8_t* codes, int8_t* q8, float* step2, float* mean,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * qlora_merge_adapter -- the adapter merged into a bf16 copy of the
+ * dequantized base for serving: W_out = dequant(W0) + (alpha/r) B A.
+ * Merging needs the base dequantized first and goes into a higher-precision
+ * copy, since merging straight back into 4 bit is lossy ("QLoRA",
+ * llm-compass, 调参与实践经验; skillbyai, Merging the adapter for serving).
+ * Per element: acc = fp32 sum over j = 0..r-1, in that order, of
+ * B[o][j] * A[j][i] (each product exact in fp32);
+ * W_out[o][i] = bf16_rne(fp32(w_hat[o][i] + fp32(s * acc))) with
+ * s = fp32(alpha / r) and w_hat the bf16 weight of qlora_dequantize_nf4.
+ * Re-quantizing W_out with qlora_quantize_nf4_bf16 is the lossy "merge back
+ * into 4 bit".
+ *
+ * w       quantized base [out, in]
+ * A       device bf16 [r, in], 16-byte aligned
+ * B       device bf16 [out, r], 16-byte aligned
+ * W_out   device bf16 [out, in], 16-byte aligned (written)
+ * Size rules: in % 64 == 0, out % 64 == 0, 1 <= r <= 256; alpha finite.
+ * Returns QLORA_OK, QLORA_ERR_INVALID_ARG, QLORA_ERR_UNSUPPORTED_SHAPE or
+ * QLORA_ERR_CUDA; nothing is launched on an error.
+ */
+int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                        uint16_t* W_out, void* stream);
+
+/*
  * qlora_dequantize_nf4 -- NF4 weight to bf16, bit-exact with the formula in
  * the format description above ("QLoRA", auryth glossary, "Hoe het werkt":
  * dequantize NF4 on the fly per layer).
@@ -237,7 +277,7 @@ int qlora_selftest_wait_timeout(void* stream);
  * the number of launches since the last reset.  Names: "quantize_blocks",
  * "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
  * "gemv", "gemv_finalize", "lora_rowwise" (us), "lora_rowwise_du" (du),
- * "lora_colwise" (dA and dB).  Events are created by the library on first use (host-side
+ * "lora_colwise" (dA and dB), "merge_adapter".  Events are created by the library on first use (host-side
  * CUDA objects, no device memory).  Not for use during stream capture.
  *
  * qlora_timing_enable: on != 0 enables, 0 disables; returns the previous state.
