@@ -36,6 +36,7 @@ Modules:
   linear    QLoRA linear forward / backward in fp64
   overhead  storage arithmetic of the quantization constants
   merge     adapter merge into a bf16 copy of the dequantized base
+  int4      the uniform INT4 absmax code the pages compare NF4 with
 """
 
-from . import nf4, linear, overhead, merge  # noqa: F401
+from . import nf4, linear, overhead, merge, int4  # noqa: F401
