@@ -483,6 +483,25 @@ def comp_quantize(q, dev, peaks, src, reps=3):
                                       "frac_hbm": qbytes_b / (tb * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                       "bytes_per_weight": 2.516}
     del wb
+    # NF4 vs the uniform INT4 code: round-trip error on normal and Student-t weights (same kernels)
+    cmp = {}
+    for dist in ("normal", "student_t5"):
+        W = synth.weight(4096, 4096, 0.02, dist, seed=21).to(dev)
+        wn = q.quantize_nf4(W)
+        w4 = q.quantize_codebook(W, q.CODEBOOK_INT4)
+        en = float((q.dequantize_nf4(wn).float() - W).norm() / W.norm())
+        e4 = float((q.dequantize_codebook(w4, q.CODEBOOK_INT4).float() - W).norm() / W.norm())
+        cmp[dist] = {"nf4_rel_error": en, "int4_rel_error": e4, "int4_over_nf4": e4 / en}
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(reps):
+        for _, W, w in weights:
+            q.quantize_codebook(W, q.CODEBOOK_INT4, out=w, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    t4 = a.elapsed_time(b) / reps
+    cmp["int4_quantize_65b_layer"] = {"ms": t4, "frac_hbm": qbytes / (t4 * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    out["nf4_vs_int4_7b_attn"] = cmp
     deq_out = [torch.empty(w.rows, w.cols, dtype=torch.bfloat16, device=dev) for _, _, w in weights]
     for (_, _, w), o in zip(weights, deq_out):
         q.dequantize_nf4(w, out=o)

@@ -31,6 +31,7 @@ __all__ = [
     "linear_fwd", "linear_bwd", "workspace_size", "last_device_status",
     "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
     "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES", "merge_adapter",
+    "quantize_codebook", "dequantize_codebook", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "OP_QUANTIZE", "OP_DEQUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD",
 ]
 
@@ -85,6 +86,9 @@ def load():
         "qlora_quantize_nf4_noalloc": (I, [P, I64, I64, P, P, P, P, P]),
         "qlora_quantize_nf4_bf16": (I, [P, I64, I64, P, P, P, P, P, SZ, P]),
         "qlora_merge_adapter": (I, [W, P, P, I, F, P, P]),
+        "qlora_codebook": (I, [I, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
+        "qlora_quantize_codebook": (I, [I, P, I64, I64, P, P, P, P, P, SZ, P]),
+        "qlora_dequantize_codebook": (I, [I, W, P, P]),
         "qlora_timing_enable": (I, [I]),
         "qlora_timing_reset": (None, []),
         "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -143,13 +147,43 @@ class NF4Weight:
         return sum(t.numel() * t.element_size() for t in (self.codes, self.q8, self.step2, self.mean))
 
 
-def codebook():
-    """The 16 NF4 levels and 15 thresholds computed by the library (host)."""
+CODEBOOK_NF4, CODEBOOK_INT4 = 0, 1
+
+
+def codebook(kind: int = CODEBOOK_NF4):
+    """The 16 levels and 15 thresholds of a codebook computed by the library
+    (host): NF4 (default) or the uniform INT4 comparison code."""
     lib = load()
     lv = (ctypes.c_float * 16)()
     th = (ctypes.c_float * 15)()
-    _check(lib.qlora_nf4_codebook(lv, th), "qlora_nf4_codebook")
+    if kind == CODEBOOK_NF4:
+        _check(lib.qlora_nf4_codebook(lv, th), "qlora_nf4_codebook")
+    else:
+        _check(lib.qlora_codebook(int(kind), lv, th), "qlora_codebook")
     return list(lv), list(th)
+
+
+def quantize_codebook(W: torch.Tensor, kind: int, out: NF4Weight | None = None, workspace=None) -> NF4Weight:
+    """Blockwise 4-bit quantization of an fp32 weight with the levels of
+    codebook `kind` (CODEBOOK_NF4 or CODEBOOK_INT4), double-quantized scales."""
+    _need(W, torch.float32, "W")
+    rows, cols = W.shape
+    w = out if out is not None else alloc_nf4(rows, cols, W.device)
+    ws = _workspace(workspace_size(OP_QUANTIZE, 0, cols, rows, 0), W.device, workspace)
+    _check(load().qlora_quantize_codebook(int(kind), _ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2),
+                                          _ptr(w.mean), _ptr(ws), ws.numel() if ws is not None else 0, _stream()),
+           "qlora_quantize_codebook")
+    return w
+
+
+def dequantize_codebook(w: NF4Weight, kind: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 [rows, cols] of a weight quantized with codebook `kind`."""
+    o = out if out is not None else torch.empty((w.rows, w.cols), dtype=torch.bfloat16, device=w.codes.device)
+    _need(o, torch.bfloat16, "out", (w.rows, w.cols))
+    cw = w._c()
+    _check(load().qlora_dequantize_codebook(int(kind), ctypes.byref(cw), _ptr(o), _stream()),
+           "qlora_dequantize_codebook")
+    return o
 
 
 def workspace_size(op: int, M: int, in_features: int, out_features: int, r: int) -> int:

@@ -25,6 +25,7 @@
 
 namespace qnf4_host {
 void build_codebook(float levels[16], float thresholds[15]);
+void build_int4_codebook(float levels[16], float thresholds[15]);
 }
 
 namespace {
@@ -38,35 +39,52 @@ struct Tables {
   Levels L;
   Thresholds T;
   qnf4::CodeTable C;
+  bool ok;      // the cell table is valid for these thresholds
 };
 
 // Cell table of nearest_code: cell n covers 16 v in [n - 16.5, n - 15.5);
 // below[n] = thresholds under the cell, inside[n] = the (at most one)
-// threshold in it or +inf.
-void build_code_table(const Thresholds& T, qnf4::CodeTable* c) {
+// threshold in it or +inf.  Returns false when a cell would hold two
+// thresholds or a threshold sits on a cell edge (where the rounding of 16 v
+// to the cell index could go either way).
+bool build_code_table(const Thresholds& T, qnf4::CodeTable* c) {
+  bool ok = true;
   for (int n = 0; n < qnf4::kCodeCells; ++n) {
     const double lo = (n - 16.5) / 16.0, hi = (n - 15.5) / 16.0;
     uint32_t below = 0;
+    int n_inside = 0;
     float inside = INFINITY;
     for (int j = 0; j < 15; ++j) {
       const double t = T.v[j];
+      if (t == lo) ok = false;
       if (t < lo) ++below;
-      else if (t < hi) inside = T.v[j];
+      else if (t < hi) {
+        inside = T.v[j];
+        ++n_inside;
+      }
     }
+    if (n_inside > 1) ok = false;
     c->below[n] = below;
     c->inside[n] = inside;
   }
+  return ok;
 }
 
-const Tables& tables() {
-  static Tables t;
+// Levels, thresholds and cell table of a codebook kind (QLORA_CODEBOOK_*).
+const Tables* tables_for(int kind) {
+  static Tables t[2];
   static std::once_flag once;
   std::call_once(once, [] {
-    qnf4_host::build_codebook(t.L.v, t.T.v);
-    build_code_table(t.T, &t.C);
+    qnf4_host::build_codebook(t[0].L.v, t[0].T.v);
+    t[0].ok = build_code_table(t[0].T, &t[0].C);
+    qnf4_host::build_int4_codebook(t[1].L.v, t[1].T.v);
+    t[1].ok = build_code_table(t[1].T, &t[1].C);
   });
-  return t;
+  if (kind < 0 || kind > 1 || !t[kind].ok) return nullptr;
+  return &t[kind];
 }
+
+const Tables& tables() { return *tables_for(QLORA_CODEBOOK_NF4); }
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -274,8 +292,7 @@ BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
 // ------------------------------------------------------------------ launches
 template <typename Tin>
 int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
-                    float* mean, void* ws, cudaStream_t st) {
-  const Tables& tb = tables();
+                    float* mean, void* ws, cudaStream_t st, const Tables& tb = tables()) {
   const int64_t n_blocks = rows * cols / 64;
   const QuantWs w = quant_ws(rows, cols);
   float* absmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.absmax_off);
@@ -562,6 +579,33 @@ int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint
 }
 
 int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
+  return qlora_dequantize_codebook(QLORA_CODEBOOK_NF4, w, W_out, stream);
+}
+
+int qlora_codebook(int kind, float levels[16], float thresholds[15]) {
+  const Tables* t = tables_for(kind);
+  if (t == nullptr || levels == nullptr) return QLORA_ERR_INVALID_ARG;
+  std::memcpy(levels, t->L.v, sizeof(t->L.v));
+  if (thresholds != nullptr) std::memcpy(thresholds, t->T.v, sizeof(t->T.v));
+  return QLORA_OK;
+}
+
+int qlora_quantize_codebook(int kind, const float* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8,
+                            float* step2, float* mean, void* workspace, size_t workspace_bytes, void* stream) {
+  const Tables* tb = tables_for(kind);
+  if (tb == nullptr) return QLORA_ERR_INVALID_ARG;
+  if (!W || !codes || !q8 || !step2 || !mean) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 16) || !aligned(q8, 16) || !aligned(step2, 16) || !aligned(mean, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (rows < 1 || cols < 64 || cols % 64 != 0 || rows * cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const QuantWs w = quant_ws(rows, cols);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
+  return launch_quantize(W, rows, cols, codes, q8, step2, mean, workspace, static_cast<cudaStream_t>(stream), *tb);
+}
+
+int qlora_dequantize_codebook(int kind, const qlora_nf4_weight* w, uint16_t* W_out, void* stream) {
+  const Tables* tb = tables_for(kind);
+  if (tb == nullptr) return QLORA_ERR_INVALID_ARG;
   if (!weight_ok(w) || !W_out || !aligned(W_out, 16)) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 64 || w->cols % 64 != 0 || w->rows * w->cols > (1ll << 40))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
@@ -571,7 +615,7 @@ int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* strea
   {
     LaunchTimer lt_("dequantize", static_cast<cudaStream_t>(stream));
     qnf4::nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      w->codes, w->q8, w->step2, w->mean, halves, W_out, tables().L);
+      w->codes, w->q8, w->step2, w->mean, halves, W_out, tb->L);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;

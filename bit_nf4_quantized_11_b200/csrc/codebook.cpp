@@ -62,4 +62,19 @@ void build_codebook(float levels[16], float thresholds[15]) {
   }
 }
 
+// Uniform INT4 comparison code: levels fp32(k/7) for k = -7..7 at codes
+// 0..14 (zero at code 7), code 15 a second +1; thresholds as above.
+void build_int4_codebook(float levels[16], float thresholds[15]) {
+  for (int k = 0; k < 15; ++k) levels[k] = static_cast<float>((k - 7) / 7.0);
+  levels[15] = 1.0f;
+  if (thresholds != nullptr) {
+    for (int j = 0; j < 15; ++j) {
+      const double mid = 0.5 * (static_cast<double>(levels[j]) + static_cast<double>(levels[j + 1]));
+      float t = static_cast<float>(mid);
+      if (static_cast<double>(t) > mid) t = std::nextafter(t, -INFINITY);
+      thresholds[j] = t;
+    }
+  }
+}
+
 }  // namespace qnf4_host

@@ -148,6 +148,38 @@ int qlora_quantize_nf4(const float* W, int64_t rows, int64_t cols,
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Codebooks.  QLORA_CODEBOOK_NF4 is the NF4 code of qlora_nf4_codebook.
+ * QLORA_CODEBOOK_INT4 is the uniform INT4 absmax code the pages compare NF4
+ * with (learn-interview-questions QLoRA page, section 2, NF4 vs. Standard
+ * INT4; llm-compass, 方法与公式 item 1): levels fp32(k/7) for k = -7..7 at
+ * codes 0..14 (zero at code 7), code 15 a second +1.  Both run through the
+ * same kernels; only the 16-entry level table and its thresholds differ.
+ */
+#define QLORA_CODEBOOK_NF4 0
+#define QLORA_CODEBOOK_INT4 1
+
+/*
+ * qlora_codebook -- host only: the 16 levels and 15 thresholds (exact
+ * midpoints of consecutive levels rounded toward -infinity) of a codebook
+ * kind.  Returns QLORA_ERR_INVALID_ARG for an unknown kind.
+ */
+int qlora_codebook(int kind, float levels[16], float thresholds[15]);
+
+/*
+ * qlora_quantize_codebook / qlora_dequantize_codebook -- qlora_quantize_nf4
+ * and qlora_dequantize_nf4 with the levels of codebook `kind` (same blocks,
+ * normalisation, tie rule, packing, double quantization, dequantization and
+ * workspace).  The stored weight does not record its codebook: dequantize it
+ * with the kind it was quantized with.  The linear-layer calls use NF4.
+ * Returns as qlora_quantize_nf4 / qlora_dequantize_nf4, and
+ * QLORA_ERR_INVALID_ARG for an unknown kind.
+ */
+int qlora_quantize_codebook(int kind, const float* W, int64_t rows, int64_t cols,
+                            uint8_t* codes, int8_t* q8, float* step2, float* mean,
+                            void* workspace, size_t workspace_bytes, void* stream);
+int qlora_dequantize_codebook(int kind, const qlora_nf4_weight* w, uint16_t* W_out, void* stream);
+
+/*
  * qlora_quantize_nf4_bf16 -- qlora_quantize_nf4 for a weight loaded in bf16
  * (the 16-bit checkpoint form; "QLoRA: Fine-Tuning on One Consumer GPU",
  * skillbyai, Merging the adapter for serving, loads the base in bfloat16).

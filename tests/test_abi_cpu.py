@@ -15,7 +15,7 @@ import numpy as np
 import pytest
 
 import bit_nf4_quantized_11_b200 as q
-from oracle import nf4
+from oracle import int4, nf4
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
@@ -52,6 +52,23 @@ def test_library_codebook_equals_oracle_bit_for_bit(lib):
 
 def test_codebook_null_levels_rejected(lib):
     assert lib.qlora_nf4_codebook(None, None) == EINVAL
+
+
+def test_int4_codebook_equals_oracle_bit_for_bit(lib):
+    lv, th = q.codebook(q.CODEBOOK_INT4)
+    assert np.array_equal(np.array(lv, dtype=np.float32).view(np.uint32), nf4.f32_bits(int4.levels()))
+    mid = int4.midpoints()
+    th32 = np.array(th, dtype=np.float32).astype(np.float64)
+    assert np.all(th32 <= mid) and np.all(np.nextafter(th32.astype(np.float32), np.float32(2)) > mid)
+    lv2, _ = q.codebook(q.CODEBOOK_NF4)
+    assert lv2 == q.codebook()[0]
+
+
+def test_codebook_kind_rejected(lib):
+    lv = (ctypes.c_float * 16)()
+    assert lib.qlora_codebook(2, lv, None) == EINVAL
+    assert lib.qlora_codebook(-1, lv, None) == EINVAL
+    assert lib.qlora_quantize_codebook(7, FAKE, 64, 64, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == EINVAL
 
 
 def test_status_strings(lib):
