@@ -33,7 +33,7 @@ exactly without relying on any fp32 hardware path.
 Modules:
   nf4       codebook, thresholds, blockwise quantize, double quantization,
             dequantize, nibble packing
-  linear    QLoRA linear forward / backward in fp64
+  linear    QLoRA linear forward / backward in fp64, with and without LoRA dropout
   overhead  storage arithmetic of the quantization constants
   merge     adapter merge into a bf16 copy of the dequantized base
   int4      the uniform INT4 absmax code the pages compare NF4 with

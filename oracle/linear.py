@@ -77,3 +77,52 @@ def lora_grads(dh, x, A, B, alpha: float):
     g = dh @ B
     u = x @ A.T
     return s * (g.T @ x), s * (dh.T @ u)
+
+
+# --------------------------------------------------------------------------
+# LoRA dropout
+# --------------------------------------------------------------------------
+# The configurations on every page set lora_dropout = 0.05 ("QLoRA",
+# aigrafen.se, the LoraConfig of the code example; llm-compass, 实现要点;
+# skillbyai, Quantized base plus LoRA; learn-interview-questions, section 3).
+# Reading D1 (the pages give no formula): dropout acts on the input of the
+# LoRA branch only, with inverted scaling, and the keep mask is an input of
+# the layer (the caller draws it), so that
+#     h  = x W^T + s ((x * k) / (1 - p)) A^T B^T
+# and the backward is the exact gradient of that expression for the same k:
+#     dx = dh W + s ((dh B) A) * k / (1 - p)
+#     dB = s dh^T (((x * k) / (1 - p)) A^T)
+#     dA = s / (1 - p) (dh B)^T (x * k)
+# with k in {0, 1} per element of x and 0 <= p < 1.  The mask is stored as
+# bits: bit (i mod 8) of byte i // 8 of a row is the keep flag of column i.
+
+
+def unpack_keep(keep_bits, cols: int) -> np.ndarray:
+    """0/1 keep mask [M, cols] of bit-packed rows [M, cols/8] (bit i%8 of
+    byte i//8, least significant bit first)."""
+    kb = np.asarray(keep_bits, dtype=np.uint8)
+    out = np.zeros((kb.shape[0], cols), dtype=np.float64)
+    for i in range(cols):
+        out[:, i] = (kb[:, i // 8] >> (i % 8)) & 1
+    return out
+
+
+def linear_fwd_dropout(x, W, A, B, alpha: float, keep, p: float):
+    """h of reading D1 in fp64; also returns u = ((x * k) / (1 - p)) A^T."""
+    x, W, A, B, keep = _f64(x), _f64(W), _f64(A), _f64(B), _f64(keep)
+    s = float(alpha) / float(A.shape[0])
+    xd = x * keep / (1.0 - p)
+    u = xd @ A.T
+    return x @ W.T + s * (u @ B.T), u
+
+
+def linear_bwd_dropout(dh, x, W, A, B, alpha: float, keep, p: float):
+    """(dx, dA, dB) of L = sum(dh * h) for the forward of reading D1."""
+    dh, x, W, A, B, keep = _f64(dh), _f64(x), _f64(W), _f64(A), _f64(B), _f64(keep)
+    s = float(alpha) / float(A.shape[0])
+    g = dh @ B
+    xd = x * keep / (1.0 - p)
+    dx = dh @ W + s * (g @ A) * keep / (1.0 - p)
+    dB = s * (dh.T @ (xd @ A.T))
+    dA = s * (g.T @ xd)
+    return dx, dA, dB

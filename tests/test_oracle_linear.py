@@ -121,3 +121,59 @@ def test_lora_grads_equal_linear_bwd():
     _, dA, dB = linear.linear_bwd(dh, x, W, A, B, 3.0)
     gA, gB = linear.lora_grads(dh, x, A, B, 3.0)
     assert np.allclose(gA, dA, rtol=1e-13, atol=1e-14) and np.allclose(gB, dB, rtol=1e-13, atol=1e-14)
+
+
+# ---------------------------------------------------------------- LoRA dropout (reading D1)
+def _keep(M, n, seed, p=0.3):
+    return (np.random.default_rng(seed).random((M, n)) >= p).astype(np.float64)
+
+
+def test_keep_mask_unpacking_matches_numpy_bit_order():
+    rng = np.random.default_rng(5)
+    bits = rng.integers(0, 256, (3, 4), dtype=np.uint8)
+    want = np.unpackbits(bits, axis=1, bitorder="little").astype(np.float64)
+    assert np.array_equal(linear.unpack_keep(bits, 32), want)
+
+
+@pytest.mark.parametrize("p", [0.05, 0.5])
+def test_dropout_backward_matches_central_differences(p):
+    x, W, A, B, dh = _problem(seed=6)
+    keep = _keep(*x.shape, seed=7)
+    alpha = 4.0
+
+    def loss(xx, AA, BB):
+        h, _ = linear.linear_fwd_dropout(xx, W, AA, BB, alpha, keep, p)
+        return float((dh * h).sum())
+
+    dx, dA, dB = linear.linear_bwd_dropout(dh, x, W, A, B, alpha, keep, p)
+    for g, a in [(_fd(lambda P: loss(P, A, B), x), dx), (_fd(lambda P: loss(x, P, B), A), dA),
+                 (_fd(lambda P: loss(x, A, P), B), dB)]:
+        assert np.allclose(g, a, rtol=1e-9, atol=1e-11)
+
+
+def test_dropout_forward_brute_force_loops():
+    x, W, A, B, _ = _problem(M=2, n_in=4, n_out=3, r=2, seed=8)
+    keep = _keep(2, 4, seed=9, p=0.5)
+    alpha, p = 3.0, 0.25
+    s = alpha / 2
+    h, _ = linear.linear_fwd_dropout(x, W, A, B, alpha, keep, p)
+    for m in range(2):
+        for o in range(3):
+            v = sum(x[m, i] * W[o, i] for i in range(4))
+            for j in range(2):
+                v += s * B[o, j] * sum(x[m, i] * keep[m, i] / (1 - p) * A[j, i] for i in range(4))
+            assert abs(h[m, o] - v) < 1e-12
+
+
+def test_dropout_limits():
+    """All kept with p = 0 is the plain layer; nothing kept leaves the base
+    matmul and zero adapter gradients."""
+    x, W, A, B, dh = _problem(seed=10)
+    ones, zeros = np.ones_like(x), np.zeros_like(x)
+    h0, _ = linear.linear_fwd(x, W, A, B, 2.0)
+    h1, _ = linear.linear_fwd_dropout(x, W, A, B, 2.0, ones, 0.0)
+    assert np.allclose(h0, h1, rtol=0, atol=1e-13)
+    h2, _ = linear.linear_fwd_dropout(x, W, A, B, 2.0, zeros, 0.3)
+    assert np.allclose(h2, x @ W.T, rtol=0, atol=1e-13)
+    dx, dA, dB = linear.linear_bwd_dropout(dh, x, W, A, B, 2.0, zeros, 0.3)
+    assert np.allclose(dx, dh @ W) and not dA.any() and not dB.any()
