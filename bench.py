@@ -28,6 +28,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -53,7 +54,7 @@ def parse():
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge"], default=None,
+    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout"], default=None,
                     help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -521,6 +522,39 @@ def comp_quantize(q, dev, peaks, src, reps=3):
     return out
 
 
+def comp_dropout(q, dev, peaks, n=50):
+    """fwd+bwd of the 7B attention projection with LoRA dropout p = 0.05 (the
+    pages' setting; keep mask drawn on the host), against the same step
+    without dropout; same FLOP count."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    a, b = ev(), ev()
+    M, n_in, n_out, r, alpha, p = 4096, 4096, 4096, 16, 32.0, 0.05
+    prob = synth.problem(M, n_in, n_out, r, seed=4)
+    w = q.quantize_nf4(prob["W"].to(dev))
+    x, A, B, dh = (prob[k].to(dev) for k in ("x", "A", "B", "dh"))
+    keep = torch.from_numpy(np.random.default_rng(4).random((M, n_in)) >= p).to(dev)
+    kb = q.pack_keep_mask(keep)
+    res = {}
+    for label, fwd, bwd in (("plain", lambda: q.linear_fwd(x, w, A, B, alpha),
+                             lambda us: q.linear_bwd(dh, x, us, w, A, B, alpha)),
+                            ("dropout_p0.05", lambda: q.linear_fwd_dropout(x, w, A, B, alpha, kb, p),
+                             lambda us: q.linear_bwd_dropout(dh, x, us, w, A, B, alpha, kb, p))):
+        for _ in range(3):
+            _, us = fwd()
+            bwd(us)
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(n):
+            _, us = fwd()
+            bwd(us)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / n
+        res[label] = {"ms": ms, "TFLOP/s": workloads.fwd_bwd_flops(M, n_in, n_out, r) / (ms * 1e-3) / 1e12}
+    res["dropout_overhead"] = res["dropout_p0.05"]["ms"] / res["plain"]["ms"] - 1.0
+    return {"lora_dropout_llama7b_attn": res}
+
+
 def comp_merge(q, dev, peaks, src, reps=5):
     """Adapter merge into a bf16 base and its lossy re-quantization to NF4, on
     the 7B attention projection (r=16) and the 65B down projection (r=64).
@@ -658,6 +692,8 @@ def components(q, dev, only=None):
         out.update(comp_workloads(q, dev, peaks))
     if only in (None, "merge"):
         out.update(comp_merge(q, dev, peaks, src))
+    if only in (None, "dropout"):
+        out.update(comp_dropout(q, dev, peaks))
     return out
 
 

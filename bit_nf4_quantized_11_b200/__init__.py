@@ -32,6 +32,7 @@ __all__ = [
     "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
     "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES", "merge_adapter",
     "quantize_codebook", "dequantize_codebook", "CODEBOOK_NF4", "CODEBOOK_INT4",
+    "linear_fwd_dropout", "linear_bwd_dropout", "pack_keep_mask", "OP_LINEAR_FWD_DROPOUT", "OP_LINEAR_BWD_DROPOUT",
     "OP_QUANTIZE", "OP_DEQUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD",
 ]
 
@@ -89,6 +90,8 @@ def load():
         "qlora_codebook": (I, [I, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float)]),
         "qlora_quantize_codebook": (I, [I, P, I64, I64, P, P, P, P, P, SZ, P]),
         "qlora_dequantize_codebook": (I, [I, W, P, P]),
+        "qlora_linear_fwd_dropout": (I, [P, I64, W, P, P, I, F, P, F, P, P, P, SZ, P]),
+        "qlora_linear_bwd_dropout": (I, [P, P, P, I64, W, P, P, I, F, P, F, P, P, P, P, SZ, P]),
         "qlora_timing_enable": (I, [I]),
         "qlora_timing_reset": (None, []),
         "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -305,6 +308,63 @@ def linear_bwd(dh, x, us, w: NF4Weight, A, B, alpha: float, dx=None, dA=None, dB
     return dx, dA, dB
 
 
+OP_LINEAR_FWD_DROPOUT, OP_LINEAR_BWD_DROPOUT = 4, 5
+
+
+def pack_keep_mask(keep: torch.Tensor) -> torch.Tensor:
+    """bool [M, n] keep mask -> the uint8 [M, n/8] bit layout of the dropout
+    calls (bit i % 8 of byte i // 8 keeps column i)."""
+    M, n = keep.shape
+    w = (1 << torch.arange(8, device=keep.device, dtype=torch.int32))
+    return (keep.reshape(M, n // 8, 8).to(torch.int32) * w).sum(-1).to(torch.uint8).contiguous()
+
+
+def linear_fwd_dropout(x, w: NF4Weight, A, B, alpha: float, keep_bits, p: float, h=None, us=None, workspace=None):
+    """Forward with LoRA dropout on the adapter input: h = x W0^T + us B^T,
+    us = bf16((alpha/r)/(1-p) (x * k) A^T); keep_bits uint8 [M, in/8]."""
+    M = x.shape[0]
+    r = A.shape[0]
+    _need(x, torch.bfloat16, "x", (M, w.cols))
+    _need(A, torch.bfloat16, "A", (r, w.cols))
+    _need(B, torch.bfloat16, "B", (w.rows, r))
+    _need(keep_bits, torch.uint8, "keep_bits", (M, w.cols // 8))
+    h = h if h is not None else torch.empty((M, w.rows), dtype=torch.bfloat16, device=x.device)
+    us = us if us is not None else torch.empty((M, r), dtype=torch.bfloat16, device=x.device)
+    _need(h, torch.bfloat16, "h", (M, w.rows))
+    _need(us, torch.bfloat16, "us", (M, r))
+    ws = _workspace(workspace_size(OP_LINEAR_FWD_DROPOUT, M, w.cols, w.rows, r), x.device, workspace)
+    cw = w._c()
+    _check(load().qlora_linear_fwd_dropout(_ptr(x), M, ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha),
+                                           _ptr(keep_bits), float(p), _ptr(h), _ptr(us), _ptr(ws),
+                                           ws.numel() if ws is not None else 0, _stream()),
+           "qlora_linear_fwd_dropout")
+    return h, us
+
+
+def linear_bwd_dropout(dh, x, us, w: NF4Weight, A, B, alpha: float, keep_bits, p: float, dx=None, dA=None, dB=None,
+                       workspace=None):
+    """Backward of :func:`linear_fwd_dropout` (same keep_bits and p)."""
+    M = x.shape[0]
+    r = A.shape[0]
+    _need(dh, torch.bfloat16, "dh", (M, w.rows))
+    _need(x, torch.bfloat16, "x", (M, w.cols))
+    _need(us, torch.bfloat16, "us", (M, r))
+    _need(A, torch.bfloat16, "A", (r, w.cols))
+    _need(B, torch.bfloat16, "B", (w.rows, r))
+    _need(keep_bits, torch.uint8, "keep_bits", (M, w.cols // 8))
+    dev = x.device
+    dx = dx if dx is not None else torch.empty((M, w.cols), dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty((r, w.cols), dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty((w.rows, r), dtype=torch.float32, device=dev)
+    ws = _workspace(workspace_size(OP_LINEAR_BWD_DROPOUT, M, w.cols, w.rows, r), dev, workspace)
+    cw = w._c()
+    _check(load().qlora_linear_bwd_dropout(_ptr(dh), _ptr(x), _ptr(us), M, ctypes.byref(cw), _ptr(A), _ptr(B), r,
+                                           float(alpha), _ptr(keep_bits), float(p), _ptr(dx), _ptr(dA), _ptr(dB),
+                                           _ptr(ws), ws.numel() if ws is not None else 0, _stream()),
+           "qlora_linear_bwd_dropout")
+    return dx, dA, dB
+
+
 def last_device_status() -> int:
     """Synchronize the current stream, read and clear the device error flag."""
     return int(load().qlora_last_device_status(_stream()))
@@ -320,7 +380,7 @@ def selftest_wait_timeout() -> int:
 
 KERNEL_NAMES = ("quantize_blocks", "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
                 "gemv", "gemv_finalize", "lora_rowwise", "lora_rowwise_du", "lora_colwise",
-                "merge_adapter")
+                "merge_adapter", "dropout_mask", "dropout_dx")
 
 
 def timing_enable(on: bool = True) -> bool:

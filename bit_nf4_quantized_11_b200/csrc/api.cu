@@ -20,6 +20,7 @@
 #include "gemm_pair_sm100.cuh"
 #include "gemv.cuh"
 #include "merge.cuh"
+#include "dropout.cuh"
 #include "quant.cuh"
 #include "skinny.cuh"
 
@@ -276,6 +277,12 @@ size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
   return M <= 16 ? gemv_ws(M, in, out) : 0;
 }
 
+size_t masked_x_bytes(int64_t M, int64_t in) { return round256(static_cast<size_t>(M) * in * 2); }
+
+size_t fwd_dropout_ws(int64_t M, int64_t in, int64_t out, int r) {
+  return masked_x_bytes(M, in) + fwd_ws(M, in, out, r);
+}
+
 struct BwdWs {
   size_t du_off, total;
 };
@@ -393,7 +400,8 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
                 cudaStream_t st) {
   CUtensorMap tm_act, tm_lora;
   if (!make_tmap_bf16(&tm_act, act, M, K)) return QLORA_ERR_CUDA;
-  if (!make_tmap_bf16(&tm_lora, lora_act, M, r)) return QLORA_ERR_CUDA;
+  if (r == 0) tm_lora = tm_act;                  // no rank-r tail: the map is never used
+  else if (!make_tmap_bf16(&tm_lora, lora_act, M, r)) return QLORA_ERR_CUDA;
   qnf4::GemmArgs a{};
   a.codes = w->codes;
   a.q8 = w->q8;
@@ -461,9 +469,9 @@ int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_
 // dB = dh^T us -> [out, r] and dA = du^T x -> [r, in] in one launch: column
 // tiles x token chunks x the two problems, chunks of a tile in one cluster.
 int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
-                      int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st) {
-  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0};
-  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1};
+                      int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st, float dA_scale = 1.f) {
+  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0, 1.f};
+  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale};
   const int smem = qnf4::kColStages * qnf4::kColStageBytes;
   QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::colwise_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int chunk_tokens = col_chunk_tokens(M);
@@ -504,6 +512,81 @@ int check_linear_shapes(int64_t M, const qlora_nf4_weight* w, int r) {
   return QLORA_OK;
 }
 
+// Forward after validation: us = bf16(s_lora * x_lora A^T) (x_lora = x, or
+// the masked x of LoRA dropout with s_lora = s / (1 - p)), then
+// h = [x | us] [W0 | B]^T; `workspace` is the GEMV part (M <= 16).
+int linear_fwd_impl(const uint16_t* x, const uint16_t* x_lora, int64_t M, const qlora_nf4_weight* w,
+                    const uint16_t* A, const uint16_t* B, int r, float s_lora, uint16_t* h, uint16_t* us_out,
+                    void* workspace, cudaStream_t st) {
+  const int64_t in = w->cols, out = w->rows;
+  int rc = launch_rowwise<false>(x_lora, A, us_out, M, in, r, s_lora, st);   // us = bf16(s x A^T)
+  if (rc != QLORA_OK) return rc;
+  if (M <= 16) {
+    const GemvPlan p = gemv_plan(in, out);
+    qnf4::GemvArgs g{};
+    g.q8 = w->q8;
+    g.step2 = w->step2;
+    g.mean = w->mean;
+    g.part = static_cast<float*>(workspace);
+    g.M = static_cast<int>(M);
+    g.in = static_cast<int>(in);
+    g.out = static_cast<int>(out);
+    g.n_st = p.n_st;
+    g.n_units = p.n_units;
+    g.local_tiles = p.local_tiles;
+    g.timeout_ns = g_timeout_ns.load();
+    g.L = tables().L;
+    CUtensorMap tm_codes, tm_x;
+    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)) ||
+        !make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(M), static_cast<uint64_t>(in), M > 8 ? 16 : 8))
+      return QLORA_ERR_CUDA;
+    {
+      LaunchTimer lt_("gemv", st);
+      const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
+      auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
+                         : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
+      QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qnf4::kGvSmem));
+      kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
+    }
+    QLORA_CUDA_TRY(cudaGetLastError());
+    const int64_t n_el = M * out;
+    {
+      LaunchTimer lt_("gemv_finalize", st);
+      qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
+          g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
+    }
+    QLORA_CUDA_TRY(cudaGetLastError());
+    return QLORA_OK;
+  }
+  return launch_gemm(false, w, x, M, in, us_out, B, r, h, out, st);  // h = [x|us] [W0|B]^T
+}
+
+int check_fwd_args(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
+                   int r, float alpha, const uint16_t* h, const uint16_t* us_out) {
+  if (!x || !weight_ok(w) || !A || !B || !h || !us_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(h, 16) || !aligned(us_out, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  return check_linear_shapes(M, w, r);
+}
+
+int check_dropout_args(const uint8_t* keep_bits, float p) {
+  if (keep_bits == nullptr || !(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+int launch_mask_apply(const uint16_t* x, const uint8_t* keep_bits, int64_t M, int64_t n, uint16_t* x_m,
+                      cudaStream_t st) {
+  const int64_t units = M * (n / 8);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+  {
+    LaunchTimer lt_("dropout_mask", st);
+    qnf4::mask_apply_kernel<<<grid, 256, 0, st>>>(x, keep_bits, M, n, x_m);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -531,6 +614,12 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t in_features, int64_t out_
     case QLORA_OP_LINEAR_BWD:
       if (M < 1 || r < 1) return 0;
       return bwd_ws(M, in_features, out_features, r).total;
+    case QLORA_OP_LINEAR_FWD_DROPOUT:
+      if (M < 1) return 0;
+      return fwd_dropout_ws(M, in_features, out_features, r);
+    case QLORA_OP_LINEAR_BWD_DROPOUT:
+      if (M < 1 || r < 1) return 0;
+      return bwd_ws(M, in_features, out_features, r).total + masked_x_bytes(M, in_features);
     default:
       return static_cast<size_t>(-1);
   }
@@ -624,59 +713,31 @@ int qlora_dequantize_codebook(int kind, const qlora_nf4_weight* w, uint16_t* W_o
 int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
                      const uint16_t* B, int r, float alpha, uint16_t* h, uint16_t* us_out, void* workspace,
                      size_t workspace_bytes, void* stream) {
-  if (!x || !weight_ok(w) || !A || !B || !h || !us_out) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(h, 16) || !aligned(us_out, 16))
-    return QLORA_ERR_INVALID_ARG;
-  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-  const int sc = check_linear_shapes(M, w, r);
+  const int sc = check_fwd_args(x, M, w, A, B, r, alpha, h, us_out);
   if (sc != QLORA_OK) return sc;
-  const int64_t in = w->cols, out = w->rows;
-  const size_t need = fwd_ws(M, in, out, r);
+  const size_t need = fwd_ws(M, w->cols, w->rows, r);
   if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
     return QLORA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const float s = alpha / static_cast<float>(r);
+  return linear_fwd_impl(x, x, M, w, A, B, r, alpha / static_cast<float>(r), h, us_out, workspace,
+                         static_cast<cudaStream_t>(stream));
+}
 
-  int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s, st);             // us = bf16(s x A^T)
+int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
+                             const uint16_t* B, int r, float alpha, const uint8_t* keep_bits, float p, uint16_t* h,
+                             uint16_t* us_out, void* workspace, size_t workspace_bytes, void* stream) {
+  int sc = check_fwd_args(x, M, w, A, B, r, alpha, h, us_out);
+  if (sc != QLORA_OK) return sc;
+  if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
+  const int64_t in = w->cols;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < fwd_dropout_ws(M, in, w->rows, r))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint16_t* x_m = static_cast<uint16_t*>(workspace);
+  int rc = launch_mask_apply(x, keep_bits, M, in, x_m, st);                 // x_m = x * k
   if (rc != QLORA_OK) return rc;
-  if (M <= 16) {
-    const GemvPlan p = gemv_plan(in, out);
-    qnf4::GemvArgs g{};
-    g.q8 = w->q8;
-    g.step2 = w->step2;
-    g.mean = w->mean;
-    g.part = static_cast<float*>(workspace);
-    g.M = static_cast<int>(M);
-    g.in = static_cast<int>(in);
-    g.out = static_cast<int>(out);
-    g.n_st = p.n_st;
-    g.n_units = p.n_units;
-    g.local_tiles = p.local_tiles;
-    g.timeout_ns = g_timeout_ns.load();
-    g.L = tables().L;
-    CUtensorMap tm_codes, tm_x;
-    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)) ||
-        !make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(M), static_cast<uint64_t>(in), M > 8 ? 16 : 8))
-      return QLORA_ERR_CUDA;
-    {
-      LaunchTimer lt_("gemv", st);
-      const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
-      auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
-                         : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
-      QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qnf4::kGvSmem));
-      kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
-    }
-    QLORA_CUDA_TRY(cudaGetLastError());
-    const int64_t n_el = M * out;
-    {
-      LaunchTimer lt_("gemv_finalize", st);
-      qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
-          g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
-    }
-    QLORA_CUDA_TRY(cudaGetLastError());
-    return QLORA_OK;
-  }
-  return launch_gemm(false, w, x, M, in, us_out, B, r, h, out, st);  // h = [x|us] [W0|B]^T
+  const float s_lora = (alpha / static_cast<float>(r)) / (1.f - p);
+  return linear_fwd_impl(x, x_m, M, w, A, B, r, s_lora, h, us_out,
+                         static_cast<uint8_t*>(workspace) + masked_x_bytes(M, in), st);
 }
 
 int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
@@ -702,6 +763,45 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, 
   rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
   if (rc != QLORA_OK) return rc;
   return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st);                // dB, dA
+}
+
+int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
+                             const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             const uint8_t* keep_bits, float p, uint16_t* dx, float* dA, float* dB, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!dh || !x || !us || !weight_ok(w) || !A || !B || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(dh, 16) || !aligned(x, 16) || !aligned(us, 16) || !aligned(A, 16) || !aligned(B, 16) ||
+      !aligned(dx, 16) || !aligned(dA, 16) || !aligned(dB, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  int sc = check_linear_shapes(M, w, r);
+  if (sc != QLORA_OK) return sc;
+  if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
+  const int64_t in = w->cols, out = w->rows;
+  const BwdWs ws = bwd_ws(M, in, out, r);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total + masked_x_bytes(M, in))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
+  uint16_t* x_m = reinterpret_cast<uint16_t*>(base + ws.total);
+  const float s = alpha / static_cast<float>(r);
+  const float inv_keep = 1.f / (1.f - p);
+
+  int rc = launch_mask_apply(x, keep_bits, M, in, x_m, st);                           // x_m = x * k
+  if (rc != QLORA_OK) return rc;
+  rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                              // du = bf16(s dh B)
+  if (rc != QLORA_OK) return rc;
+  rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);              // dx = dh W0
+  if (rc != QLORA_OK) return rc;
+  {
+    const int64_t units = cdiv(M, qnf4::kDxRows) * (in / 8);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+    LaunchTimer lt_("dropout_dx", st);
+    qnf4::dropout_dx_kernel<<<grid, 256, 0, st>>>(dx, du, A, keep_bits, M, in, r, inv_keep);  // + (du A) k/(1-p)
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return launch_lora_grads(dh, us, x_m, du, M, in, out, r, dB, dA, st, inv_keep);   // dB, dA
 }
 
 int qlora_last_device_status(void* stream) {

@@ -239,6 +239,7 @@ struct ColProblem {
   float* out;            // [P][R] (dB) or [R][P] (dA)
   int P;
   int n_major;           // 1: output layout [n][p]
+  float scale;           // applied to the reduced sum before it is stored
 };
 
 __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem prob0, ColProblem prob1,
@@ -352,7 +353,11 @@ __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem 
       constexpr int n4 = 128 * 64 / 4;
       const uint32_t red_addr = smem_u32(red);
       for (int e = rank * n4 / ks + threadIdx.x; e < (rank + 1) * n4 / ks; e += kColThreads) {
-        const float4 v = cluster_sum_f4(red_addr + e * 16, ks);
+        float4 v = cluster_sum_f4(red_addr + e * 16, ks);
+        if (pr.scale != 1.f) {
+          v.x = __fmul_rn(v.x, pr.scale); v.y = __fmul_rn(v.y, pr.scale);
+          v.z = __fmul_rn(v.z, pr.scale); v.w = __fmul_rn(v.w, pr.scale);
+        }
         if (pr.n_major) {                                            // red [n][p]: 4 consecutive p
           const int nl = e / 32, pl = (e % 32) * 4;
           if (nl < 8 * nt && p0 + pl < P)

@@ -73,7 +73,9 @@ enum {
   QLORA_OP_QUANTIZE = 0,
   QLORA_OP_DEQUANTIZE = 1,
   QLORA_OP_LINEAR_FWD = 2,
-  QLORA_OP_LINEAR_BWD = 3
+  QLORA_OP_LINEAR_BWD = 3,
+  QLORA_OP_LINEAR_FWD_DROPOUT = 4,
+  QLORA_OP_LINEAR_BWD_DROPOUT = 5
 };
 
 /* A quantized weight: device pointers in the format described above. */
@@ -275,6 +277,37 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us,
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * qlora_linear_fwd_dropout / qlora_linear_bwd_dropout -- the layer with LoRA
+ * dropout on the adapter input (lora_dropout = 0.05 in every configuration on
+ * the pages: "QLoRA", aigrafen.se; llm-compass, 实现要点; skillbyai;
+ * learn-interview-questions, section 3).  With keep mask k (0/1 per element
+ * of x) and drop probability p, inverted scaling:
+ *   h  = x W0^T + s ((x * k) / (1 - p)) A^T B^T
+ *   dx = dh W0 + s ((dh B) A) * k / (1 - p)
+ *   dB = dh^T us,  dA = du^T (x * k) / (1 - p)
+ * with us = bf16((s / (1 - p)) (x * k) A^T) (returned by the forward and
+ * passed to the backward), du = bf16(s dh B); the backward must receive the
+ * same k and p as the forward.  The base GEMMs are those of
+ * qlora_linear_fwd / _bwd; dx adds the masked rank-r term to the bf16 result
+ * of dh W0 in fp32 and rounds again to bf16.
+ *
+ * keep_bits  device uint8 [M, in/8]: bit (i % 8) of byte i/8 of row m is the
+ *            keep flag of x[m][i] (the caller draws the mask).
+ * p          drop probability, 0 <= p < 1.
+ * workspace: qlora_workspace_size(QLORA_OP_LINEAR_FWD_DROPOUT / _BWD_DROPOUT,
+ *            M, in, out, r) bytes.  Other arguments, rules and returns as
+ *            qlora_linear_fwd / qlora_linear_bwd; QLORA_ERR_INVALID_ARG for a
+ *            null mask or p outside [0, 1).
+ */
+int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
+                             const uint16_t* B, int r, float alpha, const uint8_t* keep_bits, float p, uint16_t* h,
+                             uint16_t* us_out, void* workspace, size_t workspace_bytes, void* stream);
+int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
+                             const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                             const uint8_t* keep_bits, float p, uint16_t* dx, float* dA, float* dB, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * qlora_last_device_status -- synchronizes `stream`, then reads and clears
  * the current device's error flag.  Kernels that wait on another part of the
  * device (pipeline barriers inside the GEMMs) give up after a bounded time
@@ -309,7 +342,7 @@ int qlora_selftest_wait_timeout(void* stream);
  * the number of launches since the last reset.  Names: "quantize_blocks",
  * "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
  * "gemv", "gemv_finalize", "lora_rowwise" (us), "lora_rowwise_du" (du),
- * "lora_colwise" (dA and dB), "merge_adapter".  Events are created by the library on first use (host-side
+ * "lora_colwise" (dA and dB), "merge_adapter", "dropout_mask", "dropout_dx".  Events are created by the library on first use (host-side
  * CUDA objects, no device memory).  Not for use during stream capture.
  *
  * qlora_timing_enable: on != 0 enables, 0 disables; returns the previous state.
