@@ -83,6 +83,13 @@ def test_few_token_ragged(cuda_lib, M, n_in, n_out):
     _run(cuda_lib, M, n_in, n_out, 8, 16.0, seed=100 + M, backward=False)
 
 
+@pytest.mark.parametrize("M,n_in,n_out", [(4096, 512, 2560), (4096, 2560, 512)])
+def test_two_waves_short_k(cuda_lib, M, n_in, n_out):
+    # 80 output tiles of 512 x 256: more tiles than co-resident CTA pairs, so
+    # pairs take a second tile; short K on one side, forward and dx in turn
+    _run(cuda_lib, M, n_in, n_out, 16, 32.0, seed=M + n_in)
+
+
 def test_zero_adapter_is_plain_quantized_matmul(cuda_lib):
     """B = 0: h equals x dequant(W0)^T, dA = 0 exactly."""
     q = cuda_lib
