@@ -34,6 +34,7 @@ __all__ = [
     "quantize_codebook", "dequantize_codebook", "CODEBOOK_NF4", "CODEBOOK_INT4",
     "linear_fwd_dropout", "linear_bwd_dropout", "pack_keep_mask", "OP_LINEAR_FWD_DROPOUT", "OP_LINEAR_BWD_DROPOUT",
     "OP_QUANTIZE", "OP_DEQUANTIZE", "OP_LINEAR_FWD", "OP_LINEAR_BWD",
+    "quantize_shard_plan", "quantize_shard_workspace_size", "quantize_nf4_shard_local", "quantize_nf4_shard_finish",
 ]
 
 OP_QUANTIZE, OP_DEQUANTIZE, OP_LINEAR_FWD, OP_LINEAR_BWD = 0, 1, 2, 3
@@ -92,6 +93,11 @@ def load():
         "qlora_dequantize_codebook": (I, [I, W, P, P]),
         "qlora_linear_fwd_dropout": (I, [P, I64, W, P, P, I, F, P, F, P, P, P, SZ, P]),
         "qlora_linear_bwd_dropout": (I, [P, P, P, I64, W, P, P, I, F, P, F, P, P, P, P, SZ, P]),
+        "qlora_quantize_shard_plan": (I, [I64, I, I, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
+                                          ctypes.POINTER(ctypes.c_int64)]),
+        "qlora_quantize_shard_workspace_size": (SZ, [I64, I64]),
+        "qlora_quantize_nf4_shard_local": (I, [P, I64, P, P, I64, P, SZ, P]),
+        "qlora_quantize_nf4_shard_finish": (I, [P, I64, I64, I64, P, P, P, P, SZ, P]),
         "qlora_timing_enable": (I, [I]),
         "qlora_timing_reset": (None, []),
         "qlora_timing_collect": (I, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double),
@@ -230,6 +236,56 @@ def quantize_nf4(W: torch.Tensor, out: NF4Weight | None = None, workspace=None) 
     _check(fn(_ptr(W), rows, cols, _ptr(w.codes), _ptr(w.q8), _ptr(w.step2), _ptr(w.mean), _ptr(ws),
               ws.numel() if ws is not None else 0, _stream()), name)
     return w
+
+
+def quantize_shard_plan(n_blocks_total: int, world: int, rank: int) -> tuple[int, int, int]:
+    """(block_begin, block_end, roots_per_rank) of `rank`'s slice of a weight
+    of n_blocks_total 64-weight blocks split over `world` ranks."""
+    b0, b1, cpr = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(load().qlora_quantize_shard_plan(int(n_blocks_total), int(world), int(rank), ctypes.byref(b0),
+                                            ctypes.byref(b1), ctypes.byref(cpr)), "qlora_quantize_shard_plan")
+    return b0.value, b1.value, cpr.value
+
+
+def quantize_shard_workspace_size(n_blocks_shard: int, n_roots_total: int) -> int:
+    n = load().qlora_quantize_shard_workspace_size(int(n_blocks_shard), int(n_roots_total))
+    if n == ctypes.c_size_t(-1).value:
+        raise QLoRAError(-1, "qlora_quantize_shard_workspace_size")
+    return int(n)
+
+
+def quantize_nf4_shard_local(W_shard: torch.Tensor, roots_per_rank: int, n_roots_total: int):
+    """First half of a sharded quantization: (codes uint8 [n_blocks_shard*32],
+    roots fp64 [roots_per_rank], workspace) for a shard given as fp32 weights
+    (any shape, numel % 64 == 0).  Keep the workspace for the finishing call."""
+    _need(W_shard, torch.float32, "W_shard")
+    if W_shard.numel() % 64:
+        raise ValueError("a shard holds whole 64-weight blocks")
+    nb = W_shard.numel() // 64
+    dev = W_shard.device
+    codes = torch.empty(nb * 32, dtype=torch.uint8, device=dev)
+    roots = torch.empty(roots_per_rank, dtype=torch.float64, device=dev)
+    ws = torch.empty(quantize_shard_workspace_size(nb, n_roots_total), dtype=torch.uint8, device=dev)
+    _check(load().qlora_quantize_nf4_shard_local(_ptr(W_shard) if nb else None, nb, _ptr(codes) if nb else None,
+                                                 _ptr(roots), int(roots_per_rank), _ptr(ws), ws.numel(), _stream()),
+           "qlora_quantize_nf4_shard_local")
+    return codes, roots, ws
+
+
+def quantize_nf4_shard_finish(roots_all: torch.Tensor, n_blocks_total: int, n_blocks_shard: int,
+                              workspace: torch.Tensor):
+    """Second half: (q8 int8 [n_blocks_shard], step2 fp32 [ceil(n_blocks_shard/256)],
+    mean fp32 [1]) from the all-gathered roots (fp64, rank order)."""
+    _need(roots_all, torch.float64, "roots_all")
+    dev = roots_all.device
+    q8 = torch.empty(n_blocks_shard, dtype=torch.int8, device=dev)
+    step2 = torch.empty((n_blocks_shard + 255) // 256, dtype=torch.float32, device=dev)
+    mean = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(load().qlora_quantize_nf4_shard_finish(_ptr(roots_all), roots_all.numel(), int(n_blocks_total),
+                                                  int(n_blocks_shard), _ptr(q8), _ptr(step2), _ptr(mean),
+                                                  _ptr(workspace), workspace.numel(), _stream()),
+           "qlora_quantize_nf4_shard_finish")
+    return q8, step2, mean
 
 
 def merge_adapter(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,

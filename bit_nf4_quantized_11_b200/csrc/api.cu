@@ -297,16 +297,10 @@ BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
 }
 
 // ------------------------------------------------------------------ launches
+// K1: codes and block absmaxes.  Also resets tickets[0] for the tree pass after it.
 template <typename Tin>
-int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
-                    float* mean, void* ws, cudaStream_t st, const Tables& tb = tables()) {
-  const int64_t n_blocks = rows * cols / 64;
-  const QuantWs w = quant_ws(rows, cols);
-  float* absmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.absmax_off);
-  double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + w.tree_off);
-
-  unsigned int* tickets = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + w.ticket_off);
-
+int launch_blocks(const Tin* W, int64_t n_blocks, uint8_t* codes, float* absmax, unsigned int* tickets,
+                  const Tables& tb, cudaStream_t st) {
   const int sms = device_sm_count();
   const int64_t want = cdiv(n_blocks, 64 * qnf4::kQRounds);       // 8 warps x 8 blocks x rounds per CTA
   // one wave: 4 CTAs of 256 threads fit an SM at the kernel's register count
@@ -316,17 +310,24 @@ int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, in
     qnf4::nf4_quantize_blocks_kernel<Tin><<<grid1, 256, 0, st>>>(W, n_blocks, codes, absmax, tb.C, tickets);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
 
-  // fixed summation tree: 4096x reductions; the pass that leaves at most
-  // kTreeTop sums is finished (and the mean written) by its last CTA.  Each
-  // pass resets the ticket of the pass after it (they alternate).
-  int64_t n = n_blocks;
+// Fixed summation tree from `n` leaves (block absmaxes, or the fp64 sums of
+// 4096-leaf subtrees): 4096x reductions; the pass that leaves at most
+// kTreeTop sums is finished (and mean = fp32(total / n_leaves_total) written)
+// by its last CTA.  tickets[0] must be 0 on entry; each pass resets the
+// ticket of the pass after it (they alternate).  `tree` holds the sums of
+// every pass.
+template <typename T>
+int launch_mean_tree(const T* leaves, int64_t n, double* tree, unsigned int* tickets, int64_t n_leaves_total,
+                     float* mean, cudaStream_t st) {
   int64_t parts = cdiv(n, qnf4::kTreeChunk);
   int pass = 0;
   {
     LaunchTimer lt_("scale_mean_tree", st);
-    qnf4::pairwise_tree_kernel<float><<<static_cast<unsigned>(parts), 256, 0, st>>>(
-        absmax, n, tree, parts <= qnf4::kTreeTop, tickets, n_blocks, mean, tickets + 1);
+    qnf4::pairwise_tree_kernel<T><<<static_cast<unsigned>(parts), 256, 0, st>>>(
+        leaves, n, tree, parts <= qnf4::kTreeTop, tickets, n_leaves_total, mean, tickets + 1);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   double* prev = tree;
@@ -338,12 +339,17 @@ int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, in
     {
       LaunchTimer lt_("scale_mean_tree", st);
       qnf4::pairwise_tree_kernel<double><<<static_cast<unsigned>(parts), 256, 0, st>>>(
-          prev, n, next, parts <= qnf4::kTreeTop, tickets + (pass & 1), n_blocks, mean, tickets + ((pass + 1) & 1));
+          prev, n, next, parts <= qnf4::kTreeTop, tickets + (pass & 1), n_leaves_total, mean,
+          tickets + ((pass + 1) & 1));
     }
     QLORA_CUDA_TRY(cudaGetLastError());
     prev = next;
   }
+  return QLORA_OK;
+}
 
+// K3: second-level codes of n_blocks scales against a finished mean.
+int launch_dq(const float* absmax, int64_t n_blocks, const float* mean, int8_t* q8, float* step2, cudaStream_t st) {
   const int64_t n_groups = cdiv(n_blocks, qnf4::kGroup);
   {
     LaunchTimer lt_("dq_scales", st);
@@ -352,6 +358,43 @@ int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, in
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
+}
+
+template <typename Tin>
+int launch_quantize(const Tin* W, int64_t rows, int64_t cols, uint8_t* codes, int8_t* q8, float* step2,
+                    float* mean, void* ws, cudaStream_t st, const Tables& tb = tables()) {
+  const int64_t n_blocks = rows * cols / 64;
+  const QuantWs w = quant_ws(rows, cols);
+  float* absmax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w.absmax_off);
+  double* tree = reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + w.tree_off);
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + w.ticket_off);
+  int rc = launch_blocks(W, n_blocks, codes, absmax, tickets, tb, st);
+  if (rc != QLORA_OK) return rc;
+  rc = launch_mean_tree(static_cast<const float*>(absmax), n_blocks, tree, tickets, n_blocks, mean, st);
+  if (rc != QLORA_OK) return rc;
+  return launch_dq(absmax, n_blocks, mean, q8, step2, st);
+}
+
+// Sharded quantization: rank k of `world` takes the 4096-block chunks
+// [k cpr, (k+1) cpr) of the flattened weight, cpr = ceil(chunks / world), so
+// every shard starts on a chunk (hence on a 256-block group) boundary and
+// its chunk sums are exactly the first-pass sums of the unsharded tree.
+struct ShardWs {
+  size_t absmax_off, tree_off, ticket_off, total;
+};
+
+ShardWs shard_ws(int64_t n_blocks_shard, int64_t n_roots_total) {
+  ShardWs w{};
+  w.absmax_off = 0;
+  w.tree_off = round256(static_cast<size_t>(std::max<int64_t>(n_blocks_shard, 1)) * 4);
+  int64_t count = 0, n = n_roots_total;
+  do {
+    n = cdiv(n, qnf4::kTreeChunk);
+    count += n;
+  } while (n > qnf4::kTreeTop);
+  w.ticket_off = w.tree_off + round256(static_cast<size_t>(count) * 8);
+  w.total = w.ticket_off + 256;
+  return w;
 }
 
 int gemm_tile_m(int64_t M) {
@@ -645,6 +688,80 @@ int qlora_quantize_nf4_bf16(const uint16_t* W, int64_t rows, int64_t cols, uint8
   const QuantWs w = quant_ws(rows, cols);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
   return launch_quantize(W, rows, cols, codes, q8, step2, mean, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int qlora_quantize_shard_plan(int64_t n_blocks_total, int world, int rank, int64_t* block_begin,
+                              int64_t* block_end, int64_t* roots_per_rank) {
+  if (!block_begin || !block_end || !roots_per_rank) return QLORA_ERR_INVALID_ARG;
+  if (n_blocks_total < 1 || n_blocks_total > (1ll << 34) || world < 1 || rank < 0 || rank >= world)
+    return QLORA_ERR_INVALID_ARG;
+  const int64_t chunks = cdiv(n_blocks_total, qnf4::kTreeChunk);
+  const int64_t cpr = cdiv(chunks, world);
+  *block_begin = std::min(n_blocks_total, static_cast<int64_t>(rank) * cpr * qnf4::kTreeChunk);
+  *block_end = std::min(n_blocks_total, static_cast<int64_t>(rank + 1) * cpr * qnf4::kTreeChunk);
+  *roots_per_rank = cpr;
+  return QLORA_OK;
+}
+
+size_t qlora_quantize_shard_workspace_size(int64_t n_blocks_shard, int64_t n_roots_total) {
+  if (n_blocks_shard < 0 || n_roots_total < 1) return static_cast<size_t>(-1);
+  return shard_ws(n_blocks_shard, n_roots_total).total;
+}
+
+int qlora_quantize_nf4_shard_local(const float* W_shard, int64_t n_blocks_shard, uint8_t* codes_shard,
+                                   double* roots, int64_t roots_per_rank, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!roots || roots_per_rank < 1 || n_blocks_shard < 0) return QLORA_ERR_INVALID_ARG;
+  if (n_blocks_shard > roots_per_rank * qnf4::kTreeChunk) return QLORA_ERR_INVALID_ARG;
+  if (n_blocks_shard > 0 && (!W_shard || !codes_shard || !aligned(W_shard, 16) || !aligned(codes_shard, 16)))
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned(roots, 16)) return QLORA_ERR_INVALID_ARG;
+  const ShardWs w = shard_ws(n_blocks_shard, roots_per_rank);
+  // the block absmaxes and one ticket word (the rest of the workspace is the finishing call's)
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.tree_off + 256)
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  float* absmax = reinterpret_cast<float*>(base + w.absmax_off);
+  const int64_t parts = cdiv(n_blocks_shard, qnf4::kTreeChunk);
+  if (parts < roots_per_rank)                                       // chunks past the weight sum to zero
+    QLORA_CUDA_TRY(cudaMemsetAsync(roots + parts, 0, static_cast<size_t>(roots_per_rank - parts) * 8, st));
+  if (n_blocks_shard == 0) return QLORA_OK;
+  // K1 resets its ticket word; the single first tree pass below does not
+  // finish, so it neither reads nor moves a ticket.  Both live in the tree
+  // area of the workspace, which the finishing call reuses.
+  unsigned int* scratch_ticket = reinterpret_cast<unsigned int*>(base + w.tree_off);
+  int rc = launch_blocks(W_shard, n_blocks_shard, codes_shard, absmax, scratch_ticket, tables(), st);
+  if (rc != QLORA_OK) return rc;
+  {
+    LaunchTimer lt_("scale_mean_tree", st);
+    qnf4::pairwise_tree_kernel<float><<<static_cast<unsigned>(parts), 256, 0, st>>>(
+        absmax, n_blocks_shard, roots, 0, scratch_ticket, n_blocks_shard, nullptr, nullptr);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+int qlora_quantize_nf4_shard_finish(const double* roots_all, int64_t n_roots_total, int64_t n_blocks_total,
+                                    int64_t n_blocks_shard, int8_t* q8_shard, float* step2_shard, float* mean,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!roots_all || !mean || n_roots_total < 1 || n_blocks_total < 1 || n_blocks_shard < 0 ||
+      n_blocks_shard > n_blocks_total || n_blocks_total > n_roots_total * qnf4::kTreeChunk)
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned(roots_all, 16) || !aligned(mean, 16)) return QLORA_ERR_INVALID_ARG;
+  if (n_blocks_shard > 0 && (!q8_shard || !step2_shard || !aligned(q8_shard, 16) || !aligned(step2_shard, 16)))
+    return QLORA_ERR_INVALID_ARG;
+  const ShardWs w = shard_ws(n_blocks_shard, n_roots_total);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < w.total) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  const float* absmax = reinterpret_cast<const float*>(base + w.absmax_off);
+  double* tree = reinterpret_cast<double*>(base + w.tree_off);
+  unsigned int* tickets = reinterpret_cast<unsigned int*>(base + w.ticket_off);
+  QLORA_CUDA_TRY(cudaMemsetAsync(tickets, 0, 2 * sizeof(unsigned int), st));
+  int rc = launch_mean_tree(roots_all, n_roots_total, tree, tickets, n_blocks_total, mean, st);
+  if (rc != QLORA_OK || n_blocks_shard == 0) return rc;
+  return launch_dq(absmax, n_blocks_shard, mean, q8_shard, step2_shard, st);
 }
 
 int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,

@@ -388,6 +388,64 @@ int qlora_quantize_nf4_noalloc(const float* W, int64_t rows, int64_t cols,
                                uint8_t* codes, int8_t* q8, float* step2, float* mean,
                                void* stream);
 
+/*
+ * Sharded quantization -- qlora_quantize_nf4 split over `world` ranks that
+ * each hold a contiguous slice of the flattened weight (data parallelism over
+ * blocks; the pages quantize on one device, the split is this library's).
+ *
+ * The blocks (64 consecutive weights of the row-major weight) are grouped in
+ * chunks of 4096; rank k owns the chunks [k*cpr, (k+1)*cpr) with
+ * cpr = ceil(chunks / world), i.e. the blocks [block_begin, block_end), so
+ * every shard starts on a chunk boundary and hence on a 256-block boundary of
+ * the second-level groups.  The only quantity that needs every block is the
+ * scale mean.  Its tree (qlora_quantize_nf4: fp64, zero-padded to a power of
+ * two, adjacent pairs added level by level) is cut at the chunk level: each
+ * rank sums its own chunks (roots), the ranks all-gather the roots in rank
+ * order (world * cpr doubles, zeros for chunks past the weight), and every
+ * rank finishes the same tree over them.  Adding zero-padded power-of-two
+ * subtrees is exact, so codes, q8, step2 and mean are bit-identical to one
+ * qlora_quantize_nf4 call on the whole weight.
+ *
+ * qlora_quantize_shard_plan (host only): the block range of `rank` and cpr.
+ *   n_blocks_total = rows * cols / 64 of the whole weight (1 .. 2^34);
+ *   1 <= world, 0 <= rank < world.  A trailing rank may own no block.
+ *
+ * qlora_quantize_shard_workspace_size: bytes of the workspace one rank keeps
+ *   from its local call to its finishing call (n_roots_total = world * cpr);
+ *   (size_t)-1 for bad sizes.
+ *
+ * qlora_quantize_nf4_shard_local: the rank's codes and roots.
+ *   W_shard      device fp32, n_blocks_shard * 64 weights (the shard's slice
+ *                of the flattened weight), finite values.
+ *   codes_shard  device uint8 [n_blocks_shard * 32]             (written)
+ *   roots        device fp64 [roots_per_rank], 16-byte aligned  (written;
+ *                chunk sums of the shard's block absmaxes, zero past it)
+ *   The workspace must stay untouched until the finishing call.
+ *   n_blocks_shard = 0 (an empty rank) writes zero roots only.
+ *
+ * qlora_quantize_nf4_shard_finish: mean, and the rank's q8 and step2.
+ *   roots_all    device fp64 [n_roots_total], the all-gathered roots in rank order.
+ *   q8_shard     device int8 [n_blocks_shard]                    (written)
+ *   step2_shard  device fp32 [ceil(n_blocks_shard / 256)]        (written)
+ *   mean         device fp32 [1]                                 (written)
+ *   workspace    the same one the local call used.
+ *
+ * All device calls are asynchronous on `stream`; errors return before any
+ * launch (QLORA_ERR_INVALID_ARG for bad pointers or sizes, QLORA_ERR_WORKSPACE
+ * for a missing or short workspace).
+ */
+int qlora_quantize_shard_plan(int64_t n_blocks_total, int world, int rank,
+                              int64_t* block_begin, int64_t* block_end,
+                              int64_t* roots_per_rank);
+size_t qlora_quantize_shard_workspace_size(int64_t n_blocks_shard, int64_t n_roots_total);
+int qlora_quantize_nf4_shard_local(const float* W_shard, int64_t n_blocks_shard,
+                                   uint8_t* codes_shard, double* roots, int64_t roots_per_rank,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+int qlora_quantize_nf4_shard_finish(const double* roots_all, int64_t n_roots_total,
+                                    int64_t n_blocks_total, int64_t n_blocks_shard,
+                                    int8_t* q8_shard, float* step2_shard, float* mean,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* qlora_status_string -- static English description of a status code. */
 const char* qlora_status_string(int status);
 

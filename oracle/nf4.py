@@ -222,8 +222,19 @@ def double_quantize(c: np.ndarray):
     Returns (q8 int8[n_blocks], step2 fp64[n_groups] (fp32 values), mean).
     """
     c = np.asarray(c, dtype=np.float64)
-    n = c.size
     mean = scale_mean(c)
+    q8, step2 = second_level(c, mean)
+    return q8, step2, mean
+
+
+def second_level(c: np.ndarray, mean: float):
+    """q8 and step2 of the block scales c against a given per-tensor mean
+    (the part of reading R5 after the mean): per group of 256 blocks,
+    d = fl32(c - mean), step2 = fl32(max|d| / 127),
+    q8 = clip(rint(fl32(d * fl32(1/step2))), -127, 127), 0 where step2 = 0 or
+    the product is NaN.  Returns (q8 int8[n], step2 fp64[n_groups])."""
+    c = np.asarray(c, dtype=np.float64)
+    n = c.size
     d = fl32(c - mean)                                   # fl32(c_b - mean)
     n_groups = (n + DQ_GROUP - 1) // DQ_GROUP
     q8 = np.zeros(n, dtype=np.int8)
@@ -240,7 +251,7 @@ def double_quantize(c: np.ndarray):
             q = fl32(d[sl] * inv)
         q = np.where(np.isnan(q), 0.0, q)
         q8[sl] = np.clip(np.rint(q), -127, 127).astype(np.int8)
-    return q8, step2, mean
+    return q8, step2
 
 
 # --------------------------------------------------------------------------

@@ -108,6 +108,22 @@ def test_quantize_argument_errors(lib):
     assert f(FAKE, 64, 128, FAKE, FAKE, FAKE, FAKE, FAKE + 16, ws, None) == EWS       # misaligned ws
 
 
+def test_shard_quantize_argument_errors(lib):
+    loc, fin = lib.qlora_quantize_nf4_shard_local, lib.qlora_quantize_nf4_shard_finish
+    ws = q.quantize_shard_workspace_size(4096, 2)
+    assert lib.qlora_quantize_shard_workspace_size(-1, 2) == ctypes.c_size_t(-1).value
+    assert lib.qlora_quantize_shard_workspace_size(10, 0) == ctypes.c_size_t(-1).value
+    assert loc(FAKE, 4096, FAKE, None, 1, FAKE, ws, None) == EINVAL              # no roots
+    assert loc(FAKE, 4097, FAKE, FAKE, 1, FAKE, ws, None) == EINVAL              # shard larger than its chunks
+    assert loc(FAKE + 4, 4096, FAKE, FAKE, 1, FAKE, ws, None) == EINVAL          # misaligned W
+    assert loc(FAKE, 4096, FAKE, FAKE, 1, None, ws, None) == EWS                 # no workspace
+    assert loc(FAKE, 4096, FAKE, FAKE, 1, FAKE, 1024, None) == EWS               # absmaxes do not fit
+    assert fin(FAKE, 2, 8193, 4096, FAKE, FAKE, FAKE, FAKE, ws, None) == EINVAL  # more blocks than the roots cover
+    assert fin(FAKE, 2, 4096, 4097, FAKE, FAKE, FAKE, FAKE, ws, None) == EINVAL  # shard larger than the weight
+    assert fin(FAKE, 2, 8192, 4096, FAKE, FAKE, None, FAKE, ws, None) == EINVAL  # no mean
+    assert fin(FAKE, 2, 8192, 4096, FAKE, FAKE, FAKE, FAKE, ws - 1, None) == EWS
+
+
 def test_dequantize_argument_errors(lib):
     f = lib.qlora_dequantize_nf4
     assert f(None, FAKE, None) == EINVAL

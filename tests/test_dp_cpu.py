@@ -74,3 +74,92 @@ def test_two_rank_adapter_gradient_sum():
     want = np.concatenate([dA.reshape(-1), dB.reshape(-1)])
     # fp32 all-reduce of two fp32-rounded partial sums against the fp64 whole
     np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-6 * np.abs(want).max())
+
+
+# ---------------------------------------------------------------------------
+# sharded quantization: the host side (shard plan from the C library, the
+# all-gathers, padding and assembly) on gloo ranks, with the per-rank compute
+# done by the oracle; the assembled weight must equal the oracle's
+# quantization of the whole tensor, bit for bit.
+
+class _OracleShardLib:
+    """The per-rank calls of the sharded quantizer computed by the oracle (test only)."""
+
+    def quantize_shard_plan(self, n, world, rank):
+        import bit_nf4_quantized_11_b200 as q
+        return q.quantize_shard_plan(n, world, rank)
+
+    def quantize_nf4_shard_local(self, W_shard, cpr, n_roots_total):
+        from oracle import nf4
+        Wn = W_shard.numpy().astype(np.float32).astype(np.float64).reshape(-1, 64)
+        c = nf4.block_absmax(Wn) if Wn.size else np.zeros(0)
+        codes = nf4.pack(nf4.encode(Wn, c)).reshape(-1) if Wn.size else np.zeros(0, np.uint8)
+        roots = np.array([nf4.pairwise_sum(c[i * 4096:(i + 1) * 4096]) if i * 4096 < c.size else 0.0
+                          for i in range(cpr)])
+        return torch.from_numpy(codes.astype(np.uint8)), torch.from_numpy(roots), c
+
+    def quantize_nf4_shard_finish(self, roots_all, n_total, n_shard, ws):
+        from oracle import nf4
+        mean = float(nf4.fl32(nf4.pairwise_sum(roots_all.numpy()) / float(n_total)))
+        q8, step2 = nf4.second_level(ws, mean) if n_shard else (np.zeros(0, np.int8), np.zeros(0))
+        return (torch.from_numpy(q8), torch.from_numpy(step2.astype(np.float32)),
+                torch.tensor([mean], dtype=torch.float32))
+
+
+QROWS, QCOLS = 37, 8192          # 4736 blocks: one whole 4096-block chunk and a partial one
+
+
+def _quant_rank(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        W = synth.weight(QROWS, QCOLS, 0.02, "student_t5", 11).reshape(-1)
+        n_total = W.numel() // 64
+        lib = _OracleShardLib()
+        b0, b1, _ = lib.quantize_shard_plan(n_total, world, rank)
+        shard = dp.quantize_nf4_sharded(W[b0 * 64:b1 * 64].contiguous(), n_total, lib=lib)
+        codes, q8, step2, mean = dp.gather_nf4_replica(shard, n_total)
+        if rank == 0:
+            out.put((codes.numpy().copy(), q8.numpy().copy(), step2.numpy().copy(), float(mean[0])))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_quantize_assembles_the_whole_weight(world):
+    from oracle import nf4
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    procs = [ctx.Process(target=_quant_rank, args=(k, world, port, out)) for k in range(world)]
+    for p in procs:
+        p.start()
+    codes, q8, step2, mean = out.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    W = synth.weight(QROWS, QCOLS, 0.02, "student_t5", 11).numpy()
+    ref = nf4.quantize(W)
+    assert np.float32(mean).view(np.uint32) == nf4.f32_bits(ref["mean"])
+    assert np.array_equal(q8, ref["q8"])
+    assert np.array_equal(nf4.f32_bits(step2.astype(np.float64)), nf4.f32_bits(ref["step2"]))
+    assert np.array_equal(codes, ref["packed"].reshape(-1))
+
+
+def test_shard_plan_aligns_chunks_and_covers_blocks():
+    import bit_nf4_quantized_11_b200 as q
+    for n in (1, 4095, 4096, 4097, 4736, 704512, 3 * 4096 + 5):
+        for world in (1, 2, 3, 8):
+            spans = [q.quantize_shard_plan(n, world, k) for k in range(world)]
+            cpr = spans[0][2]
+            assert all(s[2] == cpr for s in spans) and world * cpr * 4096 >= n
+            assert spans[0][0] == 0 and spans[-1][1] == n
+            for (a0, a1, _), (c0, c1, _) in zip(spans, spans[1:]):
+                assert a1 == c0
+            for b0, b1, _ in spans:
+                assert (b0 == b1 == n or b0 % 4096 == 0) and b1 - b0 <= cpr * 4096   # empty trailing ranks sit at n
+    with pytest.raises(q.QLoRAError):
+        q.quantize_shard_plan(10, 2, 2)

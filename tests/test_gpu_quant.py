@@ -108,3 +108,59 @@ def test_dequantize_matches_codebook_levels_exactly(cuda_lib):
     qw = cuda_lib.quantize_nf4(torch.from_numpy(W).cuda())
     codes = nf4.unpack(qw.codes.cpu().numpy())
     assert np.array_equal(codes, np.tile(np.arange(16, dtype=np.uint8), 8).reshape(2, 64))
+
+
+def _sharded(q, W, world):
+    """Quantize W as `world` ranks would, the ranks run one after another on
+    this GPU (independent launches; the all-gather is a concatenation in rank
+    order), and assemble the whole weight."""
+    flat = W.reshape(-1)
+    n_total = flat.numel() // 64
+    locals_ = []
+    for k in range(world):
+        b0, b1, cpr = q.quantize_shard_plan(n_total, world, k)
+        codes, roots, ws = q.quantize_nf4_shard_local(flat[b0 * 64:b1 * 64], cpr, world * cpr)
+        locals_.append((b0, b1, codes, roots, ws))
+    roots_all = torch.cat([l[3] for l in locals_])
+    parts = [q.quantize_nf4_shard_finish(roots_all, n_total, b1 - b0, ws) for b0, b1, _, _, ws in locals_]
+    assert q.last_device_status() == 0
+    means = [p[2] for p in parts]
+    assert all(torch.equal(m, means[0]) for m in means)
+    return (torch.cat([l[2] for l in locals_]), torch.cat([p[0] for p in parts]),
+            torch.cat([p[1] for p in parts]), means[0])
+
+
+@pytest.mark.parametrize("rows,cols,dist,world", [
+    (37, 8192, "student_t5", 2),    # a whole 4096-block chunk and a partial one
+    (37, 8192, "normal", 3),        # the third rank holds no block
+    (300, 640, "normal", 4),        # one partial chunk: ranks 1..3 empty
+    (4096, 11008, "student_t5", 8), # 172 chunks, 22 per rank, the last rank short
+])
+def test_sharded_quantize_equals_single_call(cuda_lib, rows, cols, dist, world):
+    q = cuda_lib
+    W = synth.weight(rows, cols, 0.02, dist, 21).cuda()
+    codes, q8, step2, mean = _sharded(q, W, world)
+    w = q.quantize_nf4(W)
+    assert torch.equal(codes, w.codes.reshape(-1))
+    assert torch.equal(q8, w.q8)
+    assert torch.equal(step2.view(torch.int32), w.step2.view(torch.int32))
+    assert torch.equal(mean.view(torch.int32), w.mean.view(torch.int32))
+    if rows * cols <= 37 * 8192:
+        ref = nf4.quantize(W.cpu().numpy())
+        assert np.array_equal(codes.cpu().numpy(), ref["packed"].reshape(-1))
+        assert np.array_equal(q8.cpu().numpy(), ref["q8"])
+        assert np.array_equal(f32_bits(step2), nf4.f32_bits(ref["step2"]))
+        assert f32_bits(mean)[0] == nf4.f32_bits(ref["mean"])
+
+
+def test_sharded_quantize_extra_tree_pass(cuda_lib):
+    """8200 x 32768 over 2 ranks: 2 x 513 gathered chunk sums, more than one
+    finishing CTA takes, so the finishing call runs a second tree pass."""
+    q = cuda_lib
+    W = synth.weight(8200, 32768, 0.02, "normal", 5).cuda()
+    codes, q8, step2, mean = _sharded(q, W, 2)
+    w = q.quantize_nf4(W)
+    assert torch.equal(codes, w.codes.reshape(-1))
+    assert torch.equal(q8, w.q8)
+    assert torch.equal(step2.view(torch.int32), w.step2.view(torch.int32))
+    assert torch.equal(mean.view(torch.int32), w.mean.view(torch.int32))
