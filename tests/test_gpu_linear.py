@@ -83,6 +83,16 @@ def test_few_token_ragged(cuda_lib, M, n_in, n_out):
     _run(cuda_lib, M, n_in, n_out, 8, 16.0, seed=100 + M, backward=False)
 
 
+@pytest.mark.parametrize("M,n_in,n_out,alpha", [
+    (520, 512, 640, 16.0),    # CTA-pair GEMM: four 64-wide LoRA stages in the K loop
+    (100, 256, 320, 8.0),     # one-CTA GEMM
+    (5, 512, 384, 16.0),      # few-token GEMV forward, GEMM backward
+])
+def test_largest_rank(cuda_lib, M, n_in, n_out, alpha):
+    # r = 256, the largest rank the library takes
+    _run(cuda_lib, M, n_in, n_out, 256, alpha, seed=M + 7)
+
+
 @pytest.mark.parametrize("M,n_in,n_out", [(4096, 512, 2560), (4096, 2560, 512)])
 def test_two_waves_short_k(cuda_lib, M, n_in, n_out):
     # 80 output tiles of 512 x 256: more tiles than co-resident CTA pairs, so
