@@ -773,11 +773,13 @@ int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint
       w->rows * w->cols > (1ll << 40))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   const float s = alpha / static_cast<float>(r);
-  const int64_t units = (w->rows / qnf4::kMergeRows) * (w->cols / 8);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+  const int64_t tiles = (w->rows / qnf4::kMergeTileRows) * cdiv(w->cols, qnf4::kMergeTileCols);
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, device_sm_count() * 16)));
+  const int smem = qnf4::merge_smem_bytes(r);
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::merge_adapter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   {
     LaunchTimer lt_("merge_adapter", static_cast<cudaStream_t>(stream));
-    qnf4::merge_adapter_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    qnf4::merge_adapter_kernel<<<grid, 256, smem, static_cast<cudaStream_t>(stream)>>>(
         w->codes, w->q8, w->step2, w->mean, A, B, r, s, w->rows, w->cols, W_out, tables().L);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
