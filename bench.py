@@ -729,6 +729,16 @@ def components(q, dev, only=None):
 # ---------------------------------------------------------------------------- main
 def main():
     args = parse()
+    if args.impl == "reference":
+        # the oracle arm runs on the host cores of rank 0 only: no device, no process group
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        if world != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     world, rank, local = dist_setup(args)
     try:
         if args.only is not None:
@@ -737,11 +747,6 @@ def main():
             if rank == 0:
                 print(json.dumps({"only": args.only,
                                   "components": components(q, torch.device("cuda", local), args.only)}), flush=True)
-            return
-        if args.impl == "reference":
-            line = run_reference(args, world, rank)
-            if line is not None:
-                print(json.dumps(line), flush=True)
             return
         line = run_ours(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
