@@ -436,7 +436,7 @@ def selftest_wait_timeout() -> int:
 
 KERNEL_NAMES = ("quantize_blocks", "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
                 "gemv", "gemv_finalize", "lora_rowwise", "lora_rowwise_du", "lora_colwise",
-                "merge_adapter", "dropout_mask", "dropout_dx")
+                "merge_adapter", "dropout_dx")
 
 
 def timing_enable(on: bool = True) -> bool:

@@ -277,11 +277,7 @@ size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
   return M <= 16 ? gemv_ws(M, in, out) : 0;
 }
 
-size_t masked_x_bytes(int64_t M, int64_t in) { return round256(static_cast<size_t>(M) * in * 2); }
-
-size_t fwd_dropout_ws(int64_t M, int64_t in, int64_t out, int r) {
-  return masked_x_bytes(M, in) + fwd_ws(M, in, out, r);
-}
+size_t fwd_dropout_ws(int64_t M, int64_t in, int64_t out, int r) { return fwd_ws(M, in, out, r); }
 
 struct BwdWs {
   size_t du_off, total;
@@ -471,9 +467,9 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
 
 template <int NT, bool kKR>
 int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int ks, int64_t M, int64_t K, int R,
-                     float scale, cudaStream_t st) {
+                     float scale, cudaStream_t st, const uint8_t* keep) {
   using C = qnf4::RowCfg<NT, kKR>;
-  auto kern = qnf4::rowwise_skinny_kernel<NT, kKR>;
+  auto kern = keep != nullptr ? qnf4::rowwise_skinny_kernel<NT, kKR, true> : qnf4::rowwise_skinny_kernel<NT, kKR, false>;
   QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
   const int n_st = static_cast<int>(K / 64);
   const int sps = static_cast<int>(cdiv(n_st, ks));
@@ -491,32 +487,36 @@ int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int 
   cfg.numAttrs = ks > 1 ? 1 : 0;
   {
     LaunchTimer lt_(kKR ? "lora_rowwise_du" : "lora_rowwise", st);
-    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, act, W, out, static_cast<int>(M), static_cast<int>(K), R, scale, sps));
+    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, act, W, out, static_cast<int>(M), static_cast<int>(K), R, scale, sps,
+                                      keep));
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
 }
 
-// out[M, R] = bf16(scale * act[M, K] . W^T) with W given as [R, K] (kKR =
-// false) or as [K, R] (kKR = true).
+// out[M, R] = bf16(scale * (act[M, K] * k) . W^T) with W given as [R, K] (kKR =
+// false) or as [K, R] (kKR = true); k the keep mask of LoRA dropout, or all
+// ones when keep is null.
 template <bool kKR>
 int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_t M, int64_t K, int R, float scale,
-                   cudaStream_t st) {
+                   cudaStream_t st, const uint8_t* keep = nullptr) {
   const int ks = rowwise_splits(M, K, R);
-  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, ks, M, K, R, scale, st);
-  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, ks, M, K, R, scale, st);
-  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, ks, M, K, R, scale, st);
-  return launch_rowwise_t<8, kKR>(act, W, out, ks, M, K, R, scale, st);
+  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
+  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
+  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
+  return launch_rowwise_t<8, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
 }
 
 // dB = dh^T us -> [out, r] and dA = du^T x -> [r, in] in one launch: column
 // tiles x token chunks x the two problems, chunks of a tile in one cluster.
 int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
-                      int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st, float dA_scale = 1.f) {
-  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0, 1.f};
-  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale};
+                      int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st, float dA_scale = 1.f,
+                      const uint8_t* keep = nullptr) {
+  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0, 1.f, nullptr};
+  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale, keep};   // dA^T = (x * k)^T du
   const int smem = qnf4::kColStages * qnf4::kColStageBytes;
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::colwise_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  auto kern = keep != nullptr ? qnf4::colwise_skinny_kernel<true> : qnf4::colwise_skinny_kernel<false>;
+  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int chunk_tokens = col_chunk_tokens(M);
   const unsigned chunks = static_cast<unsigned>(cdiv(M, chunk_tokens));
   cudaLaunchConfig_t cfg{};
@@ -533,7 +533,7 @@ int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x,
   cfg.numAttrs = 1;
   {
     LaunchTimer lt_("lora_colwise", st);
-    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, qnf4::colwise_skinny_kernel, pb, pa, static_cast<int>(M), R, chunk_tokens));
+    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, pb, pa, static_cast<int>(M), R, chunk_tokens));
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;
@@ -555,14 +555,14 @@ int check_linear_shapes(int64_t M, const qlora_nf4_weight* w, int r) {
   return QLORA_OK;
 }
 
-// Forward after validation: us = bf16(s_lora * x_lora A^T) (x_lora = x, or
-// the masked x of LoRA dropout with s_lora = s / (1 - p)), then
+// Forward after validation: us = bf16(s_lora * (x * k) A^T) (k all ones, or
+// the keep mask of LoRA dropout with s_lora = s / (1 - p)), then
 // h = [x | us] [W0 | B]^T; `workspace` is the GEMV part (M <= 16).
-int linear_fwd_impl(const uint16_t* x, const uint16_t* x_lora, int64_t M, const qlora_nf4_weight* w,
+int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlora_nf4_weight* w,
                     const uint16_t* A, const uint16_t* B, int r, float s_lora, uint16_t* h, uint16_t* us_out,
                     void* workspace, cudaStream_t st) {
   const int64_t in = w->cols, out = w->rows;
-  int rc = launch_rowwise<false>(x_lora, A, us_out, M, in, r, s_lora, st);   // us = bf16(s x A^T)
+  int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s_lora, st, keep);   // us = bf16(s (x k) A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
@@ -614,21 +614,10 @@ int check_fwd_args(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, cons
 }
 
 int check_dropout_args(const uint8_t* keep_bits, float p) {
-  if (keep_bits == nullptr || !(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
+  if (keep_bits == nullptr || !aligned(keep_bits, 4) || !(p >= 0.f && p < 1.f)) return QLORA_ERR_INVALID_ARG;
   return QLORA_OK;
 }
 
-int launch_mask_apply(const uint16_t* x, const uint8_t* keep_bits, int64_t M, int64_t n, uint16_t* x_m,
-                      cudaStream_t st) {
-  const int64_t units = M * (n / 8);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
-  {
-    LaunchTimer lt_("dropout_mask", st);
-    qnf4::mask_apply_kernel<<<grid, 256, 0, st>>>(x, keep_bits, M, n, x_m);
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  return QLORA_OK;
-}
 
 }  // namespace
 
@@ -662,7 +651,7 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t in_features, int64_t out_
       return fwd_dropout_ws(M, in_features, out_features, r);
     case QLORA_OP_LINEAR_BWD_DROPOUT:
       if (M < 1 || r < 1) return 0;
-      return bwd_ws(M, in_features, out_features, r).total + masked_x_bytes(M, in_features);
+      return bwd_ws(M, in_features, out_features, r).total;
     default:
       return static_cast<size_t>(-1);
   }
@@ -837,7 +826,7 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   const size_t need = fwd_ws(M, w->cols, w->rows, r);
   if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
     return QLORA_ERR_WORKSPACE;
-  return linear_fwd_impl(x, x, M, w, A, B, r, alpha / static_cast<float>(r), h, us_out, workspace,
+  return linear_fwd_impl(x, nullptr, M, w, A, B, r, alpha / static_cast<float>(r), h, us_out, workspace,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -848,15 +837,12 @@ int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weigh
   if (sc != QLORA_OK) return sc;
   if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
   const int64_t in = w->cols;
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < fwd_dropout_ws(M, in, w->rows, r))
+  const size_t need = fwd_dropout_ws(M, in, w->rows, r);
+  if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
     return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint16_t* x_m = static_cast<uint16_t*>(workspace);
-  int rc = launch_mask_apply(x, keep_bits, M, in, x_m, st);                 // x_m = x * k
-  if (rc != QLORA_OK) return rc;
   const float s_lora = (alpha / static_cast<float>(r)) / (1.f - p);
-  return linear_fwd_impl(x, x_m, M, w, A, B, r, s_lora, h, us_out,
-                         static_cast<uint8_t*>(workspace) + masked_x_bytes(M, in), st);
+  return linear_fwd_impl(x, keep_bits, M, w, A, B, r, s_lora, h, us_out, workspace, st);
 }
 
 int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
@@ -898,18 +884,14 @@ int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16
   if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
   const int64_t in = w->cols, out = w->rows;
   const BwdWs ws = bwd_ws(M, in, out, r);
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total + masked_x_bytes(M, in))
-    return QLORA_ERR_WORKSPACE;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
-  uint16_t* x_m = reinterpret_cast<uint16_t*>(base + ws.total);
   const float s = alpha / static_cast<float>(r);
   const float inv_keep = 1.f / (1.f - p);
 
-  int rc = launch_mask_apply(x, keep_bits, M, in, x_m, st);                           // x_m = x * k
-  if (rc != QLORA_OK) return rc;
-  rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                              // du = bf16(s dh B)
+  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                          // du = bf16(s dh B)
   if (rc != QLORA_OK) return rc;
   rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);              // dx = dh W0
   if (rc != QLORA_OK) return rc;
@@ -920,7 +902,7 @@ int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16
     qnf4::dropout_dx_kernel<<<grid, 256, 0, st>>>(dx, du, A, keep_bits, M, in, r, inv_keep);  // + (du A) k/(1-p)
   }
   QLORA_CUDA_TRY(cudaGetLastError());
-  return launch_lora_grads(dh, us, x_m, du, M, in, out, r, dB, dA, st, inv_keep);   // dB, dA
+  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st, inv_keep, keep_bits);   // dB, dA
 }
 
 int qlora_last_device_status(void* stream) {

@@ -7,8 +7,9 @@
 // llm-compass 实现要点, skillbyai, learn-interview-questions section 3; the
 // placement on the adapter input is this library's reading).
 //
-// mask_apply_kernel    x_m = x * k (exact in bf16: kept or zero), read by the
-//                      rank-r kernels in place of x
+// The masked input x * k (exact in bf16: kept or zero) is never stored: the
+// rank-r kernels apply the keep bits to the activation tiles they stage
+// (skinny.cuh).
 // dropout_dx_kernel    dx = bf16(fp32(dx_base) + (k / (1 - p)) * sum_j du[m][j] A[j][i])
 //                      after the dx GEMM ran without its rank-r tail; the sum
 //                      is an in-order fp32 fused multiply-add chain
@@ -17,27 +18,6 @@
 #include "common.cuh"
 
 namespace qnf4 {
-
-// 8 columns per thread: one 16-byte activation load, one mask byte.
-__global__ void __launch_bounds__(256) mask_apply_kernel(
-    const uint16_t* __restrict__ x, const uint8_t* __restrict__ keep_bits, int64_t M, int64_t n,
-    uint16_t* __restrict__ x_m) {
-  const int64_t n8 = n / 8;
-  const int64_t units = M * n8;
-  for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
-       u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t kb = __ldg(keep_bits + u);                     // row m byte c of [M][n/8]
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(x + u * 8));
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const uint32_t lo = (kb >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
-      const uint32_t hi = (kb >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
-      w[e] &= lo | hi;
-    }
-    *reinterpret_cast<uint4*>(x_m + u * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
 
 constexpr int kDxRows = 4;
 

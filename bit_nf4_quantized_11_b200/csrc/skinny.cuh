@@ -58,6 +58,28 @@ __device__ __forceinline__ float4 cluster_sum_f4(uint32_t addr, int ranks) {
   return v;
 }
 
+// 4-byte asynchronous copy (a row's keep bits for 32 columns), zero-filled when invalid.
+__device__ __forceinline__ void cp_async_4(uint32_t smem_dst, const void* src, bool valid) {
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(smem_dst), "l"(src), "r"(n) : "memory");
+}
+
+// Zero the bf16 values of a 16-byte chunk (8 columns) whose keep bit is 0
+// (bit e of `bits` keeps column e): exact, a value is kept or becomes +0.
+__device__ __forceinline__ void mask_chunk(uint32_t addr, uint32_t bits) {
+  uint32_t w[4];
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr)
+               : "memory");
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t lo = (bits >> (2 * e)) & 1u ? 0x0000FFFFu : 0u;
+    const uint32_t hi = (bits >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u;
+    w[e] &= lo | hi;
+  }
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+               : "memory");
+}
+
 constexpr int kRowThreads = 128;
 constexpr int kRowStages = 4;
 constexpr int kRowActBytes = 64 * 128;                  // 64 rows x 64 k bf16
@@ -72,15 +94,17 @@ struct RowCfg {
   // W tile: [RCA rows x 64 k] (128 B rows, swizzled) or [64 k rows x RCA n] (padded rows)
   static constexpr int W_PITCH = kKR ? (RCA * 2 + ((RCA * 2 / 16) % 2 == 0 ? 16 : 0)) : 128;
   static constexpr int W_BYTES = kKR ? 64 * W_PITCH : RCA * 128;
-  static constexpr int STAGE = kRowActBytes + ((W_BYTES + 127) / 128) * 128;
+  static constexpr int MASK_BYTES = 64 * 8;            // keep bits of the 64 x 64 activation tile
+  static constexpr int STAGE = kRowActBytes + ((W_BYTES + 127) / 128) * 128 + MASK_BYTES;
   static constexpr int SMEM = kRowStages * STAGE;
   static_assert(64 * RC * 4 <= SMEM, "partial tile must fit the stage ring");
 };
 
-template <int NT, bool kKR>
+template <int NT, bool kKR, bool kMask>
 __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
     const uint16_t* __restrict__ act, const uint16_t* __restrict__ W,
-    uint16_t* __restrict__ out, int M, int K, int R, float scale, int stages_per_split) {
+    uint16_t* __restrict__ out, int M, int K, int R, float scale, int stages_per_split,
+    const uint8_t* __restrict__ keep) {
   using C = RowCfg<NT, kKR>;
   extern __shared__ __align__(128) uint8_t s_row[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -91,15 +115,30 @@ __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
   const int kst_end = min(K / 64, kst_begin + stages_per_split);
   const int n_st = kst_end - kst_begin;
 
+  // activation tile.  With a keep mask (LoRA dropout, kMask) thread t loads
+  // chunks 4 (t & 1) .. +3 of row t >> 1 and the matching 4 mask bytes;
+  // without, consecutive threads take consecutive chunks.
+  const int a_row = threadIdx.x >> 1, a_ch0 = 4 * (threadIdx.x & 1);
   auto stage = [&](int i) {
     uint8_t* sa = s_row + (i % kRowStages) * C::STAGE;
     uint8_t* sw = sa + kRowActBytes;
     const int k0 = (kst_begin + i) * 64;
-    for (int e = threadIdx.x; e < 64 * 8; e += kRowThreads) {       // activation 64 x 64
-      const int row = e >> 3, ch = e & 7;
-      const bool ok = m0 + row < M;
-      const uint16_t* src = act + static_cast<int64_t>(ok ? m0 + row : 0) * K + k0 + ch * 8;
-      cp_async_16(smem_u32(sa + row * 128 + ((ch ^ (row & 7)) << 4)), src, ok);
+    if (kMask) {
+      const bool ok = m0 + a_row < M;
+      const int64_t m = ok ? m0 + a_row : 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ch = a_ch0 + j;
+        cp_async_16(smem_u32(sa + a_row * 128 + ((ch ^ (a_row & 7)) << 4)), act + m * K + k0 + ch * 8, ok);
+      }
+      cp_async_4(smem_u32(sa + C::STAGE - C::MASK_BYTES + a_row * 8 + a_ch0), keep + (m * K + k0) / 8 + a_ch0, ok);
+    } else {
+      for (int e = threadIdx.x; e < 64 * 8; e += kRowThreads) {     // activation 64 x 64
+        const int row = e >> 3, ch = e & 7;
+        const bool ok = m0 + row < M;
+        const uint16_t* src = act + static_cast<int64_t>(ok ? m0 + row : 0) * K + k0 + ch * 8;
+        cp_async_16(smem_u32(sa + row * 128 + ((ch ^ (row & 7)) << 4)), src, ok);
+      }
     }
     if (!kKR) {
       for (int e = threadIdx.x; e < C::RCA * 8; e += kRowThreads) {  // W rows n, 64 k
@@ -129,6 +168,17 @@ __global__ void __launch_bounds__(kRowThreads) rowwise_skinny_kernel(
   }
   for (int i = 0; i < n_st; ++i) {
     cp_async_wait<kRowStages - 2>();
+    if (kMask) {                                                     // this thread's own chunks, now landed
+      const uint32_t sa = smem_u32(s_row + (i % kRowStages) * C::STAGE);
+      uint32_t bits;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(sa + C::STAGE - C::MASK_BYTES + a_row * 8 + a_ch0)
+                   : "memory");
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int ch = a_ch0 + j;
+        mask_chunk(sa + a_row * 128 + ((ch ^ (a_row & 7)) << 4), (bits >> (8 * j)) & 0xFFu);
+      }
+    }
     __syncthreads();
     if (i + kRowStages - 1 < n_st) stage(i + kRowStages - 1);
     cp_async_commit();
@@ -230,7 +280,8 @@ constexpr int kColThreads = 128;
 constexpr int kColStages = 4;
 constexpr int kActStride = 128 * 2 + 16;   // bytes per staged act row (17 x 16 B)
 constexpr int kUStride = 64 * 2 + 16;      // bytes per staged u row   (9 x 16 B)
-constexpr int kColStageBytes = 32 * kActStride + 32 * kUStride;
+constexpr int kColMaskBytes = 32 * 16;      // keep bits of the 32 x 128 activation tile
+constexpr int kColStageBytes = 32 * kActStride + 32 * kUStride + kColMaskBytes;
 static_assert(128 * 64 * 4 <= kColStages * kColStageBytes, "partial tile must fit the stage ring");
 
 struct ColProblem {
@@ -240,10 +291,12 @@ struct ColProblem {
   int P;
   int n_major;           // 1: output layout [n][p]
   float scale;           // applied to the reduced sum before it is stored
+  const uint8_t* keep;   // keep bits of act ([M][P/8], bit i % 8 of byte i / 8), or null
 };
 
-__global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem prob0, ColProblem prob1,
-                                                                     int M, int R, int chunk_tokens) {
+template <bool kMask>
+__global__ void __launch_bounds__(kColThreads, kMask ? 4 : 1) colwise_skinny_kernel(ColProblem prob0, ColProblem prob1,
+                                                                        int M, int R, int chunk_tokens) {
   extern __shared__ __align__(128) uint8_t s_col[];
   const ColProblem pr = blockIdx.z == 0 ? prob0 : prob1;
   const int P = pr.P;
@@ -265,16 +318,36 @@ __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem 
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.f;
 
+    // activation tile.  With keep masks (LoRA dropout, kMask) thread t loads
+    // chunks 4 (t & 3) .. +3 of row t >> 2 and the matching 4 mask bytes;
+    // without, consecutive threads take consecutive chunks.
+    const int a_row = threadIdx.x >> 2, a_pc0 = 4 * (threadIdx.x & 3);
     auto stage = [&](int st) {
       uint8_t* s_act = s_col + (st % kColStages) * kColStageBytes;
       uint8_t* s_u = s_act + 32 * kActStride;
       const int ms = mb + st * 32;
-      for (int e = threadIdx.x; e < 512; e += kColThreads) {      // 32 rows x 128 p
-        const int row = e >> 4, pc = e & 15;
-        const int m = ms + row, p = p0 + pc * 8;
-        const bool ok = (m < m_end) && (p < P);
-        const uint16_t* src = pr.act + static_cast<int64_t>(ok ? m : 0) * P + (ok ? p : 0);
-        cp_async_16(smem_u32(s_act + row * kActStride + pc * 16), src, ok);
+      if (!kMask) {
+        for (int e = threadIdx.x; e < 512; e += kColThreads) {    // 32 rows x 128 p
+          const int row = e >> 4, pc = e & 15;
+          const int m = ms + row, p = p0 + pc * 8;
+          const bool ok = (m < m_end) && (p < P);
+          const uint16_t* src = pr.act + static_cast<int64_t>(ok ? m : 0) * P + (ok ? p : 0);
+          cp_async_16(smem_u32(s_act + row * kActStride + pc * 16), src, ok);
+        }
+      } else {
+        const int m = ms + a_row;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int pc = a_pc0 + j, p = p0 + pc * 8;
+          const bool ok = (m < m_end) && (p < P);
+          const uint16_t* src = pr.act + static_cast<int64_t>(ok ? m : 0) * P + (ok ? p : 0);
+          cp_async_16(smem_u32(s_act + a_row * kActStride + pc * 16), src, ok);
+        }
+        if (pr.keep != nullptr) {
+          const bool ok = (m < m_end) && (p0 + a_pc0 * 8 < P);
+          const uint8_t* src = pr.keep + (static_cast<int64_t>(ok ? m : 0) * P + (ok ? p0 : 0)) / 8 + (ok ? a_pc0 : 0);
+          cp_async_4(smem_u32(s_act + kColStageBytes - kColMaskBytes + a_row * 16 + a_pc0), src, ok);
+        }
       }
       for (int e = threadIdx.x; e < 256; e += kColThreads) {      // 32 rows x 64 n
         const int row = e >> 3, nc = e & 7;
@@ -292,6 +365,14 @@ __global__ void __launch_bounds__(kColThreads) colwise_skinny_kernel(ColProblem 
     }
     for (int st = 0; st < n_steps; ++st) {
       cp_async_wait<kColStages - 2>();
+      if (kMask && pr.keep != nullptr) {                           // this thread's own chunks, now landed
+        const uint32_t sa = smem_u32(s_col + (st % kColStages) * kColStageBytes);
+        uint32_t bits;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits)
+                     : "r"(sa + kColStageBytes - kColMaskBytes + a_row * 16 + a_pc0) : "memory");
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mask_chunk(sa + a_row * kActStride + (a_pc0 + j) * 16, (bits >> (8 * j)) & 0xFFu);
+      }
       __syncthreads();
       if (st + kColStages - 1 < n_steps) stage(st + kColStages - 1);
       cp_async_commit();

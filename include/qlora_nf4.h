@@ -291,13 +291,17 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us,
  * qlora_linear_fwd / _bwd; dx adds the masked rank-r term to the bf16 result
  * of dh W0 in fp32 and rounds again to bf16.
  *
- * keep_bits  device uint8 [M, in/8]: bit (i % 8) of byte i/8 of row m is the
- *            keep flag of x[m][i] (the caller draws the mask).
+ * The masked input x * k is never stored: the rank-r kernels zero the
+ * dropped elements of the activation tiles they stage.
+ *
+ * keep_bits  device uint8 [M, in/8], 4-byte aligned: bit (i % 8) of byte i/8
+ *            of row m is the keep flag of x[m][i] (the caller draws the mask).
  * p          drop probability, 0 <= p < 1.
  * workspace: qlora_workspace_size(QLORA_OP_LINEAR_FWD_DROPOUT / _BWD_DROPOUT,
- *            M, in, out, r) bytes.  Other arguments, rules and returns as
+ *            M, in, out, r) bytes (the same as without dropout; none for the
+ *            forward with M > 16).  Other arguments, rules and returns as
  *            qlora_linear_fwd / qlora_linear_bwd; QLORA_ERR_INVALID_ARG for a
- *            null mask or p outside [0, 1).
+ *            null or misaligned mask or p outside [0, 1).
  */
 int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
                              const uint16_t* B, int r, float alpha, const uint8_t* keep_bits, float p, uint16_t* h,
@@ -342,7 +346,7 @@ int qlora_selftest_wait_timeout(void* stream);
  * the number of launches since the last reset.  Names: "quantize_blocks",
  * "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
  * "gemv", "gemv_finalize", "lora_rowwise" (us), "lora_rowwise_du" (du),
- * "lora_colwise" (dA and dB), "merge_adapter", "dropout_mask", "dropout_dx".  Events are created by the library on first use (host-side
+ * "lora_colwise" (dA and dB), "merge_adapter", "dropout_dx".  Events are created by the library on first use (host-side
  * CUDA objects, no device memory).  Not for use during stream capture.
  *
  * qlora_timing_enable: on != 0 enables, 0 disables; returns the previous state.
