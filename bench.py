@@ -59,6 +59,9 @@ def parse():
     return ap.parse_args()
 
 
+NOMINAL_BF16_TFLOPS = 2250.0      # dense bf16 tensor peak of one B200 (spec figure, for context)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -272,6 +275,7 @@ def run_ours(args, world, rank, local):
                 "timing": "mean CUDA-event duration of the kernel's launches in a second K-step region "
                           "identical to the timed one, events recorded on the launching stream",
                 "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                 "flops_per_launch": dom_flops,
                 "traffic": profiled_traffic(dom, WL.name)}
 
