@@ -763,7 +763,8 @@ int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   const float s = alpha / static_cast<float>(r);
   const int64_t tiles = (w->rows / qnf4::kMergeTileRows) * cdiv(w->cols, qnf4::kMergeTileCols);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, device_sm_count() * 16)));
+  // a few CTAs per SM slot: each walks a run of tiles, long enough to reuse its staged A
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, device_sm_count() * 8)));
   const int smem = qnf4::merge_smem_bytes(r);
   QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::merge_adapter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   {

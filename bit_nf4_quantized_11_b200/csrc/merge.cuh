@@ -13,7 +13,8 @@
 // weight against 2.5 bytes of traffic), so the kernel is organised around the
 // fp32 FMA pipe: a CTA of 256 threads takes a tile of 64 rows x 256 columns
 // and stages up to 64 rank indices of A (as fp32, [j][column]) and of B
-// (transposed, [j][row]) in shared memory.  Each thread accumulates an 8 x 8
+// (transposed, [j][row]) in shared memory; a CTA walks a column-major run of
+// tiles, so for r <= 64 it stages A once per column tile.  Each thread accumulates an 8 x 8
 // block in registers; a warp covers 32 rows x 64 columns, so per rank index
 // its lanes read 256 distinct bytes of A and 128 of B (the rest broadcast)
 // for 64 FMAs each, which keeps the shared-memory pipe well below the FMA
@@ -65,11 +66,18 @@ __global__ void __launch_bounds__(256, 2) merge_adapter_kernel(
   const int tr = 32 * (warp >> 2) + 8 * (lane >> 3);                 // first of this thread's 8 rows in the tile
   const int tc = 64 * (warp & 3) + 8 * (lane & 7);                   // first of its 8 columns
   const int64_t col_tiles = (cols + kMergeTileCols - 1) / kMergeTileCols;
-  const int64_t n_tiles = (rows / kMergeTileRows) * col_tiles;
+  const int64_t row_tiles = rows / kMergeTileRows;
+  const int64_t n_tiles = row_tiles * col_tiles;
+  // Tiles column-major, a contiguous run of them per CTA: consecutive tiles
+  // share their columns, so with r <= kMergeChunk the staged A is reused
+  // until the run moves to the next column tile.
+  const int64_t t_begin = static_cast<int64_t>(blockIdx.x) * n_tiles / gridDim.x;
+  const int64_t t_end = static_cast<int64_t>(blockIdx.x + 1) * n_tiles / gridDim.x;
+  int64_t staged_i0 = -1;                                            // columns whose A is in shared memory
 
-  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-    const int64_t o0 = (tile / col_tiles) * kMergeTileRows;
-    const int64_t i0 = (tile % col_tiles) * kMergeTileCols;
+  for (int64_t tile = t_begin; tile < t_end; ++tile) {
+    const int64_t o0 = (tile % row_tiles) * kMergeTileRows;
+    const int64_t i0 = (tile / row_tiles) * kMergeTileCols;
     const int64_t i = i0 + tc;
     const bool col_ok = i < cols;                                    // cols % 64 == 0: 8-column groups are whole
     float acc[8][8];
@@ -81,8 +89,11 @@ __global__ void __launch_bounds__(256, 2) merge_adapter_kernel(
     for (int j0 = 0; j0 < r; j0 += chunk) {
       const int jc = min(chunk, r - j0);
       __syncthreads();                                               // previous chunk (or tile) fully read
-      // A[j0 + jj][i0 .. i0 + 256) as fp32, zero past the last column
-      for (int e = threadIdx.x; e < jc * (kMergeTileCols / 8); e += 256) {
+      // A[j0 + jj][i0 .. i0 + 256) as fp32, zero past the last column (kept
+      // from the previous tile when it is the same single chunk)
+      const bool stage_a = !(r <= kMergeChunk && staged_i0 == i0);
+      staged_i0 = r <= kMergeChunk ? i0 : -1;
+      for (int e = threadIdx.x; stage_a && e < jc * (kMergeTileCols / 8); e += 256) {
         const int jj = e / (kMergeTileCols / 8), c8 = e % (kMergeTileCols / 8);
         const int64_t ia = i0 + 8 * c8;
         uint4 a = make_uint4(0, 0, 0, 0);
