@@ -237,6 +237,11 @@ int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* strea
  * ("QLoRA", llm-compass, 方法与公式, displayed formula).  The dequantized
  * weight is produced tile by tile inside the GEMM and never written to memory.
  * M > 16 runs the fused tensor-core GEMM; M <= 16 a split-K streaming GEMV.
+ * The GEMM's token tile is 512 rows on a CTA pair for M > 384, else 256 or
+ * 128 rows on one CTA; the environment variable QLORA_NF4_GEMM_TILE_M = 128,
+ * 256 or 512 (read once per process) forces one of them for every M > 16, so
+ * that each GEMM kernel can be exercised on any shape (results agree within
+ * fp32 summation order).  The backward's dx GEMM follows the same rule.
  *
  * x       device bf16 [M, in]
  * w       quantized W0, rows = out, cols = in
