@@ -163,3 +163,19 @@ def test_shard_plan_aligns_chunks_and_covers_blocks():
                 assert (b0 == b1 == n or b0 % 4096 == 0) and b1 - b0 <= cpr * 4096   # empty trailing ranks sit at n
     with pytest.raises(q.QLoRAError):
         q.quantize_shard_plan(10, 2, 2)
+
+
+def test_sharded_quantize_single_process_is_the_whole_weight():
+    """World of one (no process group): the plan gives rank 0 every block and
+    the gather returns the shard itself."""
+    from oracle import nf4
+    W = synth.weight(37, 8192, 0.02, "normal", 12).reshape(-1)
+    n_total = W.numel() // 64
+    shard = dp.quantize_nf4_sharded(W, n_total, lib=_OracleShardLib())
+    assert (shard.block_begin, shard.block_end) == (0, n_total)
+    codes, q8, step2, mean = dp.gather_nf4_replica(shard, n_total)
+    ref = nf4.quantize(W.numpy().reshape(37, 8192))
+    assert np.array_equal(codes.numpy(), ref["packed"].reshape(-1))
+    assert np.array_equal(q8.numpy(), ref["q8"])
+    assert np.array_equal(nf4.f32_bits(step2.numpy().astype(np.float64)), nf4.f32_bits(ref["step2"]))
+    assert np.float32(mean[0]).view(np.uint32) == nf4.f32_bits(ref["mean"])
