@@ -187,10 +187,47 @@ bool make_tmap_codes(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Per-device facts the launch planning needs on every call, looked up once
+// per device (a failed lookup, e.g. with no device, is not cached).
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) d = 0;
+  return d;
+}
+
 int device_sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  const int c = cache[dev].load(std::memory_order_relaxed);
+  if (c > 0) return c;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 148;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// The dynamic shared-memory limit of a kernel, raised to at least `bytes`
+// on the current device.  The attribute persists for the process, so the
+// largest value set so far is remembered per kernel and device and only a
+// larger request calls cudaFuncSetAttribute again (a launch may use any
+// size up to the limit).
+cudaError_t set_max_smem(const void* kern, int bytes) {
+  struct Entry { const void* kern; int dev; int bytes; };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lk(mu);
+  Entry* e = nullptr;
+  for (Entry& x : done)
+    if (x.kern == kern && x.dev == dev) e = &x;
+  if (e != nullptr && e->bytes >= bytes) return cudaSuccess;
+  const cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err != cudaSuccess) return err;
+  if (e != nullptr) e->bytes = bytes;
+  else done.push_back(Entry{kern, dev, bytes});
+  return cudaSuccess;
 }
 
 // ------------------------------------------------------------------ workspace
@@ -223,13 +260,18 @@ struct GemvPlan {
 };
 
 int gemv_ctas_per_sm() {
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  const int c = cache[dev].load(std::memory_order_relaxed);
+  if (c > 0) return c;
   int n = 0;
-  cudaFuncSetAttribute(qnf4::nf4_gemv_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       qnf4::kGvSmem);
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel<true, true>, qnf4::kGvThreads,
+  const void* kern = reinterpret_cast<const void*>(qnf4::nf4_gemv_kernel<true, true>);
+  if (set_max_smem(kern, qnf4::kGvSmem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel<true, true>, qnf4::kGvThreads,
                                                     qnf4::kGvSmem) != cudaSuccess ||
       n < 1)
-    n = 1;
+    return 1;
+  cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -408,7 +450,7 @@ int launch_gemm_t(const qnf4::GemmArgs& args, const CUtensorMap& tm_act, const C
                   cudaStream_t st) {
   using Cfg = qnf4::GemmCfg<MS, kStages>;
   auto kern = qnf4::qlora_gemm_kernel<MS, kDx, kStages>;
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), Cfg::SMEM));
   const int64_t tiles = cdiv(args.M, Cfg::BM) * cdiv(args.N, Cfg::BN);
   {
     LaunchTimer lt_(kDx ? "gemm_dx" : "gemm_fwd", st);
@@ -423,7 +465,7 @@ int launch_gemm_pair(const qnf4::GemmArgs& args, const CUtensorMap& tm_act, cons
                      cudaStream_t st) {
   using Cfg = qnf4::PairCfg;
   auto kern = qnf4::qlora_gemm_pair_kernel<kDx>;
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM));
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), Cfg::SMEM));
   const int64_t pairs = cdiv(args.M, Cfg::BM) * cdiv(args.N, Cfg::BN);
   {
     LaunchTimer lt_(kDx ? "gemm_dx" : "gemm_fwd", st);
@@ -470,7 +512,7 @@ int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int 
                      float scale, cudaStream_t st, const uint8_t* keep) {
   using C = qnf4::RowCfg<NT, kKR>;
   auto kern = keep != nullptr ? qnf4::rowwise_skinny_kernel<NT, kKR, true> : qnf4::rowwise_skinny_kernel<NT, kKR, false>;
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), C::SMEM));
   const int n_st = static_cast<int>(K / 64);
   const int sps = static_cast<int>(cdiv(n_st, ks));
   cudaLaunchConfig_t cfg{};
@@ -516,7 +558,7 @@ int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x,
   const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale, keep};   // dA^T = (x * k)^T du
   const int smem = qnf4::kColStages * qnf4::kColStageBytes;
   auto kern = keep != nullptr ? qnf4::colwise_skinny_kernel<true> : qnf4::colwise_skinny_kernel<false>;
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), smem));
   const int chunk_tokens = col_chunk_tokens(M);
   const unsigned chunks = static_cast<unsigned>(cdiv(M, chunk_tokens));
   cudaLaunchConfig_t cfg{};
@@ -588,7 +630,7 @@ int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlo
       const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
       auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
                          : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
-      QLORA_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, qnf4::kGvSmem));
+      QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), qnf4::kGvSmem));
       kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
@@ -766,7 +808,7 @@ int qlora_merge_adapter(const qlora_nf4_weight* w, const uint16_t* A, const uint
   // a few CTAs per SM slot: each walks a run of tiles, long enough to reuse its staged A
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(tiles, device_sm_count() * 8)));
   const int smem = qnf4::merge_smem_bytes(r);
-  QLORA_CUDA_TRY(cudaFuncSetAttribute(qnf4::merge_adapter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(qnf4::merge_adapter_kernel), smem));
   {
     LaunchTimer lt_("merge_adapter", static_cast<cudaStream_t>(stream));
     qnf4::merge_adapter_kernel<<<grid, 256, smem, static_cast<cudaStream_t>(stream)>>>(
@@ -989,7 +1031,6 @@ constexpr size_t kNoAllocScratchBytes =
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
