@@ -433,7 +433,11 @@ int qlora_quantize_nf4_noalloc(const float* W, int64_t rows, int64_t cols,
  *   n_blocks_shard = 0 (an empty rank) writes zero roots only.
  *
  * qlora_quantize_nf4_shard_finish: mean, and the rank's q8 and step2.
- *   roots_all    device fp64 [n_roots_total], the all-gathered roots in rank order.
+ *   roots_all    device fp64 [n_roots_total], 16-byte aligned: the all-gathered
+ *                roots in rank order.
+ *   q8_shard, step2_shard, mean: 16-byte aligned (slices of a whole weight's
+ *                arrays at the shard's first block are, since shards start on
+ *                4096-block boundaries).
  *   q8_shard     device int8 [n_blocks_shard]                    (written)
  *   step2_shard  device fp32 [ceil(n_blocks_shard / 256)]        (written)
  *   mean         device fp32 [1]                                 (written)
