@@ -157,6 +157,25 @@ def test_linear_argument_errors(lib):
     assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 9, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ESHAPE
 
 
+def test_dropout_argument_errors(lib):
+    fwd, bwd = lib.qlora_linear_fwd_dropout, lib.qlora_linear_bwd_dropout
+    w = _weight(128, 128)
+    wb = ctypes.byref(w)
+    # keep mask: null or not 4-byte aligned, p outside [0, 1)
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, None, 0.05, FAKE, FAKE, None, 0, None) == EINVAL
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE + 2, 0.05, FAKE, FAKE, None, 0, None) == EINVAL
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, 1.0, FAKE, FAKE, None, 0, None) == EINVAL
+    assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, -0.1, FAKE, FAKE, None, 0, None) == EINVAL
+    # the few-token forward needs a workspace; the large-M one none (the mask is applied in place of a copy)
+    assert fwd(FAKE, 4, wb, FAKE, FAKE, 8, 16.0, FAKE, 0.05, FAKE, FAKE, None, 0, None) == EWS
+    assert q.workspace_size(q.OP_LINEAR_FWD_DROPOUT, 64, 128, 128, 8) == 0
+    assert q.workspace_size(q.OP_LINEAR_BWD_DROPOUT, 64, 128, 128, 8) == q.workspace_size(q.OP_LINEAR_BWD, 64, 128,
+                                                                                           128, 8)
+    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE + 1, 0.05, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+               None) == EINVAL
+    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, 0.05, FAKE, FAKE, FAKE, None, 0, None) == EWS
+
+
 def test_timeout_setter_roundtrip(lib):
     prev = q.set_wait_timeout_ns(5_000_000)
     assert q.set_wait_timeout_ns(prev) == 5_000_000
