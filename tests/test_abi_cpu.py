@@ -176,6 +176,20 @@ def test_dropout_argument_errors(lib):
     assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, 0.05, FAKE, FAKE, FAKE, None, 0, None) == EWS
 
 
+def test_merge_argument_errors(lib):
+    f = lib.qlora_merge_adapter
+    w = _weight(128, 128)
+    wb = ctypes.byref(w)
+    assert f(None, FAKE, FAKE, 8, 16.0, FAKE, None) == EINVAL
+    assert f(wb, None, FAKE, 8, 16.0, FAKE, None) == EINVAL
+    assert f(wb, FAKE, FAKE, 8, 16.0, FAKE + 8, None) == EINVAL          # misaligned output
+    assert f(wb, FAKE, FAKE, 8, float("inf"), FAKE, None) == EINVAL
+    for r in (0, 257):
+        assert f(wb, FAKE, FAKE, r, 16.0, FAKE, None) == ESHAPE
+    w2 = _weight(96, 128)
+    assert f(ctypes.byref(w2), FAKE, FAKE, 8, 16.0, FAKE, None) == ESHAPE
+
+
 def test_timeout_setter_roundtrip(lib):
     prev = q.set_wait_timeout_ns(5_000_000)
     assert q.set_wait_timeout_ns(prev) == 5_000_000
