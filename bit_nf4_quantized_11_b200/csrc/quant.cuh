@@ -115,12 +115,16 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_blocks_kernel(
       const float r = __frcp_rn(m);
       uint32_t packed[4];
       if (m > 0.f && isinf(r)) {
-        // absmax so small that 1/absmax overflows: v = w * inf is +inf (code
-        // 15), -inf (code 0), or NaN for a zero weight (the zero level, 7)
-        auto sat = [](float x) -> uint32_t { return x > 0.f ? 15u : (x < 0.f ? 0u : 7u); };
+        // absmax so small (subnormal) that 1/absmax overflows: normalise by
+        // one correctly rounded division instead (rare, block-uniform path)
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          packed[k] = sat(w[rd][k].x) | (sat(w[rd][k].y) << 4) | (sat(w[rd][k].z) << 8) | (sat(w[rd][k].w) << 12);
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t c0 = nearest_code(__fdiv_rn(w[rd][k].x, m), tab_lane);
+          const uint32_t c1 = nearest_code(__fdiv_rn(w[rd][k].y, m), tab_lane);
+          const uint32_t c2 = nearest_code(__fdiv_rn(w[rd][k].z, m), tab_lane);
+          const uint32_t c3 = nearest_code(__fdiv_rn(w[rd][k].w, m), tab_lane);
+          packed[k] = c0 | (c1 << 4) | (c2 << 8) | (c3 << 12);
+        }
       } else if (m > 0.f) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -215,8 +219,8 @@ __global__ void __launch_bounds__(256) pairwise_tree_kernel(
 // ---------------------------------------------------------------------------
 // K3: second-level codes.  One warp per group of 256 block scales:
 // d = fp32(c - mean), step2 = fp32(max|d| / 127),
-// q8 = clamp(rne(fp32(d * fp32(1/step2))), -127, 127); 0 when step2 == 0 or
-// the product is NaN.
+// q8 = clamp(rne(fp32(d * fp32(1/step2))), -127, 127), with fp32(d / step2)
+// in place of the product when fp32(1/step2) overflows; 0 when step2 == 0.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) dq_scales_kernel(
     const float* __restrict__ absmax, int64_t n_blocks, const float* __restrict__ mean_ptr,
@@ -246,13 +250,14 @@ __global__ void __launch_bounds__(256) dq_scales_kernel(
   const float st = __fdiv_rn(S, 127.0f);
   if (lane == 0) step2[g] = st;
   const float inv = (st != 0.f) ? __frcp_rn(st) : 0.f;
+  const bool by_div = isinf(inv);                  // subnormal step: divide instead (warp-uniform)
   uint32_t packed[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     int q = 0;
     if (st != 0.f) {
-      const float p = __fmul_rn(d[i], inv);
-      if (p == p) q = min(127, max(-127, __float2int_rn(p)));
+      const float p = by_div ? __fdiv_rn(d[i], st) : __fmul_rn(d[i], inv);
+      q = min(127, max(-127, __float2int_rn(p)));
     }
     packed[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
   }

@@ -124,15 +124,16 @@ size_t qlora_workspace_size(int op, int64_t M, int64_t in_features,
  * qlora_quantize_nf4 -- blockwise NF4 quantization with double quantization.
  *
  * Per block b of 64 weights: c_b = max|w| (exact); if c_b = 0 every code is 7;
- * otherwise v = fp32(w * fp32(1/c_b)) and code = #{j : v > thresholds[j]},
- * except that a NaN v (a zero weight in a block whose 1/c_b overflows to
- * infinity) is code 7.
+ * otherwise v = fp32(w * fp32(1/c_b)), or v = fp32(w / c_b) for a block whose
+ * fp32(1/c_b) overflows (a subnormal c_b below ~2.9e-39), and
+ * code = #{j : v > thresholds[j]}, the nearest level with ties to the lower.
  * Second level: mean = fp32(T / n_blocks) where T is the fp64 sum of all c_b
  * in a fixed binary tree (zero-padded to a power of two, adjacent pairs added
  * level by level) and the division is done in fp64; d_b = fp32(c_b - mean);
  * per group g of 256 blocks step2_g = fp32(max|d_b| / 127);
- * q8_b = clamp(round_half_even(fp32(d_b * fp32(1/step2_g))), -127, 127), or 0
- * when step2_g = 0 or the product is NaN.  All fp32 operations are correctly
+ * q8_b = clamp(round_half_even(fp32(d_b * fp32(1/step2_g))), -127, 127), with
+ * fp32(d_b / step2_g) in place of the product when fp32(1/step2_g) overflows,
+ * or 0 when step2_g = 0.  All fp32 operations are correctly
  * rounded (no fused multiply-add), so the result is bit-reproducible.
  * ("QLoRA", llm-compass, 方法与公式 items 1-2.)
  *

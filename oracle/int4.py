@@ -24,7 +24,7 @@ from __future__ import annotations
 import numpy as np
 
 from .nf4 import (BLOCK, ZERO_INDEX, bf16_bits_from_f32, block_absmax, dequant_scales, double_quantize, fl32,
-                  pack)
+                  normalise, pack)
 
 
 def levels() -> np.ndarray:
@@ -52,12 +52,7 @@ def encode(W: np.ndarray, c: np.ndarray) -> np.ndarray:
     blocks = W.reshape(-1, BLOCK)
     codes = np.full(blocks.shape, ZERO_INDEX, dtype=np.uint8)
     nz = c > 0
-    with np.errstate(over="ignore", invalid="ignore"):
-        recip = fl32(1.0 / c[nz])
-        v = fl32(blocks[nz] * recip[:, None])
-    enc = nearest_level(v)
-    enc[np.isnan(v)] = ZERO_INDEX
-    codes[nz] = enc
+    codes[nz] = nearest_level(normalise(blocks[nz], c[nz]))
     return codes.reshape(rows, cols)
 
 

@@ -29,18 +29,19 @@ R2 Nearest level, ties to the lower index; implemented as a comparison with the
    exact fp64 midpoints of consecutive fp32 levels.
 R3 Normalisation ``v = fl32(w * fl32(1/c))`` (reciprocal then multiply) rather
    than a division; an all-zero block (c = 0) encodes every weight as the zero
-   level (index 7).  When 1/c overflows fp32 (c below ~2.9e-39), v is +inf or
-   -inf (codes 15 and 0 by the count rule) and a zero weight gives NaN, which
-   is encoded as the zero level (7): a zero weight always maps to the exact
-   zero level.
+   level (index 7).  When 1/c overflows fp32 (c below ~2.9e-39, a subnormal
+   absmax), the reciprocal is unusable and ``v = fl32(w / c)`` (one correctly
+   rounded division) is taken instead, so such a block still gets the nearest
+   level of every weight and a zero weight the zero level.
 R4 Packing: element 2i of a row goes to the low nibble of byte i, 2i+1 to the
    high nibble; blocks are 64 consecutive weights in row-major order.
 R5 Double quantization: one fp32 mean per tensor (pairwise fp64 sum of all
    block scales, zero-padded to a power of two, divided by the block count,
    rounded to fp32); per group of 256 consecutive blocks a linear symmetric
-   int8 code with ``step2 = fl32(max|c - mean| / 127)`` and round-half-even;
-   a zero step gives code 0; a NaN product (0 * inf) gives code 0.  The
-   first-level codes always use the exact block absmax.
+   int8 code with ``step2 = fl32(max|c - mean| / 127)`` and round-half-even of
+   ``fl32(d * fl32(1/step2))``, or of ``fl32(d / step2)`` when that reciprocal
+   overflows (as in R3); a zero step gives code 0.  The first-level codes
+   always use the exact block absmax.
 R6 Dequantization: ``c_hat = fl32(fl32(q8 * step2) + mean)`` and
    ``w_hat = bf16_rne(fl32(level[code] * c_hat))``.
 R7 16-bit input: weights loaded in bf16 (as a 16-bit checkpoint is loaded
@@ -161,6 +162,20 @@ def nearest_level(v: np.ndarray) -> np.ndarray:
                            side="left").astype(np.uint8)
 
 
+def normalise(blocks: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """Normalised values v of the weights of blocks with a nonzero absmax c
+    (one row of ``blocks`` per block, reading R3): ``fl32(w * fl32(1/c))``,
+    or ``fl32(w / c)`` for a block whose fp32 reciprocal overflows."""
+    c = np.asarray(c, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        recip = fl32(1.0 / c)                       # fl32(1 / c_b), inf for tiny c_b
+    v = fl32(blocks * recip[:, None])               # fl32(w * r_b)
+    over = ~np.isfinite(recip)
+    if over.any():
+        v[over] = fl32(blocks[over] / c[over, None])   # fl32(w / c_b)
+    return v
+
+
 def encode(W: np.ndarray, c: np.ndarray) -> np.ndarray:
     """4-bit code of every weight (unpacked, shape of W), given the exact block
     absmax c (reading R3)."""
@@ -169,12 +184,7 @@ def encode(W: np.ndarray, c: np.ndarray) -> np.ndarray:
     blocks = W.reshape(-1, BLOCK)
     codes = np.full(blocks.shape, ZERO_INDEX, dtype=np.uint8)
     nz = c > 0
-    with np.errstate(over="ignore", invalid="ignore"):
-        recip = fl32(1.0 / c[nz])                   # fl32(1 / c_b), inf for tiny c_b
-        v = fl32(blocks[nz] * recip[:, None])       # fl32(w * r_b)
-    enc = nearest_level(v)
-    enc[np.isnan(v)] = ZERO_INDEX                   # 0 * inf: a zero weight
-    codes[nz] = enc
+    codes[nz] = nearest_level(normalise(blocks[nz], c[nz]))
     return codes.reshape(rows, cols)
 
 
@@ -231,8 +241,9 @@ def second_level(c: np.ndarray, mean: float):
     """q8 and step2 of the block scales c against a given per-tensor mean
     (the part of reading R5 after the mean): per group of 256 blocks,
     d = fl32(c - mean), step2 = fl32(max|d| / 127),
-    q8 = clip(rint(fl32(d * fl32(1/step2))), -127, 127), 0 where step2 = 0 or
-    the product is NaN.  Returns (q8 int8[n], step2 fp64[n_groups])."""
+    q8 = clip(rint(fl32(d * fl32(1/step2))), -127, 127), with fl32(d / step2)
+    in place of the product when fl32(1/step2) overflows, and 0 where
+    step2 = 0.  Returns (q8 int8[n], step2 fp64[n_groups])."""
     c = np.asarray(c, dtype=np.float64)
     n = c.size
     d = fl32(c - mean)                                   # fl32(c_b - mean)
@@ -246,10 +257,9 @@ def second_level(c: np.ndarray, mean: float):
         step2[g] = st
         if st == 0.0:
             continue                                     # all codes 0
-        with np.errstate(invalid="ignore", over="ignore"):
-            inv = float(fl32(1.0 / st))                  # fl32(1 / step2), may be inf
-            q = fl32(d[sl] * inv)
-        q = np.where(np.isnan(q), 0.0, q)
+        with np.errstate(over="ignore"):
+            inv = float(fl32(1.0 / st))                  # fl32(1 / step2)
+        q = fl32(d[sl] * inv) if np.isfinite(inv) else fl32(d[sl] / st)
         q8[sl] = np.clip(np.rint(q), -127, 127).astype(np.int8)
     return q8, step2
 

@@ -64,6 +64,19 @@ def test_degenerate_blocks_bit_exact(cuda_lib):
     assert np.all(codes[0, :32] == 0x77) and np.all(codes[1] == 0x77)
 
 
+def test_subnormal_tensor_divides_at_both_levels(cuda_lib):
+    """Weights ~1e-39: most blocks' absmax reciprocals overflow (first-level
+    division path) and every group's step is subnormal, so the second-level
+    codes take the division path too."""
+    W = (synth.weight(64, 1024, 1.0, "normal", 8).numpy() * np.float32(1e-39)).astype(np.float32)
+    c = nf4.block_absmax(W)
+    _, step2, _ = nf4.double_quantize(c)
+    with np.errstate(over="ignore", divide="ignore"):
+        assert np.any(~np.isfinite(np.float32(1.0) / c.astype(np.float32)))
+        assert np.all(~np.isfinite(np.float32(1.0) / step2.astype(np.float32)))
+    _check_quant(cuda_lib, torch.from_numpy(W))
+
+
 def test_equal_absmax_gives_zero_second_level(cuda_lib):
     rng = np.random.default_rng(3)
     W = rng.uniform(-0.5, 0.5, (16, 1024)).astype(np.float32)

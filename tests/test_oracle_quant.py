@@ -147,12 +147,78 @@ def test_second_level_codes_use_full_int8_range():
 
 
 def test_partial_last_group():
-    rng = np.random.default_rng(6)
-    W = (rng.standard_normal((5, 64 * 61)) * 0.02).astype(np.float32)  # 305 blocks
+    """305 blocks with absmax 1, 2, ..., 305 (a partial second group of 49),
+    worked by hand: mean = 46665 / 305 = 153, d_b = b + 1 - 153 ranges over
+    -152..103 in group 0 and 104..152 in group 1, so both steps are
+    fl32(152/127); q8 is +-127 at the ends, 0 at d = 0, and within half a
+    step (plus the fp32 roundings) of d * 127 / 152 everywhere."""
+    c = np.arange(1, 306, dtype=np.float64)
+    W = np.zeros((5, 64 * 61), dtype=np.float32)
+    W.reshape(-1, 64)[:, 17] = c                    # one weight per block sets its absmax
     q = nf4.quantize(W)
+    assert np.array_equal(q["absmax"], c)
+    assert q["mean"] == 153.0
     assert q["step2"].shape == (2,) and q["q8"].shape == (305,)
-    d_last = nf4.fl32(q["absmax"][256:] - q["mean"])
-    assert q["step2"][1] == nf4.fl32(np.abs(d_last).max() / 127.0)
+    assert np.all(q["step2"] == float(np.float32(152.0 / 127.0)))
+    assert q["q8"][0] == -127 and q["q8"][304] == 127 and q["q8"][152] == 0
+    exact = (c - 153.0) * 127.0 / 152.0
+    assert np.all(np.abs(q["q8"] - exact) <= 0.5 + 1e-4)
+
+
+def _mean_fixtures():
+    with open(os.path.join(GOLDEN, "scale_mean.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, spec = (t.strip() for t in line.split(";"))
+            tok = spec.split()
+            if tok[0] == "range":
+                vals = np.arange(int(tok[1]), int(tok[2]) + 1, dtype=np.float64)
+            elif tok[0] == "rep":
+                vals = np.full(int(tok[1]), float(tok[2]))
+            else:
+                vals = np.array([float(t) for t in tok])
+            yield int(bits, 16), vals
+
+
+def _mean_mismatches(mean_fn):
+    return [(hex(b), v.size) for b, v in _mean_fixtures()
+            if int(np.array([mean_fn(v)], dtype=np.float32).view(np.uint32)[0]) != b]
+
+
+def test_scale_mean_fixtures():
+    """Hand-worked means of block counts that are not powers of two."""
+    assert _mean_mismatches(nf4.scale_mean) == []
+
+
+def test_scale_mean_fixtures_through_quantize():
+    for bits, vals in _mean_fixtures():
+        W = np.zeros((1, 64 * vals.size), dtype=np.float32)
+        W.reshape(-1, 64)[:, 5] = vals
+        q = nf4.quantize(W)
+        assert int(np.array([q["mean"]], dtype=np.float32).view(np.uint32)[0]) == bits
+
+
+def test_scale_mean_fixtures_reject_wrong_divisors():
+    """The fixtures catch a mean divided by the zero-padded tree length, by
+    the number of 256-block groups, or rounded to fp32 before the division."""
+    def padded(c):
+        n = 1
+        while n < len(c):
+            n *= 2
+        return float(nf4.fl32(nf4.pairwise_sum(c) / n))
+
+    def per_group(c):
+        return float(nf4.fl32(nf4.pairwise_sum(c) / ((len(c) + 255) // 256)))
+
+    def fp32_sum(c):
+        return float(nf4.fl32(float(nf4.fl32(nf4.pairwise_sum(c))) / len(c)))
+
+    assert len(_mean_mismatches(padded)) == 5
+    assert len(_mean_mismatches(per_group)) == 5
+    assert len(_mean_mismatches(fp32_sum)) == 0      # all fixture sums are exact in fp32
+    assert len(_mean_mismatches(lambda c: float(np.mean(c)))) == 0
 
 
 def test_pairwise_tree_fixtures():
@@ -246,13 +312,36 @@ def test_quantize_rows_equals_full_quantize_rows():
 
 
 def test_reciprocal_overflow_block():
-    """Absmax below ~2.9e-39: 1/c overflows to inf; nonzero weights saturate to
-    the extreme levels by sign and zero weights stay at the zero level."""
+    """Absmax below ~2.9e-39: fl32(1/c) overflows, so every weight of the
+    block is normalised by one correctly rounded division and gets its
+    nearest level (brute force in exact rationals); zero weights stay at the
+    zero level."""
+    tiny = np.float32(2.0 ** -149)                  # smallest subnormal
     W = np.zeros((1, 64), dtype=np.float32)
-    W[0, :4] = [2e-39, -2e-39, 0.0, -0.0]
-    W[0, 4] = 1e-39
+    W[0, :8] = [2e-39, -2e-39, 0.0, -0.0, 1e-39, 3 * tiny, -5 * tiny, 1.3e-39]
+    W[0, 8] = np.float32(1.9e-39)
     q = nf4.quantize(W)
-    assert q["absmax"][0] == np.float32(2e-39)
-    assert list(q["codes"][0, :5]) == [15, 0, 7, 7, 15]
-    assert np.all(q["codes"][0, 5:] == 7)
+    c = np.float32(2e-39)
+    assert q["absmax"][0] == c
+    assert not np.isfinite(np.float32(1.0) / c)     # the reciprocal really overflows
+    levels = nf4.codebook()
+    for k in range(64):
+        quotient = Fraction(float(W[0, k])) / Fraction(float(c))
+        v = float(np.float32(float(quotient)))      # the correctly rounded fp32 quotient
+        assert q["codes"][0, k] == brute_nearest(v, levels), k
+    assert list(q["codes"][0, :5]) == [15, 0, 7, 7, 12]   # 1e-39 / 2e-39 = 0.5 -> level 12
 
+
+def test_second_level_reciprocal_overflow():
+    """A group whose step's fp32 reciprocal overflows (max |c - mean| below
+    ~3.7e-37) is coded by division: q8 = rint(fl32(d / step2)), checked in
+    exact rationals, instead of saturating every nonzero d to +-127."""
+    mu = float(np.float32(3e-38))
+    scales = nf4.fl32(mu + np.array([1e-38, -1e-38, 5e-39, 2.5e-39, 0.0]))
+    q8, step2 = nf4.second_level(scales, mu)
+    d = nf4.fl32(scales - mu)
+    st = float(np.float32(np.abs(d).max() / 127.0))
+    assert step2[0] == st and not np.isfinite(np.float32(1.0) / np.float32(st))
+    want = np.clip(np.rint([float(np.float32(float(Fraction(x) / Fraction(st)))) for x in d]), -127, 127)
+    assert np.array_equal(q8, want.astype(np.int8))
+    assert q8[0] == 127 and q8[1] == -127 and 0 < abs(int(q8[2])) < 127 and q8[4] == 0
