@@ -88,8 +88,8 @@ const Tables* tables_for(int kind) {
 const Tables& tables() { return *tables_for(QLORA_CODEBOOK_NF4); }
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
-inline size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+constexpr int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+constexpr size_t round256(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
 
 // ------------------------------------------------------------------ timing
 struct TimedLaunch {
@@ -236,7 +236,7 @@ struct QuantWs {
   int64_t tree_count;  // doubles reserved for all tree passes
 };
 
-QuantWs quant_ws(int64_t rows, int64_t cols) {
+constexpr QuantWs quant_ws(int64_t rows, int64_t cols) {
   QuantWs w{};
   const int64_t n_blocks = rows * cols / 64;
   w.absmax_off = 0;
@@ -1026,26 +1026,66 @@ constexpr size_t kNoAllocScratchBytes =
     ((static_cast<size_t>(kNoAllocMaxBlocks) * 4 + 255) & ~static_cast<size_t>(255)) +
     ((static_cast<size_t>(kNoAllocMaxBlocks / qnf4::kTreeChunk + 1) * 8 + 255) & ~static_cast<size_t>(255)) + 256;
 
+// The largest tensor the array accepts fits the quantizer's scratch layout
+// (block absmaxes, every tree pass's sums, the ticket words).
+static_assert(quant_ws(1, kNoAllocMaxBlocks * 64).total <= kNoAllocScratchBytes,
+              "the no-allocation scratch is smaller than the quantizer's workspace at its maximum size");
+static_assert(quant_ws(kNoAllocMaxBlocks / 4096, 4096 * 64).total <= kNoAllocScratchBytes,
+              "the no-allocation scratch is smaller than the quantizer's workspace at its maximum size");
+
 // One copy per device that loads the library.  In host code this name is a
 // host-side stand-in, never a device address: the address comes from
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// Identifier of the calling thread's current CUDA context (0 if unknown).
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+struct NoAllocAddr {
+  void* ptr;
+  unsigned long long ctx;   // context the address belongs to
+};
+NoAllocAddr g_noalloc_addr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device, looked up once
-// per device (with that device current).
+// per device (with that device current) and again only if the device's
+// context was replaced since (a reset destroys the module and its array).
 void* noalloc_scratch_for_current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  const unsigned long long ctx = current_context_id();      // 0 before the runtime made a context current
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocAddr& e = g_noalloc_addr[dev];
+  if (e.ptr == nullptr || ctx == 0 || e.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_addr[dev] = p;
+    e.ptr = p;
+    e.ctx = current_context_id();                           // the lookup made the context current
   }
-  return g_noalloc_addr[dev];
+  return e.ptr;
 }
 
 }  // namespace

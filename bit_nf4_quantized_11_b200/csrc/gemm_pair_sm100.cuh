@@ -67,6 +67,8 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
   uint64_t* acc_full = bars + 2 * kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // (even CTA) the number of stages whose copies each CTA of the pair issued
+  volatile int* issued_by = reinterpret_cast<volatile int*>(tmem_holder + 2);
 
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
@@ -118,10 +120,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
       tma_prefetch_desc(&tm_lora);
+      int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1u;
         wait(empty + s, ph ^ 1u);
+        if (*abort_flag) break;                           // a wait timed out: issue nothing more
         if (leader) mbar_arrive_expect_tx(full + s, 2 * Cfg::A_STAGE);    // both CTAs' bytes
         const uint32_t bar = mapa_shared(smem_u32(full + s), 0);
         const uint32_t dst = smem_u32(a_ring + s * Cfg::A_STAGE);
@@ -138,15 +142,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
           else
             tma_load_2d_pair(dst + sub * Cfg::A_SUB, &tm_lora, bar, (it - n_main) * 64, row);
         }
+        ++issued;
       }
-      // Copies of both CTAs complete on the even CTA's barriers: it waits
-      // (bounded) for the last phase of every stage before the final cluster
-      // barrier, so no copy of either CTA is in flight at exit.
-      if (leader) {
-        const int first = n_iter > kStages ? n_iter - kStages : 0;
-        for (int it = first; it < n_iter; ++it)
-          mbar_wait_cluster_bounded(full + (it % kStages), (it / kStages) & 1u, tmo);
-      }
+      // Copies of both CTAs complete on the even CTA's barriers, which drains
+      // them after the cluster barrier below; it needs both issued counts.
+      asm volatile("st.shared::cluster.u32 [%0], %1;"
+                   :: "r"(mapa_shared(smem_u32(const_cast<int*>(issued_by + rank)), 0)), "r"(issued) : "memory");
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
@@ -156,6 +157,7 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1u;
         wait(full + s, ph);
+        if (*abort_flag) break;                           // commit what was issued, then finish
         tc_fence_after_sync();
         const uint32_t a_base = smem_u32(a_ring + s * Cfg::A_STAGE);
         const uint32_t b_base = smem_u32(b_ring + s * Cfg::B_STAGE);
@@ -318,6 +320,16 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
 
   tc_fence_before_sync();
   __syncthreads();
+  cluster_sync_all();                 // both issued counts are visible to the even CTA
+  if (leader && warp == 0 && lane == 0) {
+    // Wait (bounded) for the stages whose copies may still be in flight: a
+    // stage more than kStages behind the last one issued was consumed, so
+    // its copies have landed.  Without a timeout every phase has completed
+    // and these waits return at once.
+    const int n = max(issued_by[0], issued_by[1]);
+    for (int it = n > kStages ? n - kStages : 0; it < n; ++it)
+      mbar_wait_cluster_bounded(full + (it % kStages), (it / kStages) & 1u, tmo);
+  }
   cluster_sync_all();                 // no CTA leaves while its pair may still use its memory
   if (warp == 1) {
     tc_fence_after_sync();

@@ -133,10 +133,12 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
     if (lane == 0) {
       tma_prefetch_desc(&tm_act);
       tma_prefetch_desc(&tm_lora);
+      int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1u;
         pipe_wait(empty + s, ph ^ 1u, tmo, abort_flag);
+        if (*abort_flag) break;                           // a wait timed out: issue nothing more
         mbar_arrive_expect_tx(full_a + s, Cfg::A_STAGE);
         const uint32_t dst = smem_u32(a_ring + s * Cfg::A_STAGE);
 #pragma unroll
@@ -146,10 +148,11 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
           else
             tma_load_2d(dst + sub * Cfg::A_SUB, &tm_lora, full_a + s, (it - n_main) * 64, m0 + sub * 128);
         }
+        ++issued;
       }
-      // make sure no copy is still in flight when the CTA exits
-      const int first = n_iter > kStages ? n_iter - kStages : 0;
-      for (int it = first; it < n_iter; ++it)
+      // make sure no copy is still in flight when the CTA exits: only the
+      // last kStages issued stages can be unconsumed
+      for (int it = issued > kStages ? issued - kStages : 0; it < issued; ++it)
         mbar_wait_bounded(full_a + (it % kStages), (it / kStages) & 1u, tmo);
     }
   } else if (warp == 1) {
@@ -161,6 +164,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
         const uint32_t ph = (it / kStages) & 1u;
         pipe_wait(full_a + s, ph, tmo, abort_flag);
         pipe_wait(full_b + s, ph, tmo, abort_flag);
+        if (*abort_flag) break;                           // commit what was issued, then finish
         tc_fence_after_sync();
         const uint32_t a_base = smem_u32(a_ring + s * Cfg::A_STAGE);
         const uint32_t b_base = smem_u32(b_ring + s * Cfg::B_STAGE);

@@ -381,8 +381,10 @@ int qlora_timing_collect(const char* kernel, double* total_ms, int64_t* launches
  * library holds until the process exits.  The call itself allocates nothing.
  *
  * The first call on a device looks up that array's device address (once per
- * device, with the device current); make that first call before any stream
- * capture begins.  Every call shares the one array: calls that can overlap on
+ * device, with the device current), and so does the first call after the
+ * device's context was destroyed and recreated (cudaDeviceReset), which
+ * gives the array a new address; make the first call (and the first after
+ * a reset) before any stream capture begins.  Every call shares the one array: calls that can overlap on
  * the GPU (different streams, or different host threads) race on it and must
  * be ordered by the caller.  The array keeps the previous call's contents;
  * each call overwrites every scratch value before reading it, so nothing has

@@ -16,6 +16,7 @@ import torch
 
 import bit_nf4_quantized_11_b200 as q
 from bit_nf4_quantized_11_b200 import synth
+from oracle import nf4
 
 pytestmark = pytest.mark.gpu
 
@@ -53,6 +54,13 @@ def test_noalloc_quantizer_matches_workspace_quantizer(cuda_lib):
         assert q.last_device_status() == 0
         for a, b in ((out.codes, ref.codes), (out.q8, ref.q8), (out.step2, ref.step2), (out.mean, ref.mean)):
             assert np.array_equal(_bits(a), _bits(b))
+        if i == 1:
+            # the second call also against the CPU oracle directly
+            o = nf4.quantize(W.cpu().numpy())
+            assert np.array_equal(out.codes.cpu().numpy(), o["packed"])
+            assert np.array_equal(out.q8.cpu().numpy(), o["q8"])
+            assert np.array_equal(_bits(out.step2), nf4.f32_bits(o["step2"]).view(np.uint8))
+            assert np.array_equal(_bits(out.mean), nf4.f32_bits([o["mean"]]).view(np.uint8))
 
 
 def test_noalloc_quantizer_rejects_sizes_beyond_its_scratch(cuda_lib):
