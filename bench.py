@@ -1,20 +1,24 @@
 #!/usr/bin/env python
 """Benchmark of the QLoRA NF4 linear layer on B200; prints ONE JSON line.
 
-Step = one QLoRA linear forward + backward (all kernels of the hot path:
-LoRA down-projection, fused dequant GEMM forward, du, fused dequant GEMM dx,
-dA, dB) on the Llama-7B attention-projection workload: in = out = 4096,
-M = 4096 tokens (batch 4 x seq 1024), r = 16, alpha = 32, frozen weight
-quantized once to NF4 with double quantization before timing.
+Step = forward + backward of all seven QLoRA linears of one Llama-65B-shaped
+decoder layer (q, k, v, o 8192x8192; gate, up 8192->22016; down 22016->8192;
+all NF4 with double quantization, LoRA r = 64, alpha = 16 on every one),
+M = 2048 tokens, each projection on its own seeded input: per projection the
+hot path's kernels (LoRA down-projection, fused dequant GEMM forward, du,
+fused dequant GEMM dx, dA and dB).  The frozen weights are quantized before
+timing; quantizing all seven is timed separately and reported in the same
+line.  Components (7B attention and MLP fwd+bwd, the 70B few-token GEMV, the
+quantizer variants, the adapter merge, LoRA dropout) follow on N = 1.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 N > 1: launched with torch.distributed.run, one rank per GPU; every rank runs
-its own batch (data parallel, weak scaling) and the adapter gradients dA, dB
-are summed across ranks with one NCCL all-reduce per step.  Time = max over
-ranks of the CUDA-event time of exactly K steps, bracketed by barrier +
-synchronize.  `--impl reference` times the fp64 CPU oracle (rank 0 only) on a
-bounded token sample of the same workload.
+its own batch (data parallel, weak scaling) and the adapter gradients of the
+layer (one flat fp32 buffer) are summed across ranks with one NCCL all-reduce
+per step.  Time = max over ranks of the CUDA-event time of exactly K steps,
+bracketed by barrier + synchronize.  `--impl reference` times the fp64 CPU
+oracle (rank 0 only) on a bounded token sample of the same workload.
 """
 
 from __future__ import annotations
@@ -39,7 +43,7 @@ from bit_nf4_quantized_11_b200 import dp, synth, workloads  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 quant/GEMV GB/s, % of B200 roofline"
 L2_BYTES = 126 * 2 ** 20
-WL = workloads.ATTN_7B
+WL = workloads.LAYER_65B          # the largest configuration that fits one GPU
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -47,14 +51,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--rotations", type=int, default=4)
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout"], default=None,
+    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout", "layer_step"],
+                    default=None,
                     help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -182,54 +186,86 @@ def barrier(world):
 
 
 # ---------------------------------------------------------------------------- our arm
-def step_flops(M, n_in, n_out, r):
-    return workloads.fwd_bwd_flops(M, n_in, n_out, r)
+def gemm_flops(kernel, M, n_in, n_out, r):
+    """Algorithmic FLOPs of one launch of a fused dequant GEMM: the forward
+    contracts [x | us] with [W0 | B] (K = in + r), dx [dh | du] with [W0 ; A]."""
+    return 2.0 * M * (n_out * (n_in + r) if kernel == "gemm_fwd" else n_in * (n_out + r))
 
 
-def make_copies(q, M, n_in, n_out, r, n_rot, seed0, dev):
-    copies = []
-    for i in range(n_rot):
-        p = synth.problem(M, n_in, n_out, r, WL.w_std, WL.w_dist, seed=seed0 + 17 * i)
-        c = {k: p[k].to(dev) for k in ("x", "A", "B", "dh")}
-        c["w"] = q.quantize_nf4(p["W"].to(dev))
-        copies.append(c)
-    torch.cuda.synchronize()
-    return copies
+class LayerState:
+    """One rank's device-resident copy of the headline workload: every
+    projection's fp32 weight (for the quantizer figure), its NF4 weight, its
+    own inputs x, dh, the adapters A, B, the outputs and the workspaces; the
+    adapter gradients of all projections live in one flat buffer."""
+
+    def __init__(self, q, wl, seed0, dev):
+        self.q, self.wl, self.M, self.r, self.alpha = q, wl, wl.M[0], wl.r, wl.alpha
+        self.shapes = [(n_in, n_out) for _, n_in, n_out in wl.projections]
+        self.flat, grads = dp.layer_grad_buffers(self.r, self.shapes, dev)
+        self.proj = []
+        for i, ((label, n_in, n_out), (dA, dB)) in enumerate(zip(wl.projections, grads)):
+            p = synth.problem(self.M, n_in, n_out, self.r, wl.w_std, wl.w_dist, seed=seed0 + i)
+            c = {k: p[k].to(dev) for k in ("W", "x", "A", "B", "dh")}
+            del p
+            c["label"], c["n_in"], c["n_out"] = label, n_in, n_out
+            c["w"] = q.alloc_nf4(n_out, n_in, dev)
+            c["h"] = torch.empty(self.M, n_out, dtype=torch.bfloat16, device=dev)
+            c["us"] = torch.empty(self.M, self.r, dtype=torch.bfloat16, device=dev)
+            c["dx"] = torch.empty(self.M, n_in, dtype=torch.bfloat16, device=dev)
+            c["dA"], c["dB"] = dA, dB
+            self.proj.append(c)
+        ws = lambda op: max(max(1, q.workspace_size(op, self.M, n_in, n_out, self.r))  # noqa: E731
+                            for n_in, n_out in self.shapes)
+        self.ws_f = torch.empty(ws(q.OP_LINEAR_FWD), dtype=torch.uint8, device=dev)
+        self.ws_b = torch.empty(ws(q.OP_LINEAR_BWD), dtype=torch.uint8, device=dev)
+        self.ws_q = torch.empty(max(q.workspace_size(q.OP_QUANTIZE, 0, n_in, n_out, 0) for n_in, n_out in self.shapes),
+                                dtype=torch.uint8, device=dev)
+        self.quantize()
+        torch.cuda.synchronize()
+
+    def quantize(self):
+        for c in self.proj:
+            self.q.quantize_nf4(c["W"], out=c["w"], workspace=self.ws_q)
+
+    def step(self, world=1):
+        q, a = self.q, self.alpha
+        for c in self.proj:
+            q.linear_fwd(c["x"], c["w"], c["A"], c["B"], a, h=c["h"], us=c["us"], workspace=self.ws_f)
+            q.linear_bwd(c["dh"], c["x"], c["us"], c["w"], c["A"], c["B"], a, dx=c["dx"], dA=c["dA"], dB=c["dB"],
+                         workspace=self.ws_b)
+        if world > 1:                       # data-parallel adapter-gradient sum, one all-reduce per layer
+            dp.allreduce_adapter_grads(self.flat)
+
+    def flops(self):
+        return sum(workloads.fwd_bwd_flops(self.M, n_in, n_out, self.r) for n_in, n_out in self.shapes)
+
+    def gemm_flops(self, kernel):
+        return sum(gemm_flops(kernel, self.M, n_in, n_out, self.r) for n_in, n_out in self.shapes)
+
+    def input_bytes(self):
+        return sum(c[k].numel() * c[k].element_size() for c in self.proj for k in ("x", "dh")) + \
+            sum(c["w"].nbytes() for c in self.proj)
 
 
 def run_ours(args, world, rank, local):
     import bit_nf4_quantized_11_b200 as q
     q.load()
     dev = torch.device("cuda", local)
-    (_, n_in, n_out), = WL.projections
-    M, r, alpha = WL.M[0], WL.r, WL.alpha
-    copies = make_copies(q, M, n_in, n_out, r, args.rotations, 1000 * rank, dev)
-    h = torch.empty(M, n_out, dtype=torch.bfloat16, device=dev)
-    us = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    dx = torch.empty(M, n_in, dtype=torch.bfloat16, device=dev)
-    grads, dA, dB = dp.adapter_grad_buffers(r, n_in, n_out, dev)
-    ws_f = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_FWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_BWD, M, n_in, n_out, r)), dtype=torch.uint8, device=dev)
+    L = LayerState(q, WL, 1000 * rank, dev)
 
-    def step(i):
-        c = copies[i % len(copies)]
-        q.linear_fwd(c["x"], c["w"], c["A"], c["B"], alpha, h=h, us=us, workspace=ws_f)
-        q.linear_bwd(c["dh"], c["x"], us, c["w"], c["A"], c["B"], alpha, dx=dx, dA=dA, dB=dB, workspace=ws_b)
-        if world > 1:                       # data-parallel adapter-gradient sum
-            dp.allreduce_adapter_grads(grads)
-
-    for i in range(args.warmup):
-        step(i)
+    for _ in range(args.warmup):
+        L.step(world)
     torch.cuda.synchronize()
     if q.last_device_status() != 0:
         raise RuntimeError("device wait timed out during warm-up")
 
     stream = torch.cuda.current_stream()
 
-    def timed_region(per_kernel: bool):
-        """K steps between barrier+synchronize, CUDA events on this stream;
-        with per_kernel, the library also brackets each of its launches with
-        events (the headline value comes from the region without them)."""
+    def timed_region(per_kernel: bool, body, n):
+        """n calls of body between barrier+synchronize, CUDA events on this
+        stream; with per_kernel, the library also brackets each of its
+        launches with events (the headline value comes from the region
+        without them)."""
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         q.timing_reset()
         q.timing_enable(per_kernel)
@@ -237,8 +273,8 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         with ClockSampler(local) as clk:
             e0.record(stream)
-            for i in range(args.steps):
-                step(i)
+            for _ in range(n):
+                body()
             e1.record(stream)
             torch.cuda.synchronize()
         barrier(world)
@@ -247,12 +283,13 @@ def run_ours(args, world, rank, local):
             raise RuntimeError("device wait timed out in the timed region")
         return max_over_ranks(e0.elapsed_time(e1), world), clk
 
-    ms_max, clk = timed_region(per_kernel=False)
-    flops = step_flops(M, n_in, n_out, r)
+    step = lambda: L.step(world)  # noqa: E731
+    ms_max, clk = timed_region(False, step, args.steps)
+    flops = L.flops()
     value = world * args.steps * flops / (ms_max * 1e-3) / 1e12
 
     # identical second region with per-kernel events: breakdown, launch count, roofline
-    ms_events, _ = timed_region(per_kernel=True)
+    ms_events, _ = timed_region(True, step, args.steps)
     kern = {}
     launches = 0
     for name in q.KERNEL_NAMES:
@@ -266,98 +303,137 @@ def run_ours(args, world, rank, local):
 
     peaks, peak_src = load_peaks()
     dom = max(("gemm_fwd", "gemm_dx"), key=lambda k: kern.get(k, {}).get("ms_per_step", 0.0))
-    dom_flops = 2.0 * M * (n_out * (n_in + r) if dom == "gemm_fwd" else n_in * (n_out + r))
+    launches_per_step = kern[dom]["launches"] / args.steps
+    dom_flops = L.gemm_flops(dom) / launches_per_step            # mean algorithmic FLOPs per launch
     achieved = dom_flops / (kern[dom]["avg_us"] * 1e-6) / 1e12
+    region_s = ms_max * 1e-3
+    long_region = region_s >= 2.0
+    peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
     roofline = {"kernel": dom, "bound": "tensor", "achieved": achieved,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"],
-                "peak_source": f"bf16_tflops_sustained of {peak_src} (kernel timed inside a long run of steps)",
-                "timing": "mean CUDA-event duration of the kernel's launches in a second K-step region "
-                          "identical to the timed one, events recorded on the launching stream",
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_source": ("bf16_tflops_sustained" if long_region else "bf16_tflops (burst)")
+                               + f" of {peak_src}: the timed region lasts {region_s:.2f} s "
+                               + ("(seconds-long, power-capped)" if long_region else "(well under the seconds-long "
+                                  "loop the sustained figure was measured on)"),
+                "timing": "mean CUDA-event duration of the kernel's launches (one per projection and step) in a "
+                          "second K-step region identical to the timed one, events recorded on the launching "
+                          "stream; achieved = mean algorithmic FLOPs per launch / mean duration",
                 "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
                 "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                 "flops_per_launch": dom_flops,
+                "step_frac_of_peak": value / world / peak,
                 "traffic": profiled_traffic(dom, WL.name)}
 
-    e2e = None if args.no_e2e else measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev)
+    # quantizing all seven weights, timed on its own (3.24 GB of fp32 weights > L2)
+    n_q = max(3, min(20, args.steps))
+    ms_q, _ = timed_region(False, L.quantize, n_q)
+    qbytes = sum(workloads.quant_bytes(n_out, n_in) for n_in, n_out in L.shapes)
+    qgbs = world * n_q * qbytes / (ms_q * 1e-3) / 1e9
+    quant = {"what": "NF4 + double quantization of the layer's seven fp32 weights "
+                     f"({sum(a * b for a, b in L.shapes) / 1e6:.1f} M weights)",
+             "ms": ms_q / n_q, "GB/s": qgbs, "unit": "GB/s", "bytes": qbytes,
+             "bound": "hbm", "peak": peaks["hbm_gbs"], "frac": qgbs / world / peaks["hbm_gbs"],
+             "peak_source": f"hbm_gbs of {peak_src}",
+             "bytes_rule": "4 B read + 0.5 B codes + 1/64 B scale codes + 4 B per 256 blocks per weight"}
 
-    rot_bytes = args.rotations * (2 * M * n_in + 2 * M * n_out + copies[0]["w"].nbytes())
+    e2e = None if args.no_e2e else measure_e2e(q, args, L, world, dev)
+
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic: seeded N(0,1) bf16 activations and output grads, N(0,0.02^2) fp32 "
-                "weight quantized once to NF4 + double quant, U(+-1/64) A, N(0,0.01^2) B",
-        "config": {"workload": WL.name, "in_features": n_in, "out_features": n_out,
-                   "tokens_per_gpu": M, "r": r, "alpha": alpha, "global_tokens": M * world,
+        "data": f"synthetic: seeded N(0,1) bf16 activations and output grads per projection, N(0,{WL.w_std}^2) fp32 "
+                "weights quantized to NF4 + double quant, U(+-1/sqrt(in)) A, N(0,0.01^2) B",
+        "config": {"workload": WL.name,
+                   "projections": [f"{lab} {a}->{b}" for lab, a, b in WL.projections],
+                   "tokens_per_gpu": L.M, "r": L.r, "alpha": L.alpha, "global_tokens": L.M * world,
                    "parallelism": f"dp{world}",
-                   "l2": f"inputs rotated over {args.rotations} copies ({rot_bytes / 2**20:.0f} MiB > 126 MiB L2)",
+                   "l2": f"inputs larger than L2: one step reads {L.input_bytes() / 2**20:.0f} MiB of distinct "
+                         "weights and activations (> 126 MiB L2), no projection's data is reused within a step",
                    "flops_per_step_per_gpu": flops},
         "roofline": roofline,
+        "quantize": quant,
         "e2e": e2e,
         "gpu_launches": launches,
         "ms_per_step_with_kernel_events": ms_events / args.steps,
         "clocks": clk.summary(),
         "kernels": kern,
     }
+    del L
+    torch.cuda.empty_cache()
     return line
 
 
-def measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev):
+def measure_e2e(q, args, L, world, dev):
     """Same step through the public API with inputs in pinned host memory:
-    every step copies x, dh host->device and h, dx, dA, dB device->host.
-    Steps are pipelined over two buffer sets on three streams (host->device
-    copies, the layer, device->host copies), so the copies of one step
-    overlap the layer of its neighbours; every step's own copies are inside
-    the timed region."""
-    c = copies[0]
-    n = max(10, min(100, args.steps // 10))
-    xh = [c["x"].cpu().pin_memory() for _ in range(2)]
-    dhh = [c["dh"].cpu().pin_memory() for _ in range(2)]
-    xs = [torch.empty_like(c["x"]) for _ in range(2)]
-    dhs = [torch.empty_like(c["dh"]) for _ in range(2)]
-    hs = [torch.empty(M, n_out, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    uss = [torch.empty(M, r, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    dxs = [torch.empty(M, n_in, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-    gs = [dp.adapter_grad_buffers(r, n_in, n_out, dev) for _ in range(2)]
-    h_host = [torch.empty(M, n_out, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    dx_host = [torch.empty(M, n_in, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    g_host = [torch.empty(r * n_in + n_out * r, dtype=torch.float32).pin_memory() for _ in range(2)]
+    every step copies each projection's x, dh host->device and its h, dx
+    device->host, and the layer's flat adapter gradients (dA, dB of all
+    projections) device->host.  Projections are pipelined over two buffer
+    sets on three streams (host->device copies, the layer, device->host
+    copies), so the copies of one projection overlap the compute of its
+    neighbours; every step's own copies are inside the timed region."""
+    P = len(L.proj)
+    n = max(3, min(10, args.steps // 5))
+    bufs = []
+    for c in L.proj:
+        sets = []
+        for _ in range(2):
+            sets.append({"xh": c["x"].cpu().pin_memory(), "dhh": c["dh"].cpu().pin_memory(),
+                         "x": torch.empty_like(c["x"]), "dh": torch.empty_like(c["dh"]),
+                         "h": torch.empty_like(c["h"]), "us": torch.empty_like(c["us"]),
+                         "dx": torch.empty_like(c["dx"]),
+                         "h_host": torch.empty(c["h"].shape, dtype=torch.bfloat16).pin_memory(),
+                         "dx_host": torch.empty(c["dx"].shape, dtype=torch.bfloat16).pin_memory()})
+        bufs.append(sets)
+    grads = [dp.layer_grad_buffers(L.r, L.shapes, dev) for _ in range(2)]
+    g_host = [torch.empty(grads[0][0].numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
     s_in, s_run, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ws_f = torch.empty(max(q.workspace_size(q.OP_LINEAR_FWD, M, n_in, n_out, r), 1), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(max(q.workspace_size(q.OP_LINEAR_BWD, M, n_in, n_out, r), 1), dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event()  # noqa: E731
-    loaded, computed, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
-    used = [ev(), ev()]
+    loaded = [[ev(), ev()] for _ in range(P)]
+    used = [[ev(), ev()] for _ in range(P)]
+    computed = [[ev(), ev()] for _ in range(P)]
+    drained = [[ev(), ev()] for _ in range(P)]
+    g_done, g_drained = [ev(), ev()], [ev(), ev()]
 
     def step(i):
         k = i % 2
-        with torch.cuda.stream(s_in):
-            if i >= 2:
-                s_in.wait_event(used[k])                    # step i-2 no longer reads this input set
-            xs[k].copy_(xh[k], non_blocking=True)
-            dhs[k].copy_(dhh[k], non_blocking=True)
-            loaded[k].record(s_in)
+        flat, views = grads[k]
+        for p, c in enumerate(L.proj):
+            b = bufs[p][k]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(used[p][k])             # step i-2 no longer reads this input set
+                b["x"].copy_(b["xh"], non_blocking=True)
+                b["dh"].copy_(b["dhh"], non_blocking=True)
+                loaded[p][k].record(s_in)
+            with torch.cuda.stream(s_run):
+                s_run.wait_event(loaded[p][k])
+                if i >= 2:
+                    s_run.wait_event(drained[p][k])         # step i-2's outputs are on the host
+                    if p == 0:
+                        s_run.wait_event(g_drained[k])      # and its gradients
+                dA, dB = views[p]
+                q.linear_fwd(b["x"], c["w"], c["A"], c["B"], L.alpha, h=b["h"], us=b["us"], workspace=L.ws_f)
+                q.linear_bwd(b["dh"], b["x"], b["us"], c["w"], c["A"], c["B"], L.alpha, dx=b["dx"], dA=dA, dB=dB,
+                             workspace=L.ws_b)
+                used[p][k].record(s_run)
+                computed[p][k].record(s_run)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[p][k])
+                b["h_host"].copy_(b["h"], non_blocking=True)
+                b["dx_host"].copy_(b["dx"], non_blocking=True)
+                drained[p][k].record(s_out)
         with torch.cuda.stream(s_run):
-            s_run.wait_event(loaded[k])
-            if i >= 2:
-                s_run.wait_event(drained[k])                # step i-2's outputs are on the host
-            flat, dA, dB = gs[k]
-            q.linear_fwd(xs[k], c["w"], c["A"], c["B"], alpha, h=hs[k], us=uss[k], workspace=ws_f)
-            q.linear_bwd(dhs[k], xs[k], uss[k], c["w"], c["A"], c["B"], alpha, dx=dxs[k], dA=dA, dB=dB,
-                         workspace=ws_b)
             if world > 1:
                 dp.allreduce_adapter_grads(flat)
-            used[k].record(s_run)
-            computed[k].record(s_run)
+            g_done[k].record(s_run)
         with torch.cuda.stream(s_out):
-            s_out.wait_event(computed[k])
-            h_host[k].copy_(hs[k], non_blocking=True)
-            dx_host[k].copy_(dxs[k], non_blocking=True)
-            g_host[k].copy_(gs[k][0], non_blocking=True)
-            drained[k].record(s_out)
+            s_out.wait_event(g_done[k])
+            g_host[k].copy_(flat, non_blocking=True)
+            g_drained[k].record(s_out)
 
-    for i in range(4):
+    for i in range(2):
         step(i)
     torch.cuda.synchronize()
     barrier(world)
@@ -365,15 +441,17 @@ def measure_e2e(q, args, copies, M, n_in, n_out, r, alpha, world, dev):
     e0.record(s_in)
     for i in range(n):
         step(i)
-    e1.record(s_out)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world)
-    flops = step_flops(M, n_in, n_out, r)
-    return {"value": world * n * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": 2 * M * n_in + 2 * M * n_out,
-            "d2h_bytes_per_step": 2 * M * n_out + 2 * M * n_in + 4 * r * n_in + 4 * n_out * r,
+    h2d = sum(c["x"].numel() * 2 + c["dh"].numel() * 2 for c in L.proj)
+    d2h = sum(c["h"].numel() * 2 + c["dx"].numel() * 2 for c in L.proj) + 4 * grads[0][0].numel()
+    return {"value": world * n * L.flops() / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": n, "ms_per_step": ms / n,
-            "pipeline": "2 buffer sets on 3 streams: the host<->device copies of neighbouring steps overlap the layer"}
+            "pipeline": "per projection: 2 buffer sets on 3 streams, the host<->device copies of neighbouring "
+                        "projections overlap the compute; the step ends when its last copy to the host is done"}
 
 
 # ---------------------------------------------------------------------------- oracle legs
@@ -389,14 +467,20 @@ def blas_threads():
 
 
 class OracleLayer:
-    """The fp64 oracle set up once on the workload's weight (quantized and
-    dequantized by the oracle itself)."""
+    """The fp64 oracle set up once on one projection of the headline layer
+    (its weight quantized and dequantized by the oracle itself).  The oracle
+    is timed on a token sample through this projection: quantizing all seven
+    of the layer's weights in fp64 NumPy would take minutes and ~10 GB of host
+    memory, and the oracle's FLOP rate does not depend on which projection
+    it runs."""
+
+    PROJ = 0          # q_proj, 8192 x 8192
 
     def __init__(self, seed=0):
         from oracle import linear, nf4
-        (_, n_in, n_out), = WL.projections
-        self.linear, self.n_in, self.n_out, self.r, self.alpha = linear, n_in, n_out, WL.r, WL.alpha
-        p = synth.problem(WL.M[0], n_in, n_out, WL.r, WL.w_std, WL.w_dist, seed)
+        label, n_in, n_out = WL.projections[self.PROJ]
+        self.label, self.linear, self.n_in, self.n_out, self.r, self.alpha = label, linear, n_in, n_out, WL.r, WL.alpha
+        p = synth.problem(WL.M[0], n_in, n_out, WL.r, WL.w_std, WL.w_dist, seed + self.PROJ)
         qo = nf4.quantize(p["W"].numpy())
         self.Wd = nf4.dequantize(qo["codes"], qo["q8"], qo["step2"], qo["mean"])
         self.x = p["x"].float().numpy().astype("float64")
@@ -409,23 +493,26 @@ class OracleLayer:
         x, dh = self.x[sl], self.dh[sl]
         self.linear.linear_fwd(x, self.Wd, self.A, self.B, self.alpha)
         self.linear.linear_bwd(dh, x, self.Wd, self.A, self.B, self.alpha)
-        return step_flops(x.shape[0], self.n_in, self.n_out, self.r)
+        return workloads.fwd_bwd_flops(x.shape[0], self.n_in, self.n_out, self.r)
+
+    def describe(self, m):
+        return (f"fp64 NumPy oracle fwd+bwd of {m} of the {WL.M[0]} tokens through the layer's {self.label} "
+                f"({self.n_out}x{self.n_in}, r={self.r}), the oracle's own NF4 weight")
 
 
 def cpu_baseline(budget_s=15.0):
     ol = OracleLayer()
     t0 = time.perf_counter()
-    ol.step(0, 64)
-    per_tok = (time.perf_counter() - t0) / 64
-    m = int(max(64, min(WL.M[0], budget_s / max(per_tok, 1e-9))))
-    # whole steps repeated until about budget_s of work (one step when it alone is longer)
+    ol.step(0, 32)
+    per_tok = (time.perf_counter() - t0) / 32
+    m = int(max(32, min(WL.M[0], budget_s / max(per_tok, 1e-9))))
+    # whole samples repeated until about budget_s of work (one when it alone is longer)
     reps = max(1, int(budget_s / max(per_tok * m, 1e-9)))
     t0 = time.perf_counter()
     flops = sum(ol.step(0, m) for _ in range(reps))
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"fp64 NumPy oracle fwd+bwd of {m} of the {WL.M[0]} tokens through the full "
-                      f"{ol.n_out}x{ol.n_in} layer (r={ol.r}), {reps} time(s); {dt:.1f} s"}
+            "sample": f"{ol.describe(m)}, {reps} time(s); {dt:.1f} s"}
 
 
 def run_reference(args, world, rank):
@@ -446,15 +533,15 @@ def run_reference(args, world, rank):
     dt = time.perf_counter() - t0
     value = flops / dt / 1e12
     cores = blas_threads()
-    sample = f"fp64 NumPy oracle fwd+bwd of {m} tokens per step through the full {ol.n_out}x{ol.n_in} layer"
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded inputs as the GPU arm)",
-        "config": {"workload": WL.name, "in_features": ol.n_in, "out_features": ol.n_out,
+        "config": {"workload": WL.name, "sampled_projection": f"{ol.label} {ol.n_in}->{ol.n_out}",
                    "tokens_per_step": m, "r": ol.r, "alpha": ol.alpha},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{ol.describe(m)} per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -655,23 +742,32 @@ def comp_gemv(q, dev, peaks, n=60):
         B = synth.lora_B(n_out, g.r).to(dev)
         for M in g.M:
             x = synth.activations(M, n_in, seed=M).to(dev)
+            h = torch.empty(M, n_out, dtype=torch.bfloat16, device=dev)
+            us = torch.empty(M, g.r, dtype=torch.bfloat16, device=dev)
+            wsf = torch.empty(max(1, q.workspace_size(q.OP_LINEAR_FWD, M, n_in, n_out, g.r)), dtype=torch.uint8,
+                              device=dev)
+            call = lambda i: q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha, h=h, us=us, workspace=wsf)  # noqa: E731
             for i in range(3):
-                q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha)
+                call(i)
             torch.cuda.synchronize()
-            q.timing_reset()
-            q.timing_enable(True)
-            a.record()
+            a.record()                                  # whole calls, no per-kernel events
             for i in range(n):
-                q.linear_fwd(x, ws_list[i % 3], A, B, g.alpha)
+                call(i)
             b.record()
             torch.cuda.synchronize()
-            q.timing_enable(False)
             call_ms = a.elapsed_time(b) / n
+            q.timing_reset()                            # the same calls again, kernels bracketed by events
+            q.timing_enable(True)
+            for i in range(n):
+                call(i)
+            torch.cuda.synchronize()
+            q.timing_enable(False)
             kms, kn = q.timing_collect("gemv")
             wbytes = workloads.gemv_weight_bytes(n_out, n_in)
             gres[f"{label}_{n_in}x{n_out}_M{M}"] = {
                 "call_us": 1e3 * call_ms, "gemv_kernel_us": 1e3 * kms / kn if kn else None,
                 "packed_weight_GB/s_call": wbytes / (call_ms * 1e-3) / 1e9,
+                "frac_hbm_call": wbytes / (call_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "packed_weight_GB/s_kernel": wbytes / (kms / kn * 1e-3) / 1e9 if kn else None,
                 "frac_hbm_kernel": (wbytes / (kms / kn * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kn else None}
         del ws_list
@@ -679,37 +775,36 @@ def comp_gemv(q, dev, peaks, n=60):
     return {"gemv_70b": gres}
 
 
-def comp_workloads(q, dev, peaks):
-    """fwd+bwd of the 7B MLP (3 projections) and the 65B decoder layer (7 projections)."""
-    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    a, b = ev(), ev()
+def comp_workloads(q, dev, peaks, n=10):
+    """fwd+bwd of the 7B attention projection and of the 7B MLP (3 projections),
+    each projection on its own inputs, clean CUDA-event timing."""
     out = {}
-    for wl in (workloads.MLP_7B, workloads.LAYER_65B):
-        M = wl.M[0]
-        tot_ms, tot_flops = 0.0, 0.0
-        for i, (label, n_in, n_out) in enumerate(wl.projections):
-            p = synth.problem(M, n_in, n_out, wl.r, wl.w_std, wl.w_dist, seed=i)
-            w = q.quantize_nf4(p["W"].to(dev))
-            x, A, B, dh = (p[k].to(dev) for k in ("x", "A", "B", "dh"))
-            del p
-            for _ in range(2):
-                hh, us = q.linear_fwd(x, w, A, B, wl.alpha)
-                q.linear_bwd(dh, x, us, w, A, B, wl.alpha)
-            torch.cuda.synchronize()
-            n = 5
-            a.record()
-            for _ in range(n):
-                hh, us = q.linear_fwd(x, w, A, B, wl.alpha)
-                q.linear_bwd(dh, x, us, w, A, B, wl.alpha)
-            b.record()
-            torch.cuda.synchronize()
-            tot_ms += a.elapsed_time(b) / n
-            tot_flops += step_flops(M, n_in, n_out, wl.r)
-            del w, x, A, B, dh, hh, us
-            torch.cuda.empty_cache()
-        out[wl.name] = {"ms": tot_ms, "TFLOP/s": tot_flops / (tot_ms * 1e-3) / 1e12,
-                        "frac_bf16_sustained": tot_flops / (tot_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]}
+    for wl in (workloads.ATTN_7B, workloads.MLP_7B):
+        L = LayerState(q, wl, 0, dev)
+        for _ in range(3):
+            L.step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            L.step()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / n
+        tf = L.flops() / (ms * 1e-3) / 1e12
+        out[wl.name] = {"ms": ms, "TFLOP/s": tf, "frac_bf16_burst": tf / peaks["bf16_tflops"],
+                        "frac_bf16_sustained": tf / peaks["bf16_tflops_sustained"]}
+        del L
+        torch.cuda.empty_cache()
     return out
+
+
+def layer_step_once(q, dev):
+    """One untimed step of the headline layer (for a profiler's launch list)."""
+    L = LayerState(q, WL, 0, dev)
+    L.step()
+    torch.cuda.synchronize()
+    return {"ok": q.last_device_status() == 0, "projections": len(L.proj)}
 
 
 def components(q, dev, only=None):
@@ -727,6 +822,8 @@ def components(q, dev, only=None):
         out.update(comp_merge(q, dev, peaks, src))
     if only in (None, "dropout"):
         out.update(comp_dropout(q, dev, peaks))
+    if only == "layer_step":
+        out.update(layer_step_once(q, dev))
     return out
 
 

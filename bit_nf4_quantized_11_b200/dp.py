@@ -43,6 +43,19 @@ def adapter_grad_buffers(r: int, n_in: int, n_out: int, device) -> tuple[torch.T
     return flat, dA, dB
 
 
+def layer_grad_buffers(r: int, shapes, device):
+    """(flat, [(dA, dB), ...]) for several projections ((n_in, n_out), ...) of
+    one layer: every projection's dA [r, in] and dB [out, r] are fp32 views of
+    one contiguous buffer, so the layer's gradient sum is one all-reduce."""
+    sizes = [r * n_in + n_out * r for n_in, n_out in shapes]
+    flat = torch.empty(sum(sizes), dtype=torch.float32, device=device)
+    views, off = [], 0
+    for (n_in, n_out), n in zip(shapes, sizes):
+        views.append((flat[off: off + r * n_in].view(r, n_in), flat[off + r * n_in: off + n].view(n_out, r)))
+        off += n
+    return flat, views
+
+
 def allreduce_adapter_grads(flat: torch.Tensor, group=None) -> None:
     """Sum the flat adapter-gradient buffer over the ranks of `group`."""
     if torch.distributed.is_available() and torch.distributed.is_initialized():

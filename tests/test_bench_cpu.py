@@ -25,4 +25,4 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["n_gpus"] == 1
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
-    assert d["config"]["workload"].startswith("llama7b-attn")
+    assert d["config"]["workload"].startswith("llama65b-decoder-layer")

@@ -55,6 +55,21 @@ def _rank(rank, world, port, out):
         torch.distributed.destroy_process_group()
 
 
+def test_layer_grad_buffers_are_disjoint_views():
+    shapes = [(64, 128), (128, 96), (96, 64)]
+    flat, views = dp.layer_grad_buffers(8, shapes, "cpu")
+    assert flat.numel() == sum(8 * a + b * 8 for a, b in shapes)
+    flat.zero_()
+    for i, ((dA, dB), (n_in, n_out)) in enumerate(zip(views, shapes)):
+        assert dA.shape == (8, n_in) and dB.shape == (n_out, 8)
+        dA.fill_(2 * i + 1)
+        dB.fill_(2 * i + 2)
+    # every element of the flat buffer belongs to exactly one view, in order
+    want = torch.cat([torch.full((8 * a,), 2.0 * i + 1) if j == 0 else torch.full((b * 8,), 2.0 * i + 2)
+                      for i, (a, b) in enumerate(shapes) for j in (0, 1)])
+    assert torch.equal(flat, want)
+
+
 def test_two_rank_adapter_gradient_sum():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))

@@ -135,7 +135,18 @@ def test_full_size_65b_down(cuda_lib):
     _run(cuda_lib, 2048, 22016, 8192, 64, 16.0, w_std=0.01, sample_rows=_sample(2048, 128))
 
 
-@pytest.mark.parametrize("M,n_in,n_out", [(1, 8192, 28672), (16, 8192, 28672), (4, 28672, 8192)])
+def test_full_size_7b_mlp_down(cuda_lib):
+    _run(cuda_lib, 8192, 11008, 4096, 16, 32.0, w_dist="student_t5", sample_rows=_sample(8192, 128))
+
+
+@pytest.mark.parametrize("n_in,n_out", [(8192, 8192), (8192, 22016)])
+def test_full_size_65b_layer(cuda_lib, n_in, n_out):
+    # q/k/v/o share the 8192 x 8192 shape; gate and up share 8192 -> 22016
+    _run(cuda_lib, 2048, n_in, n_out, 64, 16.0, w_std=0.01, seed=n_out, sample_rows=_sample(2048, 128))
+
+
+@pytest.mark.parametrize("M,n_in,n_out", [(1, 8192, 28672), (4, 8192, 28672), (16, 8192, 28672),
+                                           (1, 28672, 8192), (4, 28672, 8192), (16, 28672, 8192)])
 def test_full_size_70b_gemv(cuda_lib, M, n_in, n_out):
     _run(cuda_lib, M, n_in, n_out, 16, 32.0, w_std=0.015, backward=False,
          sample_out=_sample(n_out, 512, seed=M))
