@@ -23,6 +23,8 @@
 #include "dropout.cuh"
 #include "quant.cuh"
 #include "skinny.cuh"
+#include "lora_sm100.cuh"
+#include "pad.cuh"
 
 namespace qnf4_host {
 void build_codebook(float levels[16], float thresholds[15]);
@@ -173,13 +175,14 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
 }
 
 // 2-D byte tensor [rows, cols] (packed NF4 codes, cols = in / 2), box
-// {128 bytes, 256 rows}, 128B swizzle, out-of-range bytes read as zero.
+// {128 bytes, 16 rows} (one warp's code tile of the GEMV), 128B swizzle,
+// out-of-range bytes read as zero.
 bool make_tmap_codes(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(qnf4::kGvStageK / 2), static_cast<cuuint32_t>(qnf4::kGvRows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(qnf4::kGvSlice / 2), static_cast<cuuint32_t>(qnf4::kGvTile)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -254,45 +257,71 @@ constexpr QuantWs quant_ws(int64_t rows, int64_t cols) {
   return w;
 }
 
+// Few-token GEMV plan: warps own 256-column K slices, a CTA's WARPS slices
+// form a K group, items are (group, 16-row tile); one CTA per SM.
 struct GemvPlan {
-  int ctas, local_tiles, n_st;
-  int64_t n_units;
+  int nt;                 // 8 or 16 token columns
+  int warps, n_slices, groups, tiles, ctas;
+  int64_t n_items;
+  size_t ws;              // workspace: the group partials (groups > 1)
 };
 
-int gemv_ctas_per_sm() {
+// Of the four MMA steps of a block, how many decode the rows g + 8 with the
+// register table instead of the shared one (QLORA_NF4_GEMV_REG_STEPS
+// overrides the default for tuning).
+int gemv_reg_steps() {
+  static int v = [] {
+    const char* e = std::getenv("QLORA_NF4_GEMV_REG_STEPS");
+    const int n = e ? std::atoi(e) : 0;
+    return (n == 1 || n == 2) ? n : 0;
+  }();
+  return v;
+}
+
+template <int NT>
+using GemvKernel = void (*)(const CUtensorMap, const qnf4::GemvArgs);
+
+template <int NT>
+GemvKernel<NT> gemv_kernel_for() {
+  switch (gemv_reg_steps()) {
+    case 1: return qnf4::nf4_gemv_kernel<NT, 1>;
+    case 2: return qnf4::nf4_gemv_kernel<NT, 2>;
+    default: return qnf4::nf4_gemv_kernel<NT, 0>;
+  }
+}
+
+template <int NT>
+int gemv_ctas_per_sm_t() {
+  using C = qnf4::GvCfg<NT>;
   static std::atomic<int> cache[kMaxDevices];
   const int dev = current_device();
   const int c = cache[dev].load(std::memory_order_relaxed);
   if (c > 0) return c;
   int n = 0;
-  const void* kern = reinterpret_cast<const void*>(qnf4::nf4_gemv_kernel<true, true>);
-  if (set_max_smem(kern, qnf4::kGvSmem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel<true, true>, qnf4::kGvThreads,
-                                                    qnf4::kGvSmem) != cudaSuccess ||
-      n < 1)
+  const GemvKernel<NT> k = gemv_kernel_for<NT>();
+  if (set_max_smem(reinterpret_cast<const void*>(k), C::SMEM) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::THREADS, C::SMEM) != cudaSuccess || n < 1)
     return 1;
   cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
-// Persistent grid (every CTA resident at once) splitting the (256-row tile x
-// 256-column unit) sequence evenly; local_tiles bounds the tiles one CTA's
-// range touches.
-GemvPlan gemv_plan(int64_t in, int64_t out) {
+GemvPlan gemv_plan(int64_t M, int64_t in, int64_t out) {
   GemvPlan p{};
-  p.n_st = static_cast<int>(cdiv(in, qnf4::kGvStageK));
-  p.n_units = cdiv(out, qnf4::kGvRows) * p.n_st;
-  const int64_t resident = static_cast<int64_t>(gemv_ctas_per_sm()) * device_sm_count();
-  p.ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(resident, p.n_units)));
-  const int64_t per_cta = cdiv(p.n_units, p.ctas);
-  p.local_tiles = static_cast<int>(cdiv(per_cta, p.n_st) + 1);
+  p.nt = M > 8 ? 16 : 8;
+  p.warps = p.nt == 8 ? qnf4::GvCfg<8>::WARPS : qnf4::GvCfg<16>::WARPS;
+  p.n_slices = static_cast<int>(cdiv(in, qnf4::kGvSlice));
+  p.groups = static_cast<int>(cdiv(p.n_slices, p.warps));
+  p.tiles = static_cast<int>(out / qnf4::kGvTile);
+  p.n_items = static_cast<int64_t>(p.groups) * p.tiles;
+  const int per_sm = p.nt == 8 ? gemv_ctas_per_sm_t<8>() : gemv_ctas_per_sm_t<16>();
+  const int64_t resident = static_cast<int64_t>(per_sm) * device_sm_count();
+  p.ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(resident, p.n_items)));
+  p.ws = p.groups > 1 ? round256(static_cast<size_t>(p.groups) * out * M * 4) : 0;
   return p;
 }
 
-size_t gemv_ws(int64_t M, int64_t in, int64_t out) {
-  const GemvPlan p = gemv_plan(in, out);
-  return round256(static_cast<size_t>(p.ctas) * p.local_tiles * M * qnf4::kGvRows * 4);
-}
+size_t gemv_ws(int64_t M, int64_t in, int64_t out) { return gemv_plan(M, in, out).ws; }
 
 // K splits of the row-wise rank-r product: enough CTAs (64 rows x one
 // 64-wide rank chunk x one K range each) to keep ~2 per SM streaming, with at
@@ -314,24 +343,62 @@ int col_chunk_tokens(int64_t M) {
   return static_cast<int>(cdiv(cdiv(M, chunks), 32) * 32);
 }
 
+// LoRA rank as the kernels take it: a multiple of 8 (16-byte rows).
+constexpr int padded_rank(int r) { return (r + 7) / 8 * 8; }
+
+// Zero-padded copies used when r % 8 != 0 (pad.cuh): A [rp, in], B [out, rp],
+// us [M, rp], and in the backward dA [rp, in], dB [out, rp] (fp32).
+struct PadWs {
+  size_t a_off, b_off, us_off, da_off, db_off, total;
+};
+
+PadWs pad_ws(int64_t M, int64_t in, int64_t out, int r, bool backward, size_t base) {
+  PadWs w{};
+  if (r % 8 == 0) {
+    w.total = base;
+    return w;
+  }
+  const size_t rp = static_cast<size_t>(padded_rank(r));
+  w.a_off = base;
+  w.b_off = w.a_off + round256(rp * in * 2);
+  w.us_off = w.b_off + round256(out * rp * 2);
+  w.da_off = w.us_off + round256(M * rp * 2);
+  w.db_off = w.da_off + (backward ? round256(rp * in * 4) : 0);
+  w.total = w.db_off + (backward ? round256(out * rp * 4) : 0);
+  return w;
+}
+
 size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
-  (void)r;
-  return M <= 16 ? gemv_ws(M, in, out) : 0;
+  return pad_ws(M, in, out, r, false, M <= 16 ? gemv_ws(M, in, out) : 0).total;
 }
 
 size_t fwd_dropout_ws(int64_t M, int64_t in, int64_t out, int r) { return fwd_ws(M, in, out, r); }
 
 struct BwdWs {
-  size_t du_off, total;
+  size_t du_off;
+  PadWs pad;
+  size_t total;
 };
 
 BwdWs bwd_ws(int64_t M, int64_t in, int64_t out, int r) {
-  (void)in;
-  (void)out;
   BwdWs w{};
   w.du_off = 0;
-  w.total = round256(static_cast<size_t>(M) * r * 2);
+  w.pad = pad_ws(M, in, out, r, true, round256(static_cast<size_t>(M) * padded_rank(r) * 2));
+  w.total = w.pad.total;
   return w;
+}
+
+template <typename T>
+int launch_copy_pad(const T* src, int64_t src_rows, int64_t src_cols, T* dst, int64_t dst_rows, int64_t dst_cols,
+                    cudaStream_t st) {
+  const int64_t n = dst_rows * dst_cols;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), device_sm_count() * 8)));
+  {
+    LaunchTimer lt_("lora_pad", st);
+    qnf4::copy_pad_kernel<T><<<grid, 256, 0, st>>>(src, src_rows, src_cols, dst, dst_rows, dst_cols);
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
 }
 
 // ------------------------------------------------------------------ launches
@@ -536,12 +603,104 @@ int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int 
   return QLORA_OK;
 }
 
+// ------------------------------------------------------------------ tcgen05 rank-r products
+int lr_n_alloc(int N) {
+  int a = 32;
+  while (a < N) a *= 2;
+  return a;
+}
+
+// Contraction split over a cluster: the smallest power of two (<= 8) that
+// gives at least one CTA per SM, keeping at least 2 stages per split.
+int lr_splits(int64_t tiles, int64_t stages) {
+  int ks = 1;
+  while (ks < 8 && tiles * ks < device_sm_count() && stages / (2 * ks) >= 2) ks *= 2;
+  return ks;
+}
+
+template <bool kCol, bool kBMN>
+int launch_lora_umma(const CUtensorMap (&tm)[4], const qnf4::LrArgs& a, int ks, unsigned grid_x, const char* name,
+                     cudaStream_t st) {
+  auto kern = qnf4::lora_umma_kernel<kCol, kBMN>;
+  const int smem = qnf4::lr_smem_bytes(a.N, kBMN);
+  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), smem));
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid_x, static_cast<unsigned>(ks), 1);
+  cfg.blockDim = dim3(qnf4::kLrThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(ks);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ks > 1 ? 1 : 0;
+  {
+    LaunchTimer lt_(name, st);
+    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, tm[0], tm[1], tm[2], tm[3], a));
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return QLORA_OK;
+}
+
+// Row form: out[M, r] = bf16(scale * act[M, K] . w^T), w given as [r, K]
+// (w_n_major = false: A of the forward) or as [K, r] (true: B of du).
+int launch_lora_row(const uint16_t* act, const uint16_t* w, uint16_t* out, int64_t M, int64_t K, int r, float scale,
+                    bool w_n_major, const char* name, cudaStream_t st) {
+  qnf4::LrArgs a{};
+  a.r = r;
+  a.N = (r + 15) / 16 * 16;
+  a.n_alloc = lr_n_alloc(a.N);
+  a.K = static_cast<int>(K);
+  a.p[0] = qnf4::LrProblem{out, static_cast<int>(M), static_cast<int>(cdiv(M, 128)), 0, scale};
+  a.p[1] = a.p[0];
+  a.timeout_ns = g_timeout_ns.load();
+  const int64_t stages = cdiv(K, 64);
+  const int ks = lr_splits(a.p[0].tiles, stages);
+  a.stages_per_split = static_cast<int>(cdiv(stages, ks));
+  CUtensorMap tm[4];
+  if (!make_tmap_bf16(&tm[0], act, M, K, 128)) return QLORA_ERR_CUDA;
+  const bool ok = w_n_major ? make_tmap_bf16(&tm[1], w, K, r, 64) : make_tmap_bf16(&tm[1], w, r, K, a.N);
+  if (!ok) return QLORA_ERR_CUDA;
+  tm[2] = tm[0];
+  tm[3] = tm[1];
+  const unsigned gx = static_cast<unsigned>(a.p[0].tiles);
+  return w_n_major ? launch_lora_umma<false, true>(tm, a, ks, gx, name, st)
+                   : launch_lora_umma<false, false>(tm, a, ks, gx, name, st);
+}
+
+// Col form, both adapter gradients in one launch: dB [out, r] = dh^T us and
+// dA [r, in] = (x^T du)^T * dA_scale.
+int launch_lora_col(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
+                    int64_t in, int64_t out, int r, float* dB, float* dA, float dA_scale, cudaStream_t st) {
+  qnf4::LrArgs a{};
+  a.r = r;
+  a.N = (r + 15) / 16 * 16;
+  a.n_alloc = lr_n_alloc(a.N);
+  a.K = static_cast<int>(M);
+  a.p[0] = qnf4::LrProblem{dB, static_cast<int>(out), static_cast<int>(cdiv(out, 128)), 0, 1.f};
+  a.p[1] = qnf4::LrProblem{dA, static_cast<int>(in), static_cast<int>(cdiv(in, 128)), 1, dA_scale};
+  a.timeout_ns = g_timeout_ns.load();
+  const int64_t stages = cdiv(M, 64);
+  const int ks = lr_splits(a.p[0].tiles + a.p[1].tiles, stages);
+  a.stages_per_split = static_cast<int>(cdiv(stages, ks));
+  CUtensorMap tm[4];
+  if (!make_tmap_bf16(&tm[0], dh, M, out, 64) || !make_tmap_bf16(&tm[1], us, M, r, 64) ||
+      !make_tmap_bf16(&tm[2], x, M, in, 64) || !make_tmap_bf16(&tm[3], du, M, r, 64))
+    return QLORA_ERR_CUDA;
+  return launch_lora_umma<true, true>(tm, a, ks, static_cast<unsigned>(a.p[0].tiles + a.p[1].tiles), "lora_colwise",
+                                      st);
+}
+
 // out[M, R] = bf16(scale * (act[M, K] * k) . W^T) with W given as [R, K] (kKR =
 // false) or as [K, R] (kKR = true); k the keep mask of LoRA dropout, or all
-// ones when keep is null.
+// ones when keep is null (then the tcgen05 kernel runs).
 template <bool kKR>
 int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_t M, int64_t K, int R, float scale,
                    cudaStream_t st, const uint8_t* keep = nullptr) {
+  if (keep == nullptr)
+    return launch_lora_row(act, W, out, M, K, R, scale, kKR, kKR ? "lora_rowwise_du" : "lora_rowwise", st);
   const int ks = rowwise_splits(M, K, R);
   if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
   if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
@@ -554,6 +713,7 @@ int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_
 int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
                       int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st, float dA_scale = 1.f,
                       const uint8_t* keep = nullptr) {
+  if (keep == nullptr) return launch_lora_col(dh, us, x, du, M, in, out, R, dB, dA, dA_scale, st);
   const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0, 1.f, nullptr};
   const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale, keep};   // dA^T = (x * k)^T du
   const int smem = qnf4::kColStages * qnf4::kColStageBytes;
@@ -590,7 +750,7 @@ bool weight_ok(const qlora_nf4_weight* w) {
 int check_linear_shapes(int64_t M, const qlora_nf4_weight* w, int r) {
   if (M < 1 || w->rows < 64 || w->cols < 64) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (w->cols % 64 != 0 || w->rows % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (r < 8 || r > 256 || r % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (r < 1 || r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (M > (1ll << 31) - 1024 || w->rows > (1ll << 30) || w->cols > (1ll << 30))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
   if (w->rows * w->cols > (1ll << 40)) return QLORA_ERR_UNSUPPORTED_SHAPE;
@@ -607,43 +767,126 @@ int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlo
   int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s_lora, st, keep);   // us = bf16(s (x k) A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
-    const GemvPlan p = gemv_plan(in, out);
+    const GemvPlan p = gemv_plan(M, in, out);
     qnf4::GemvArgs g{};
     g.q8 = w->q8;
     g.step2 = w->step2;
     g.mean = w->mean;
+    g.x = x;
+    g.us = us_out;
+    g.B = B;
+    g.h = h;
     g.part = static_cast<float*>(workspace);
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
-    g.n_st = p.n_st;
-    g.n_units = p.n_units;
-    g.local_tiles = p.local_tiles;
+    g.r = r;
+    g.n_slices = p.n_slices;
+    g.groups = p.groups;
+    g.tiles = p.tiles;
+    g.n_items = p.n_items;
     g.timeout_ns = g_timeout_ns.load();
     g.L = tables().L;
-    CUtensorMap tm_codes, tm_x;
-    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)) ||
-        !make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(M), static_cast<uint64_t>(in), M > 8 ? 16 : 8))
+    CUtensorMap tm_codes;
+    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)))
       return QLORA_ERR_CUDA;
     {
       LaunchTimer lt_("gemv", st);
-      const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
-      auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
-                         : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
-      QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), qnf4::kGvSmem));
-      kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
+      if (p.nt == 8) {
+        const GemvKernel<8> k = gemv_kernel_for<8>();
+        QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(k), qnf4::GvCfg<8>::SMEM));
+        k<<<p.ctas, qnf4::GvCfg<8>::THREADS, qnf4::GvCfg<8>::SMEM, st>>>(tm_codes, g);
+      } else {
+        const GemvKernel<16> k = gemv_kernel_for<16>();
+        QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(k), qnf4::GvCfg<16>::SMEM));
+        k<<<p.ctas, qnf4::GvCfg<16>::THREADS, qnf4::GvCfg<16>::SMEM, st>>>(tm_codes, g);
+      }
     }
     QLORA_CUDA_TRY(cudaGetLastError());
-    const int64_t n_el = M * out;
-    {
+    if (p.groups > 1) {
+      const int64_t n_el = M * out;
       LaunchTimer lt_("gemv_finalize", st);
       qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
-          g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
+          g.part, p.groups, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
+      QLORA_CUDA_TRY(cudaGetLastError());
     }
-    QLORA_CUDA_TRY(cudaGetLastError());
     return QLORA_OK;
   }
   return launch_gemm(false, w, x, M, in, us_out, B, r, h, out, st);  // h = [x|us] [W0|B]^T
+}
+
+// Forward at any rank: r % 8 == 0 runs linear_fwd_impl directly; otherwise
+// on zero-padded copies of A and B at rp = r rounded up to 8, with us
+// computed at rp in the workspace and copied back to [M, r].
+int linear_fwd_any_rank(const uint16_t* x, const uint8_t* keep, int64_t M, const qlora_nf4_weight* w,
+                        const uint16_t* A, const uint16_t* B, int r, float s_lora, uint16_t* h, uint16_t* us_out,
+                        void* workspace, cudaStream_t st) {
+  if (r % 8 == 0) return linear_fwd_impl(x, keep, M, w, A, B, r, s_lora, h, us_out, workspace, st);
+  const int64_t in = w->cols, out = w->rows;
+  const int rp = padded_rank(r);
+  const PadWs pw = pad_ws(M, in, out, r, false, M <= 16 ? gemv_ws(M, in, out) : 0);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* A_p = reinterpret_cast<uint16_t*>(base + pw.a_off);
+  uint16_t* B_p = reinterpret_cast<uint16_t*>(base + pw.b_off);
+  uint16_t* us_p = reinterpret_cast<uint16_t*>(base + pw.us_off);
+  int rc = launch_copy_pad(A, r, in, A_p, rp, in, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(B, out, r, B_p, out, rp, st);
+  if (rc == QLORA_OK) rc = linear_fwd_impl(x, keep, M, w, A_p, B_p, rp, s_lora, h, us_p, workspace, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(us_p, M, rp, us_out, M, r, st);
+  return rc;
+}
+
+// Backward after validation, rank a multiple of 8: du = bf16(s dh B) into
+// `du`, then dx (with its rank-r tail, or without it plus the masked term
+// when keep is given) and dB, dA.
+int linear_bwd_impl(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
+                    const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float s,
+                    const uint8_t* keep, float inv_keep, uint16_t* dx, float* dA, float* dB, uint16_t* du,
+                    cudaStream_t st) {
+  const int64_t in = w->cols, out = w->rows;
+  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                           // du = bf16(s dh B)
+  if (rc != QLORA_OK) return rc;
+  if (keep == nullptr) {
+    rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
+    if (rc != QLORA_OK) return rc;
+    return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st);                  // dB, dA
+  }
+  rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);                // dx = dh W0
+  if (rc != QLORA_OK) return rc;
+  {
+    const int64_t units = cdiv(M, qnf4::kDxRows) * (in / 8);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+    LaunchTimer lt_("dropout_dx", st);
+    qnf4::dropout_dx_kernel<<<grid, 256, 0, st>>>(dx, du, A, keep, M, in, r, inv_keep);  // + (du A) k/(1-p)
+  }
+  QLORA_CUDA_TRY(cudaGetLastError());
+  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st, inv_keep, keep);     // dB, dA
+}
+
+// Backward at any rank (the padded copies as in linear_fwd_any_rank; dA and
+// dB are computed at rp and copied back to [r, in] and [out, r]).
+int linear_bwd_any_rank(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
+                        const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float s,
+                        const uint8_t* keep, float inv_keep, uint16_t* dx, float* dA, float* dB, void* workspace,
+                        cudaStream_t st) {
+  const int64_t in = w->cols, out = w->rows;
+  const BwdWs ws = bwd_ws(M, in, out, r);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
+  if (r % 8 == 0) return linear_bwd_impl(dh, x, us, M, w, A, B, r, s, keep, inv_keep, dx, dA, dB, du, st);
+  const int rp = padded_rank(r);
+  uint16_t* A_p = reinterpret_cast<uint16_t*>(base + ws.pad.a_off);
+  uint16_t* B_p = reinterpret_cast<uint16_t*>(base + ws.pad.b_off);
+  uint16_t* us_p = reinterpret_cast<uint16_t*>(base + ws.pad.us_off);
+  float* dA_p = reinterpret_cast<float*>(base + ws.pad.da_off);
+  float* dB_p = reinterpret_cast<float*>(base + ws.pad.db_off);
+  int rc = launch_copy_pad(A, r, in, A_p, rp, in, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(B, out, r, B_p, out, rp, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(us, M, r, us_p, M, rp, st);
+  if (rc == QLORA_OK) rc = linear_bwd_impl(dh, x, us_p, M, w, A_p, B_p, rp, s, keep, inv_keep, dx, dA_p, dB_p, du, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(dA_p, rp, in, dA, r, in, st);
+  if (rc == QLORA_OK) rc = launch_copy_pad(dB_p, out, rp, dB, out, r, st);
+  return rc;
 }
 
 int check_fwd_args(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B,
@@ -869,8 +1112,8 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, co
   const size_t need = fwd_ws(M, w->cols, w->rows, r);
   if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
     return QLORA_ERR_WORKSPACE;
-  return linear_fwd_impl(x, nullptr, M, w, A, B, r, alpha / static_cast<float>(r), h, us_out, workspace,
-                         static_cast<cudaStream_t>(stream));
+  return linear_fwd_any_rank(x, nullptr, M, w, A, B, r, alpha / static_cast<float>(r), h, us_out, workspace,
+                             static_cast<cudaStream_t>(stream));
 }
 
 int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weight* w, const uint16_t* A,
@@ -885,7 +1128,7 @@ int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weigh
     return QLORA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float s_lora = (alpha / static_cast<float>(r)) / (1.f - p);
-  return linear_fwd_impl(x, keep_bits, M, w, A, B, r, s_lora, h, us_out, workspace, st);
+  return linear_fwd_any_rank(x, keep_bits, M, w, A, B, r, s_lora, h, us_out, workspace, st);
 }
 
 int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
@@ -898,19 +1141,10 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, 
   if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
   const int sc = check_linear_shapes(M, w, r);
   if (sc != QLORA_OK) return sc;
-  const int64_t in = w->cols, out = w->rows;
-  const BwdWs ws = bwd_ws(M, in, out, r);
+  const BwdWs ws = bwd_ws(M, w->cols, w->rows, r);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
-  const float s = alpha / static_cast<float>(r);
-
-  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                         // du = bf16(s dh B)
-  if (rc != QLORA_OK) return rc;
-  rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
-  if (rc != QLORA_OK) return rc;
-  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st);                // dB, dA
+  return linear_bwd_any_rank(dh, x, us, M, w, A, B, r, alpha / static_cast<float>(r), nullptr, 1.f, dx, dA, dB,
+                             workspace, static_cast<cudaStream_t>(stream));
 }
 
 int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
@@ -925,27 +1159,10 @@ int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16
   int sc = check_linear_shapes(M, w, r);
   if (sc != QLORA_OK) return sc;
   if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
-  const int64_t in = w->cols, out = w->rows;
-  const BwdWs ws = bwd_ws(M, in, out, r);
+  const BwdWs ws = bwd_ws(M, w->cols, w->rows, r);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint16_t* du = reinterpret_cast<uint16_t*>(base + ws.du_off);
-  const float s = alpha / static_cast<float>(r);
-  const float inv_keep = 1.f / (1.f - p);
-
-  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                          // du = bf16(s dh B)
-  if (rc != QLORA_OK) return rc;
-  rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);              // dx = dh W0
-  if (rc != QLORA_OK) return rc;
-  {
-    const int64_t units = cdiv(M, qnf4::kDxRows) * (in / 8);
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
-    LaunchTimer lt_("dropout_dx", st);
-    qnf4::dropout_dx_kernel<<<grid, 256, 0, st>>>(dx, du, A, keep_bits, M, in, r, inv_keep);  // + (du A) k/(1-p)
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st, inv_keep, keep_bits);   // dB, dA
+  return linear_bwd_any_rank(dh, x, us, M, w, A, B, r, alpha / static_cast<float>(r), keep_bits, 1.f / (1.f - p), dx,
+                             dA, dB, workspace, static_cast<cudaStream_t>(stream));
 }
 
 int qlora_last_device_status(void* stream) {

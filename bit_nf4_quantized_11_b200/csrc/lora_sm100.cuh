@@ -1,0 +1,283 @@
+// lora_sm100.cuh -- the rank-r contractions of the QLoRA layer on tcgen05.
+//
+// ("QLoRA", llm-compass, 方法与公式: h = dequant(W0) x + (alpha/r) B A x, with
+// gradients for A and B only; aigrafen.se, opening paragraph.)
+//
+// All four products have one dimension equal to the LoRA rank r and stream a
+// token-sized operand from HBM once, so they are bound by that read.  Each is
+// one tcgen05 tile product D[128 x N] (+)= A . B^T with N = r rounded up to a
+// multiple of 16 (at most 256), fp32 accumulation in tensor memory, both
+// operands staged by TMA (128-byte swizzle) in a ring of shared-memory stages:
+//
+//   row form  out[m][j] = bf16(scale * sum_k act[m][k] * w(j, k))
+//     us = bf16(s x A^T)   act = x  [M, in]  (K-major), w = A [r, in]  (K-major)
+//     du = bf16(s dh B)    act = dh [M, out] (K-major), w = B [out, r] (N-major)
+//   col form  D[f][j] = scale * sum_m act[m][f] * u[m][j]
+//     dB   = dh^T us       act = dh [M, out] (MN-major), u = us [M, r] (N-major)
+//     dA^T = x^T du        act = x  [M, in]  (MN-major), u = du [M, r] (N-major)
+//
+// The tile rows are tokens (row form) or features (col form); the
+// contraction (K of the row form, the tokens of the col form) is split over
+// the CTAs of a thread-block cluster (at most 8).  Each CTA moves its fp32
+// partial tile from tensor memory to its own shared memory; then every CTA
+// adds up its share of the tile's rows over distributed shared memory,
+// partials in rank order (deterministic), and stores it.
+//
+// Roles (128 threads): warp 0 lane 0 issues the TMA loads, warp 1 allocates
+// tensor memory and its lane 0 issues the MMAs; afterwards the four warps
+// read the accumulator (warp w owns rows 32 w .. 32 w + 31, its TMEM lanes).
+// Every wait is bounded: on timeout the CTA sets the device error flag,
+// issues nothing more, waits (bounded) for what it issued and exits.
+// No TMA multicast is used.
+#pragma once
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+constexpr int kLrThreads = 128;
+constexpr int kLrStages = 4;
+constexpr int kLrTileRows = 128;
+constexpr int kLrAStage = kLrTileRows * 64 * 2;           // 16 KB: 128 rows x 64 k (or two 64-wide MN atoms)
+
+// Instruction descriptor, kind::f16 with bf16 A and B, fp32 D; either
+// operand K-major or MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+struct LrProblem {
+  void* out;             // row form: bf16 [rows, r]; col form: fp32 [rows, r] or, transposed, [r, rows]
+  int rows;              // tokens (row form) or features (col form)
+  int tiles;             // ceil(rows / 128)
+  int transpose_out;     // col form: write D^T (dA [r, in])
+  float scale;
+};
+
+struct LrArgs {
+  LrProblem p[2];        // blockIdx.x < p[0].tiles: problem 0, else problem 1
+  int K;                 // contraction length (row form: features; col form: tokens)
+  int r;                 // rank
+  int N;                 // r rounded up to 16
+  int n_alloc;           // TMEM columns (power of two >= 32, >= N)
+  int stages_per_split;  // 64-wide contraction stages per CTA of the cluster
+  uint64_t timeout_ns;
+};
+
+// Shared bytes of one stage of the B operand (N rows x 64 k K-major, or
+// ceil(N / 64) atoms of 64 n x 64 k) and of the fp32 partial tile (padded rows).
+__host__ __device__ constexpr int lr_b_stage(int N, bool b_mn_major) {
+  return b_mn_major ? ((N + 63) / 64) * 8192 : ((N * 128 + 1023) / 1024) * 1024;
+}
+__host__ __device__ constexpr int lr_partial_pitch(int N) { return N * 4 + 16; }
+__host__ __device__ constexpr int lr_smem_bytes(int N, bool b_mn_major) {
+  const int ring = kLrStages * (kLrAStage + lr_b_stage(N, b_mn_major));
+  const int part = kLrTileRows * lr_partial_pitch(N);
+  return (ring > part ? ring : part) + 256 + 1024;
+}
+
+// kCol: col form (A MN-major, output fp32); otherwise row form (A K-major,
+// output bf16).  kBMN: B operand N-major.
+template <bool kCol, bool kBMN>
+__global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
+    const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
+    const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1, const LrArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  const int N = args.N;
+  const int b_stage = lr_b_stage(N, kBMN);
+  const int ring_bytes = kLrStages * (kLrAStage + b_stage);
+  const int part_bytes = kLrTileRows * lr_partial_pitch(N);
+  uint8_t* a_ring = smem;
+  uint8_t* b_ring = smem + kLrStages * kLrAStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (ring_bytes > part_bytes ? ring_bytes : part_bytes));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kLrStages;
+  uint64_t* acc_full = bars + 2 * kLrStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int prob = static_cast<int>(blockIdx.x) < args.p[0].tiles ? 0 : 1;
+  // fields of this CTA's problem (selected, not indexed: no local-memory copy)
+  void* const p_out = prob == 0 ? args.p[0].out : args.p[1].out;
+  const int p_rows = prob == 0 ? args.p[0].rows : args.p[1].rows;
+  const bool p_transpose = (prob == 0 ? args.p[0].transpose_out : args.p[1].transpose_out) != 0;
+  const float p_scale = prob == 0 ? args.p[0].scale : args.p[1].scale;
+  const int tile = prob == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - args.p[0].tiles;
+  const CUtensorMap* tm_a = prob == 0 ? &tm_a0 : &tm_a1;
+  const CUtensorMap* tm_b = prob == 0 ? &tm_b0 : &tm_b1;
+  const int row0 = tile * kLrTileRows;
+  const int ks = static_cast<int>(gridDim.y);
+  const int split = static_cast<int>(blockIdx.y);
+  const int n_stages_total = (args.K + 63) / 64;
+  const int st_begin = split * args.stages_per_split;
+  const int st_end = min(n_stages_total, st_begin + args.stages_per_split);
+  const int n_iter = max(0, st_end - st_begin);
+  const uint64_t tmo = args.timeout_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLrStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, static_cast<uint32_t>(args.n_alloc));
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_holder;
+
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    if (*abort_flag) return;
+    if (!mbar_wait_bounded(bar, parity, tmo)) {
+      *abort_flag = 1;
+      raise_device_error(1);
+    }
+  };
+
+  const uint32_t stage_tx = static_cast<uint32_t>(kLrAStage + b_stage);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(tm_a);
+      tma_prefetch_desc(tm_b);
+      int issued = 0;
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % kLrStages;
+        wait(empty + s, ((it / kLrStages) & 1u) ^ 1u);
+        if (*abort_flag) break;
+        mbar_arrive_expect_tx(full + s, stage_tx);
+        const uint32_t a_dst = smem_u32(a_ring + s * kLrAStage);
+        const uint32_t b_dst = smem_u32(b_ring + s * b_stage);
+        const int k0 = (st_begin + it) * 64;
+        if (!kCol) {
+          tma_load_2d(a_dst, tm_a, full + s, k0, row0);                      // [128 rows x 64 k]
+        } else {
+          tma_load_2d(a_dst, tm_a, full + s, row0, k0);                      // two atoms of 64 features x 64 tokens
+          tma_load_2d(a_dst + 8192, tm_a, full + s, row0 + 64, k0);
+        }
+        if (!kBMN) {
+          tma_load_2d(b_dst, tm_b, full + s, k0, 0);                         // [N rows x 64 k]
+        } else {
+          for (int a = 0; a * 64 < N; ++a) tma_load_2d(b_dst + a * 8192, tm_b, full + s, a * 64, k0);
+        }
+        ++issued;
+      }
+      // only the last kLrStages issued stages can still be in flight
+      for (int it = issued > kLrStages ? issued - kLrStages : 0; it < issued; ++it)
+        mbar_wait_bounded(full + (it % kLrStages), (it / kLrStages) & 1u, tmo);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t idesc = umma_idesc_bf16_ab(kLrTileRows, N, kCol, kBMN);
+      for (int it = 0; it < n_iter; ++it) {
+        const int s = it % kLrStages;
+        wait(full + s, (it / kLrStages) & 1u);
+        if (*abort_flag) break;
+        tc_fence_after_sync();
+        const uint32_t a_base = smem_u32(a_ring + s * kLrAStage);
+        const uint32_t b_base = smem_u32(b_ring + s * b_stage);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t adesc = kCol ? umma_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                      : umma_desc_sw128(a_base + kk * 32, 16, 1024);
+          const uint64_t bdesc = kBMN ? umma_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                      : umma_desc_sw128(b_base + kk * 32, 16, 1024);
+          umma_bf16_ss(tmem_base, adesc, bdesc, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(empty + s);
+      }
+      umma_commit(acc_full);
+      mbar_wait_bounded(acc_full, 0, tmo);
+    }
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  // Wait for the accumulator (the commit arrives even when no stage was
+  // issued; an empty split leaves zeros).
+  __syncwarp();
+  wait(acc_full, 0);
+  tc_fence_after_sync();
+  const int row = warp * 32 + lane;                                  // this thread's TMEM lane / tile row
+  const int pitch = lr_partial_pitch(N);
+  uint8_t* part = smem;                                              // the ring is free once acc_full completed
+  __syncthreads();                                                   // every stage read by the tensor cores
+  for (int c0 = 0; c0 < N; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
+    tmem_ld_wait();
+    if (n_iter == 0) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0u;                        // nothing accumulated
+    }
+    const uint32_t dst = smem_u32(part + row * pitch + c0 * 4);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (c0 + 4 * i < N) sts_v4(dst + 16 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (ks > 1) cluster_sync_all();                                    // every CTA's partial is in place
+
+  // this CTA's share of the tile's rows, summed over the cluster in rank order
+  const int share = kLrTileRows / ks;
+  const int r_lo = split * share;
+  const int n4 = args.r / 4;                                         // float4 groups of the rank
+  for (int e = threadIdx.x; e < share * n4; e += kLrThreads) {
+    int rr, c4;
+    if (kCol && p_transpose) {                                   // rows fastest: coalesced dA^T stores
+      rr = r_lo + e % share;
+      c4 = e / share;
+    } else {
+      rr = r_lo + e / n4;
+      c4 = e % n4;
+    }
+    const int grow = row0 + rr;
+    const uint32_t addr = smem_u32(part + rr * pitch + c4 * 16);
+    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int rk = 0; rk < ks; ++rk) {
+      float4 u;
+      if (ks == 1) {
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(u.x), "=f"(u.y), "=f"(u.z), "=f"(u.w)
+                     : "r"(addr) : "memory");
+      } else {
+        asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(u.x), "=f"(u.y), "=f"(u.z), "=f"(u.w) : "r"(mapa_shared(addr, rk)) : "memory");
+      }
+      t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+    }
+    if (grow >= p_rows) continue;
+    const float sc = p_scale;
+    if (!kCol) {
+      uint16_t* o = static_cast<uint16_t*>(p_out) + static_cast<int64_t>(grow) * args.r + c4 * 4;
+      *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2_rn(t.x * sc, t.y * sc), pack_bf16x2_rn(t.z * sc, t.w * sc));
+    } else if (!p_transpose) {
+      float* o = static_cast<float*>(p_out) + static_cast<int64_t>(grow) * args.r + c4 * 4;
+      *reinterpret_cast<float4*>(o) = make_float4(t.x * sc, t.y * sc, t.z * sc, t.w * sc);
+    } else {
+      float* o = static_cast<float*>(p_out);
+      const int64_t ld = p_rows;
+      o[static_cast<int64_t>(c4 * 4 + 0) * ld + grow] = t.x * sc;
+      o[static_cast<int64_t>(c4 * 4 + 1) * ld + grow] = t.y * sc;
+      o[static_cast<int64_t>(c4 * 4 + 2) * ld + grow] = t.z * sc;
+      o[static_cast<int64_t>(c4 * 4 + 3) * ld + grow] = t.w * sc;
+    }
+  }
+  if (ks > 1) cluster_sync_all();                                    // no CTA leaves while others read it
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, static_cast<uint32_t>(args.n_alloc));
+  }
+}
+
+}  // namespace qnf4

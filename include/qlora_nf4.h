@@ -251,7 +251,12 @@ int qlora_dequantize_nf4(const qlora_nf4_weight* w, uint16_t* W_out, void* strea
  * us_out  device bf16 [M, r] (written): the scaled LoRA activation, kept for
  *         the backward.
  * workspace: qlora_workspace_size(QLORA_OP_LINEAR_FWD, M, in, out, r) bytes.
- * Size rules: M >= 1; in % 64 == 0; out % 64 == 0; r % 8 == 0, 8 <= r <= 256.
+ * Size rules: M >= 1; in % 64 == 0; out % 64 == 0; 1 <= r <= 256 ("QLoRA",
+ * llm-compass, 调参与实践经验: the rank is a free hyper-parameter, 16-64
+ * typical).  The kernels work on rank multiples of 8 (16-byte rows of the
+ * [tokens, r] and [out, r] tensors); for any other r the call runs at r
+ * rounded up to 8 on zero-padded copies of A, B and us held in the
+ * workspace (the padding adds exactly zero) and copies us back to [M, r].
  */
 int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w,
                      const uint16_t* A, const uint16_t* B, int r, float alpha,
@@ -274,7 +279,9 @@ int qlora_linear_fwd(const uint16_t* x, int64_t M, const qlora_nf4_weight* w,
  * dx device bf16 [M, in]; dA device fp32 [r, in]; dB device fp32 [out, r]
  * (all written, not accumulated).
  * workspace: qlora_workspace_size(QLORA_OP_LINEAR_BWD, M, in, out, r) bytes.
- * Size rules as for qlora_linear_fwd.
+ * Size rules as for qlora_linear_fwd; for r % 8 != 0 the padded copies of A,
+ * B, us and of dA, dB (fp32) live in the workspace and dA, dB are copied back
+ * to [r, in] and [out, r].
  */
 int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us,
                      int64_t M, const qlora_nf4_weight* w,

@@ -143,18 +143,23 @@ def test_linear_argument_errors(lib):
     assert fwd(None, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == EINVAL
     assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE + 8, None, 0, None) == EINVAL
     assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, float("nan"), FAKE, FAKE, None, 0, None) == EINVAL
-    # shape rules: r multiple of 8 in [8, 256], M >= 1, in/out multiples of 64
-    for r in (0, 4, 12, 264):
+    # shape rules: 1 <= r <= 256, M >= 1, in/out multiples of 64
+    for r in (0, -3, 257, 264):
         assert fwd(FAKE, 64, wb, FAKE, FAKE, r, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
+    # a rank that is not a multiple of 8 runs on padded copies in the workspace
+    for r in (1, 4, 12):
+        assert fwd(FAKE, 64, wb, FAKE, FAKE, r, 16.0, FAKE, FAKE, None, 0, None) == EWS
+        assert lib.qlora_workspace_size(2, 64, 128, 128, r) > 0
     assert fwd(FAKE, 0, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
     w2 = _weight(96, 128)
     assert fwd(FAKE, 64, ctypes.byref(w2), FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == ESHAPE
-    # GEMV path needs a workspace
-    assert fwd(FAKE, 4, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == EWS
+    # the GEMV path needs a workspace when K spans several groups of slices
+    w3 = _weight(128, 8192)
+    assert fwd(FAKE, 4, ctypes.byref(w3), FAKE, FAKE, 8, 16.0, FAKE, FAKE, None, 0, None) == EWS
     # backward always needs one
     assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, FAKE, None, 0, None) == EWS
     assert bwd(FAKE, FAKE, None, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == EINVAL
-    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 9, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ESHAPE
+    assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 257, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ESHAPE
 
 
 def test_dropout_argument_errors(lib):
@@ -166,8 +171,10 @@ def test_dropout_argument_errors(lib):
     assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE + 2, 0.05, FAKE, FAKE, None, 0, None) == EINVAL
     assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, 1.0, FAKE, FAKE, None, 0, None) == EINVAL
     assert fwd(FAKE, 64, wb, FAKE, FAKE, 8, 16.0, FAKE, -0.1, FAKE, FAKE, None, 0, None) == EINVAL
-    # the few-token forward needs a workspace; the large-M one none (the mask is applied in place of a copy)
-    assert fwd(FAKE, 4, wb, FAKE, FAKE, 8, 16.0, FAKE, 0.05, FAKE, FAKE, None, 0, None) == EWS
+    # the few-token forward needs a workspace when K spans several slice groups;
+    # the large-M one none (the mask is applied in place of a copy)
+    w3 = _weight(128, 8192)
+    assert fwd(FAKE, 4, ctypes.byref(w3), FAKE, FAKE, 8, 16.0, FAKE, 0.05, FAKE, FAKE, None, 0, None) == EWS
     assert q.workspace_size(q.OP_LINEAR_FWD_DROPOUT, 64, 128, 128, 8) == 0
     assert q.workspace_size(q.OP_LINEAR_BWD_DROPOUT, 64, 128, 128, 8) == q.workspace_size(q.OP_LINEAR_BWD, 64, 128,
                                                                                            128, 8)

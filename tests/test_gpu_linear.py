@@ -93,6 +93,17 @@ def test_largest_rank(cuda_lib, M, n_in, n_out, alpha):
     _run(cuda_lib, M, n_in, n_out, 256, alpha, seed=M + 7)
 
 
+@pytest.mark.parametrize("r", [1, 4, 12, 20])
+@pytest.mark.parametrize("M,n_in,n_out", [
+    (520, 512, 640),      # CTA-pair GEMM
+    (100, 256, 320),      # one-CTA GEMM
+    (5, 576, 384),        # few-token GEMV forward, GEMM backward
+])
+def test_rank_not_multiple_of_8(cuda_lib, M, n_in, n_out, r):
+    # any rank 1 <= r <= 256: the layer runs on zero-padded copies at r rounded up to 8
+    _run(cuda_lib, M, n_in, n_out, r, 2.0 * r, seed=M + r)
+
+
 @pytest.mark.parametrize("M,n_in,n_out", [(4096, 512, 2560), (4096, 2560, 512)])
 def test_two_waves_short_k(cuda_lib, M, n_in, n_out):
     # 80 output tiles of 512 x 256: more tiles than co-resident CTA pairs, so
