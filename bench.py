@@ -57,7 +57,8 @@ def parse():
     ap.add_argument("--no-components", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout", "layer_step"],
+    ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout", "layer_step",
+                                       "q_proj_steps"],
                     default=None,
                     help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
@@ -670,7 +671,20 @@ def comp_dropout(q, dev, peaks, n=50):
         b.record()
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / n
-        res[label] = {"ms": ms, "TFLOP/s": workloads.fwd_bwd_flops(M, n_in, n_out, r) / (ms * 1e-3) / 1e12}
+        q.timing_reset()                            # the same steps again, kernels bracketed by events
+        q.timing_enable(True)
+        for _ in range(n):
+            _, us = fwd()
+            bwd(us)
+        torch.cuda.synchronize()
+        q.timing_enable(False)
+        kern = {}
+        for name in q.KERNEL_NAMES:
+            t, k = q.timing_collect(name)
+            if k:
+                kern[name] = 1e3 * t / n
+        res[label] = {"ms": ms, "TFLOP/s": workloads.fwd_bwd_flops(M, n_in, n_out, r) / (ms * 1e-3) / 1e12,
+                      "kernel_us_per_step": kern}
     res["dropout_overhead"] = res["dropout_p0.05"]["ms"] / res["plain"]["ms"] - 1.0
     return {"lora_dropout_llama7b_attn": res}
 
@@ -799,12 +813,29 @@ def comp_workloads(q, dev, peaks, n=10):
     return out
 
 
-def layer_step_once(q, dev):
-    """One untimed step of the headline layer (for a profiler's launch list)."""
-    L = LayerState(q, WL, 0, dev)
+def layer_step_once(q, dev, projections=None, steps=1):
+    """Untimed steps of the headline layer, or of some of its projections
+    (for a profiler's launch list or a capture on a smaller device footprint)."""
+    wl = WL
+    if projections is not None:
+        import dataclasses
+        wl = dataclasses.replace(WL, projections=tuple(WL.projections[i] for i in projections))
+    L = LayerState(q, wl, 0, dev)
     L.step()
     torch.cuda.synchronize()
-    return {"ok": q.last_device_status() == 0, "projections": len(L.proj)}
+    q.timing_reset()
+    q.timing_enable(True)
+    for _ in range(steps):
+        L.step()
+    torch.cuda.synchronize()
+    q.timing_enable(False)
+    kern = {}
+    for name in q.KERNEL_NAMES:
+        t, n = q.timing_collect(name)
+        if n:
+            kern[name] = {"avg_us": 1e3 * t / n, "launches": n}
+    return {"ok": q.last_device_status() == 0, "projections": [p[0] for p in wl.projections], "steps": steps,
+            "kernels": kern}
 
 
 def components(q, dev, only=None):
@@ -824,6 +855,8 @@ def components(q, dev, only=None):
         out.update(comp_dropout(q, dev, peaks))
     if only == "layer_step":
         out.update(layer_step_once(q, dev))
+    if only == "q_proj_steps":
+        out.update(layer_step_once(q, dev, projections=(0,), steps=4))
     return out
 
 

@@ -22,7 +22,6 @@
 #include "merge.cuh"
 #include "dropout.cuh"
 #include "quant.cuh"
-#include "skinny.cuh"
 #include "lora_sm100.cuh"
 #include "pad.cuh"
 
@@ -175,14 +174,13 @@ bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t c
 }
 
 // 2-D byte tensor [rows, cols] (packed NF4 codes, cols = in / 2), box
-// {128 bytes, 16 rows} (one warp's code tile of the GEMV), 128B swizzle,
-// out-of-range bytes read as zero.
+// {128 bytes, 256 rows}, 128B swizzle, out-of-range bytes read as zero.
 bool make_tmap_codes(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(qnf4::kGvSlice / 2), static_cast<cuuint32_t>(qnf4::kGvTile)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(qnf4::kGvStageK / 2), static_cast<cuuint32_t>(qnf4::kGvRows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -257,90 +255,44 @@ constexpr QuantWs quant_ws(int64_t rows, int64_t cols) {
   return w;
 }
 
-// Few-token GEMV plan: warps own 256-column K slices, a CTA's WARPS slices
-// form a K group, items are (group, 16-row tile); one CTA per SM.
 struct GemvPlan {
-  int nt;                 // 8 or 16 token columns
-  int warps, n_slices, groups, tiles, ctas;
-  int64_t n_items;
-  size_t ws;              // workspace: the group partials (groups > 1)
+  int ctas, local_tiles, n_st;
+  int64_t n_units;
 };
 
-// Of the four MMA steps of a block, how many decode the rows g + 8 with the
-// register table instead of the shared one (QLORA_NF4_GEMV_REG_STEPS
-// overrides the default for tuning).
-int gemv_reg_steps() {
-  static int v = [] {
-    const char* e = std::getenv("QLORA_NF4_GEMV_REG_STEPS");
-    const int n = e ? std::atoi(e) : 0;
-    return (n == 1 || n == 2) ? n : 0;
-  }();
-  return v;
-}
-
-template <int NT>
-using GemvKernel = void (*)(const CUtensorMap, const qnf4::GemvArgs);
-
-template <int NT>
-GemvKernel<NT> gemv_kernel_for() {
-  switch (gemv_reg_steps()) {
-    case 1: return qnf4::nf4_gemv_kernel<NT, 1>;
-    case 2: return qnf4::nf4_gemv_kernel<NT, 2>;
-    default: return qnf4::nf4_gemv_kernel<NT, 0>;
-  }
-}
-
-template <int NT>
-int gemv_ctas_per_sm_t() {
-  using C = qnf4::GvCfg<NT>;
+int gemv_ctas_per_sm() {
   static std::atomic<int> cache[kMaxDevices];
   const int dev = current_device();
   const int c = cache[dev].load(std::memory_order_relaxed);
   if (c > 0) return c;
   int n = 0;
-  const GemvKernel<NT> k = gemv_kernel_for<NT>();
-  if (set_max_smem(reinterpret_cast<const void*>(k), C::SMEM) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, C::THREADS, C::SMEM) != cudaSuccess || n < 1)
+  const void* kern = reinterpret_cast<const void*>(qnf4::nf4_gemv_kernel<true, true>);
+  if (set_max_smem(kern, qnf4::kGvSmem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, qnf4::nf4_gemv_kernel<true, true>, qnf4::kGvThreads,
+                                                    qnf4::kGvSmem) != cudaSuccess ||
+      n < 1)
     return 1;
   cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
-GemvPlan gemv_plan(int64_t M, int64_t in, int64_t out) {
+// Persistent grid (every CTA resident at once) splitting the (256-row tile x
+// 256-column unit) sequence evenly; local_tiles bounds the tiles one CTA's
+// range touches.
+GemvPlan gemv_plan(int64_t in, int64_t out) {
   GemvPlan p{};
-  p.nt = M > 8 ? 16 : 8;
-  p.warps = p.nt == 8 ? qnf4::GvCfg<8>::WARPS : qnf4::GvCfg<16>::WARPS;
-  p.n_slices = static_cast<int>(cdiv(in, qnf4::kGvSlice));
-  p.groups = static_cast<int>(cdiv(p.n_slices, p.warps));
-  p.tiles = static_cast<int>(out / qnf4::kGvTile);
-  p.n_items = static_cast<int64_t>(p.groups) * p.tiles;
-  const int per_sm = p.nt == 8 ? gemv_ctas_per_sm_t<8>() : gemv_ctas_per_sm_t<16>();
-  const int64_t resident = static_cast<int64_t>(per_sm) * device_sm_count();
-  p.ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(resident, p.n_items)));
-  p.ws = p.groups > 1 ? round256(static_cast<size_t>(p.groups) * out * M * 4) : 0;
+  p.n_st = static_cast<int>(cdiv(in, qnf4::kGvStageK));
+  p.n_units = cdiv(out, qnf4::kGvRows) * p.n_st;
+  const int64_t resident = static_cast<int64_t>(gemv_ctas_per_sm()) * device_sm_count();
+  p.ctas = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(resident, p.n_units)));
+  const int64_t per_cta = cdiv(p.n_units, p.ctas);
+  p.local_tiles = static_cast<int>(cdiv(per_cta, p.n_st) + 1);
   return p;
 }
 
-size_t gemv_ws(int64_t M, int64_t in, int64_t out) { return gemv_plan(M, in, out).ws; }
-
-// K splits of the row-wise rank-r product: enough CTAs (64 rows x one
-// 64-wide rank chunk x one K range each) to keep ~2 per SM streaming, with at
-// least 4 K stages (256 columns) per range.  The splits of a row tile form one
-// cluster (reduced over distributed shared memory), so there are at most 8.
-int rowwise_splits(int64_t M, int64_t K, int r) {
-  const int64_t tiles = cdiv(M, 64) * cdiv(r, 64);
-  const int64_t n_st = K / 64;
-  const int64_t want = cdiv(2 * device_sm_count(), tiles);
-  int64_t ks = std::max<int64_t>(1, std::min<int64_t>({want, n_st / 4, 8}));
-  ks = cdiv(n_st, cdiv(n_st, ks));                     // no empty split
-  return static_cast<int>(ks);
-}
-
-// Token chunks of the column-wise products: one cluster of at most 8 chunks
-// per 128-wide column tile, each chunk a multiple of 32 tokens.
-int col_chunk_tokens(int64_t M) {
-  const int64_t chunks = std::max<int64_t>(1, std::min<int64_t>(qnf4::kColMaxChunks, cdiv(M, 256)));
-  return static_cast<int>(cdiv(cdiv(M, chunks), 32) * 32);
+size_t gemv_ws(int64_t M, int64_t in, int64_t out) {
+  const GemvPlan p = gemv_plan(in, out);
+  return round256(static_cast<size_t>(p.ctas) * p.local_tiles * M * qnf4::kGvRows * 4);
 }
 
 // LoRA rank as the kernels take it: a multiple of 8 (16-byte rows).
@@ -562,6 +514,7 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
   a.K = static_cast<int>(K);
   a.r = r;
   a.w_cols = static_cast<int>(w->cols);
+  a.codes_32b = aligned(w->codes, 32) ? 1 : 0;
   a.L = tables().L;
   a.timeout_ns = g_timeout_ns.load();
   const int tm = gemm_tile_m(M);
@@ -574,35 +527,6 @@ int launch_gemm(bool dx, const qlora_nf4_weight* w, const uint16_t* act, int64_t
                    : launch_gemm_t<1, true, 4>(a, tm_act, tm_lora, st);
 }
 
-template <int NT, bool kKR>
-int launch_rowwise_t(const uint16_t* act, const uint16_t* W, uint16_t* out, int ks, int64_t M, int64_t K, int R,
-                     float scale, cudaStream_t st, const uint8_t* keep) {
-  using C = qnf4::RowCfg<NT, kKR>;
-  auto kern = keep != nullptr ? qnf4::rowwise_skinny_kernel<NT, kKR, true> : qnf4::rowwise_skinny_kernel<NT, kKR, false>;
-  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), C::SMEM));
-  const int n_st = static_cast<int>(K / 64);
-  const int sps = static_cast<int>(cdiv(n_st, ks));
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(cdiv(M, 64)), static_cast<unsigned>(ks), static_cast<unsigned>(cdiv(R, C::RC)));
-  cfg.blockDim = dim3(qnf4::kRowThreads);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(ks);
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = ks > 1 ? 1 : 0;
-  {
-    LaunchTimer lt_(kKR ? "lora_rowwise_du" : "lora_rowwise", st);
-    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, act, W, out, static_cast<int>(M), static_cast<int>(K), R, scale, sps,
-                                      keep));
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  return QLORA_OK;
-}
-
 // ------------------------------------------------------------------ tcgen05 rank-r products
 int lr_n_alloc(int N) {
   int a = 32;
@@ -610,19 +534,27 @@ int lr_n_alloc(int N) {
   return a;
 }
 
-// Contraction split over a cluster: the smallest power of two (<= 8) that
-// gives at least one CTA per SM, keeping at least 2 stages per split.
-int lr_splits(int64_t tiles, int64_t stages) {
-  int ks = 1;
-  while (ks < 8 && tiles * ks < device_sm_count() && stages / (2 * ks) >= 2) ks *= 2;
-  return ks;
+// Launch shape of a rank-r product: a ring of 4 stages (measured best: deeper
+// rings in one CTA per SM streamed slower), two CTAs per SM where the
+// shared memory allows it; the contraction is split over a cluster (a power
+// of two <= 8) as far as the CTAs still fit about one per SM, keeping at
+// least 2 stages per split.
+struct LrShape {
+  int ks, ring;
+};
+
+LrShape lr_shape(int64_t tiles, int64_t stages) {
+  const int sms = device_sm_count();
+  LrShape sh{1, 4};
+  while (sh.ks < 8 && tiles * sh.ks * 2 <= sms && stages / (2 * sh.ks) >= 2) sh.ks *= 2;
+  return sh;
 }
 
 template <bool kCol, bool kBMN>
 int launch_lora_umma(const CUtensorMap (&tm)[4], const qnf4::LrArgs& a, int ks, unsigned grid_x, const char* name,
                      cudaStream_t st) {
   auto kern = qnf4::lora_umma_kernel<kCol, kBMN>;
-  const int smem = qnf4::lr_smem_bytes(a.N, kBMN);
+  const int smem = qnf4::lr_smem_bytes(a.N, kBMN, a.ring);
   QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), smem));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid_x, static_cast<unsigned>(ks), 1);
@@ -647,17 +579,20 @@ int launch_lora_umma(const CUtensorMap (&tm)[4], const qnf4::LrArgs& a, int ks, 
 // Row form: out[M, r] = bf16(scale * act[M, K] . w^T), w given as [r, K]
 // (w_n_major = false: A of the forward) or as [K, r] (true: B of du).
 int launch_lora_row(const uint16_t* act, const uint16_t* w, uint16_t* out, int64_t M, int64_t K, int r, float scale,
-                    bool w_n_major, const char* name, cudaStream_t st) {
+                    bool w_n_major, const char* name, cudaStream_t st, const uint8_t* keep = nullptr) {
   qnf4::LrArgs a{};
   a.r = r;
   a.N = (r + 15) / 16 * 16;
   a.n_alloc = lr_n_alloc(a.N);
   a.K = static_cast<int>(K);
-  a.p[0] = qnf4::LrProblem{out, static_cast<int>(M), static_cast<int>(cdiv(M, 128)), 0, scale};
+  a.p[0] = qnf4::LrProblem{out, static_cast<int>(M), static_cast<int>(cdiv(M, 128)), 0, scale, keep,
+                           static_cast<int>(K)};
   a.p[1] = a.p[0];
   a.timeout_ns = g_timeout_ns.load();
   const int64_t stages = cdiv(K, 64);
-  const int ks = lr_splits(a.p[0].tiles, stages);
+  const LrShape sh = lr_shape(a.p[0].tiles, stages);
+  const int ks = sh.ks;
+  a.ring = sh.ring;
   a.stages_per_split = static_cast<int>(cdiv(stages, ks));
   CUtensorMap tm[4];
   if (!make_tmap_bf16(&tm[0], act, M, K, 128)) return QLORA_ERR_CUDA;
@@ -673,17 +608,22 @@ int launch_lora_row(const uint16_t* act, const uint16_t* w, uint16_t* out, int64
 // Col form, both adapter gradients in one launch: dB [out, r] = dh^T us and
 // dA [r, in] = (x^T du)^T * dA_scale.
 int launch_lora_col(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
-                    int64_t in, int64_t out, int r, float* dB, float* dA, float dA_scale, cudaStream_t st) {
+                    int64_t in, int64_t out, int r, float* dB, float* dA, float dA_scale, cudaStream_t st,
+                    const uint8_t* keep = nullptr) {
   qnf4::LrArgs a{};
   a.r = r;
   a.N = (r + 15) / 16 * 16;
   a.n_alloc = lr_n_alloc(a.N);
   a.K = static_cast<int>(M);
-  a.p[0] = qnf4::LrProblem{dB, static_cast<int>(out), static_cast<int>(cdiv(out, 128)), 0, 1.f};
-  a.p[1] = qnf4::LrProblem{dA, static_cast<int>(in), static_cast<int>(cdiv(in, 128)), 1, dA_scale};
+  a.p[0] = qnf4::LrProblem{dB, static_cast<int>(out), static_cast<int>(cdiv(out, 128)), 0, 1.f, nullptr,
+                           static_cast<int>(out)};
+  a.p[1] = qnf4::LrProblem{dA, static_cast<int>(in), static_cast<int>(cdiv(in, 128)), 1, dA_scale, keep,
+                           static_cast<int>(in)};
   a.timeout_ns = g_timeout_ns.load();
   const int64_t stages = cdiv(M, 64);
-  const int ks = lr_splits(a.p[0].tiles + a.p[1].tiles, stages);
+  const LrShape sh = lr_shape(a.p[0].tiles + a.p[1].tiles, stages);
+  const int ks = sh.ks;
+  a.ring = sh.ring;
   a.stages_per_split = static_cast<int>(cdiv(stages, ks));
   CUtensorMap tm[4];
   if (!make_tmap_bf16(&tm[0], dh, M, out, 64) || !make_tmap_bf16(&tm[1], us, M, r, 64) ||
@@ -695,50 +635,18 @@ int launch_lora_col(const uint16_t* dh, const uint16_t* us, const uint16_t* x, c
 
 // out[M, R] = bf16(scale * (act[M, K] * k) . W^T) with W given as [R, K] (kKR =
 // false) or as [K, R] (kKR = true); k the keep mask of LoRA dropout, or all
-// ones when keep is null (then the tcgen05 kernel runs).
+// ones when keep is null.
 template <bool kKR>
 int launch_rowwise(const uint16_t* act, const uint16_t* W, uint16_t* out, int64_t M, int64_t K, int R, float scale,
                    cudaStream_t st, const uint8_t* keep = nullptr) {
-  if (keep == nullptr)
-    return launch_lora_row(act, W, out, M, K, R, scale, kKR, kKR ? "lora_rowwise_du" : "lora_rowwise", st);
-  const int ks = rowwise_splits(M, K, R);
-  if (R <= 8) return launch_rowwise_t<1, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
-  if (R <= 16) return launch_rowwise_t<2, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
-  if (R <= 32) return launch_rowwise_t<4, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
-  return launch_rowwise_t<8, kKR>(act, W, out, ks, M, K, R, scale, st, keep);
+  return launch_lora_row(act, W, out, M, K, R, scale, kKR, kKR ? "lora_rowwise_du" : "lora_rowwise", st, keep);
 }
 
-// dB = dh^T us -> [out, r] and dA = du^T x -> [r, in] in one launch: column
-// tiles x token chunks x the two problems, chunks of a tile in one cluster.
+// dB = dh^T us -> [out, r] and dA = du^T (x * k) * dA_scale -> [r, in] in one launch.
 int launch_lora_grads(const uint16_t* dh, const uint16_t* us, const uint16_t* x, const uint16_t* du, int64_t M,
                       int64_t in, int64_t out, int R, float* dB, float* dA, cudaStream_t st, float dA_scale = 1.f,
                       const uint8_t* keep = nullptr) {
-  if (keep == nullptr) return launch_lora_col(dh, us, x, du, M, in, out, R, dB, dA, dA_scale, st);
-  const qnf4::ColProblem pb{dh, us, dB, static_cast<int>(out), 0, 1.f, nullptr};
-  const qnf4::ColProblem pa{x, du, dA, static_cast<int>(in), 1, dA_scale, keep};   // dA^T = (x * k)^T du
-  const int smem = qnf4::kColStages * qnf4::kColStageBytes;
-  auto kern = keep != nullptr ? qnf4::colwise_skinny_kernel<true> : qnf4::colwise_skinny_kernel<false>;
-  QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), smem));
-  const int chunk_tokens = col_chunk_tokens(M);
-  const unsigned chunks = static_cast<unsigned>(cdiv(M, chunk_tokens));
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(cdiv(std::max(in, out), 128)), chunks, 2);
-  cfg.blockDim = dim3(qnf4::kColThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = chunks;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  {
-    LaunchTimer lt_("lora_colwise", st);
-    QLORA_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, pb, pa, static_cast<int>(M), R, chunk_tokens));
-  }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  return QLORA_OK;
+  return launch_lora_col(dh, us, x, du, M, in, out, R, dB, dA, dA_scale, st, keep);
 }
 
 // ------------------------------------------------------------------ validation
@@ -767,49 +675,40 @@ int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlo
   int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s_lora, st, keep);   // us = bf16(s (x k) A^T)
   if (rc != QLORA_OK) return rc;
   if (M <= 16) {
-    const GemvPlan p = gemv_plan(M, in, out);
+    const GemvPlan p = gemv_plan(in, out);
     qnf4::GemvArgs g{};
     g.q8 = w->q8;
     g.step2 = w->step2;
     g.mean = w->mean;
-    g.x = x;
-    g.us = us_out;
-    g.B = B;
-    g.h = h;
     g.part = static_cast<float*>(workspace);
     g.M = static_cast<int>(M);
     g.in = static_cast<int>(in);
     g.out = static_cast<int>(out);
-    g.r = r;
-    g.n_slices = p.n_slices;
-    g.groups = p.groups;
-    g.tiles = p.tiles;
-    g.n_items = p.n_items;
+    g.n_st = p.n_st;
+    g.n_units = p.n_units;
+    g.local_tiles = p.local_tiles;
     g.timeout_ns = g_timeout_ns.load();
     g.L = tables().L;
-    CUtensorMap tm_codes;
-    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)))
+    CUtensorMap tm_codes, tm_x;
+    if (!make_tmap_codes(&tm_codes, w->codes, static_cast<uint64_t>(out), static_cast<uint64_t>(in / 2)) ||
+        !make_tmap_bf16(&tm_x, x, static_cast<uint64_t>(M), static_cast<uint64_t>(in), M > 8 ? 16 : 8))
       return QLORA_ERR_CUDA;
     {
       LaunchTimer lt_("gemv", st);
-      if (p.nt == 8) {
-        const GemvKernel<8> k = gemv_kernel_for<8>();
-        QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(k), qnf4::GvCfg<8>::SMEM));
-        k<<<p.ctas, qnf4::GvCfg<8>::THREADS, qnf4::GvCfg<8>::SMEM, st>>>(tm_codes, g);
-      } else {
-        const GemvKernel<16> k = gemv_kernel_for<16>();
-        QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(k), qnf4::GvCfg<16>::SMEM));
-        k<<<p.ctas, qnf4::GvCfg<16>::THREADS, qnf4::GvCfg<16>::SMEM, st>>>(tm_codes, g);
-      }
+      const bool paired = in % qnf4::kGvStageK == 0, two_tok = M > 8;   // four whole blocks per unit
+      auto kern = paired ? (two_tok ? qnf4::nf4_gemv_kernel<true, true> : qnf4::nf4_gemv_kernel<true, false>)
+                         : (two_tok ? qnf4::nf4_gemv_kernel<false, true> : qnf4::nf4_gemv_kernel<false, false>);
+      QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), qnf4::kGvSmem));
+      kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
-    if (p.groups > 1) {
-      const int64_t n_el = M * out;
+    const int64_t n_el = M * out;
+    {
       LaunchTimer lt_("gemv_finalize", st);
       qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
-          g.part, p.groups, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
-      QLORA_CUDA_TRY(cudaGetLastError());
+          g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
     }
+    QLORA_CUDA_TRY(cudaGetLastError());
     return QLORA_OK;
   }
   return launch_gemm(false, w, x, M, in, us_out, B, r, h, out, st);  // h = [x|us] [W0|B]^T
@@ -1092,13 +991,13 @@ int qlora_dequantize_codebook(int kind, const qlora_nf4_weight* w, uint16_t* W_o
   if (!weight_ok(w) || !W_out || !aligned(W_out, 16)) return QLORA_ERR_INVALID_ARG;
   if (w->rows < 1 || w->cols < 64 || w->cols % 64 != 0 || w->rows * w->cols > (1ll << 40))
     return QLORA_ERR_UNSUPPORTED_SHAPE;
-  const int64_t halves = w->rows * w->cols / 32;
-  const int64_t want = cdiv(halves, 256);
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, device_sm_count() * 16)));
+  const int64_t words = w->rows * w->cols / 8;
+  const int64_t want = cdiv(words, 8 * 128 * qnf4::kDqRounds);        // 8 warps x 128 words x rounds per CTA
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, device_sm_count() * 8)));
   {
     LaunchTimer lt_("dequantize", static_cast<cudaStream_t>(stream));
     qnf4::nf4_dequantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      w->codes, w->q8, w->step2, w->mean, halves, W_out, tb->L);
+      w->codes, w->q8, w->step2, w->mean, words, W_out, tb->L);
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return QLORA_OK;

@@ -9,7 +9,7 @@
 //
 // The masked input x * k (exact in bf16: kept or zero) is never stored: the
 // rank-r kernels apply the keep bits to the activation tiles they stage
-// (skinny.cuh).
+// (lora_sm100.cuh).
 // dropout_dx_kernel    dx = bf16(fp32(dx_base) + (k / (1 - p)) * sum_j du[m][j] A[j][i])
 //                      after the dx GEMM ran without its rank-r tail; the sum
 //                      is an in-order fp32 fused multiply-add chain

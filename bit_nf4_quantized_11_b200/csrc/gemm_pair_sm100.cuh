@@ -223,8 +223,12 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
       if (col_valid && it < n_main) {
         const uint8_t* p = code_ptr + it * code_step;
         const int64_t blk = q8_idx + it * q8_step;
-        d.c0 = ld_nc_v4(p);
-        d.c1 = ld_nc_v4(p + 16);
+        if (args.codes_32b) {
+          ld_nc_v8(p, d.c0, d.c1);
+        } else {
+          d.c0 = ld_nc_v4(p);
+          d.c1 = ld_nc_v4(p + 16);
+        }
         d.q = __ldg(args.q8 + blk);
         d.st = __ldg(args.step2 + blk / 256);
       }
@@ -268,13 +272,17 @@ qlora_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_act,
       }
     };
 
-    StageIn na{};
+    // codes and scale codes are loaded two of this group's turns ahead (eight
+    // stages), so their global-load latency overlaps two turns of MMAs
+    StageIn na{}, nb{};
     load_stage(group, na);
+    load_stage(group + G, nb);
     const bool warp_lead = lane == 0;
 
     for (int it = group; it < n_iter; it += G) {
       const StageIn cur = na;
-      load_stage(it + G, na);
+      na = nb;
+      load_stage(it + 2 * G, nb);
       uint4 v[8];
       produce(it, cur, v);                          // before waiting for the buffer
 

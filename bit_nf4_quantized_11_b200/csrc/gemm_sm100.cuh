@@ -47,6 +47,7 @@ struct GemmArgs {
   int K;                  // main contraction length (forward: in, dx: out)
   int r;                  // LoRA rank (multiple of 8)
   int w_cols;             // columns of W0 (= in)
+  int codes_32b;          // codes 32-byte aligned: a thread's 32 code bytes in one load
   Levels L;
   uint64_t timeout_ns;
 };
@@ -234,8 +235,12 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,
       if (col_valid && it < n_main) {
         const uint8_t* p = code_ptr + it * code_step;
         const int64_t blk = q8_idx + it * q8_step;
-        d.c0 = ld_nc_v4(p);
-        d.c1 = ld_nc_v4(p + 16);
+        if (args.codes_32b) {
+          ld_nc_v8(p, d.c0, d.c1);
+        } else {
+          d.c0 = ld_nc_v4(p);
+          d.c1 = ld_nc_v4(p + 16);
+        }
         d.q = __ldg(args.q8 + blk);
         d.st = __ldg(args.step2 + blk / 256);
       }

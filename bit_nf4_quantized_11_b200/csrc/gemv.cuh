@@ -2,104 +2,80 @@
 //
 // With 1..16 tokens the layer is bound by streaming the packed weight from
 // HBM (0.52 byte per weight), so the kernel is organised around that stream
-// and around the issue and load/store-unit budget per weight it leaves
-// ("QLoRA", llm-compass, 方法与公式: h = dequant(W0) x + (alpha/r) B A x; the
-// auryth glossary's "Hoe het werkt" diagram: W0 is dequantized on the fly per
-// layer).
+// and around the issue and load/store-unit budget per weight it leaves.  The
+// work is (row tile of 256 weight rows) x (unit of 256 K columns = four
+// 64-weight blocks) units, ordered tile-major; a persistent grid of one CTA
+// per SM splits the unit sequence evenly, so every CTA streams the same
+// number of bytes whatever the shape.
 //
-// Work decomposition.  Every warp of a CTA owns one 256-column K slice (four
-// 64-weight blocks); the WARPS slices of a CTA form a K group.  An item is
-// (K group, 16-row tile); items are ordered group-major and a persistent grid
-// of one CTA per SM splits them evenly by work, so each CTA mostly stays in
-// one group and each warp keeps the activations of its slice in registers
-// for the whole run (loaded once per group, never re-read per tile).
+// Per unit, one thread issues two TMA loads into a ring of shared-memory
+// stages: the 256 x 128-byte code tile and the 8- (or 16-) token x 256-column
+// activation tile, both with 128-byte swizzle so that the reads below are
+// bank-conflict free.  16 warps own 16 rows each (the 16-row operand of a
+// warp-level bf16 MMA); per unit a thread reads, for rows g and g+8, 16
+// consecutive codes of each of the four blocks, and its warp releases the
+// code part of the stage as soon as they are in registers.  Second-level
+// scale codes (four per row and unit) are fetched one unit ahead, group
+// steps are cached.
 //
-// Stream.  Each warp runs its own TMA pipeline: lane 0 loads the 16 x 128-byte
-// code tile of its slice (128-byte swizzle) into a private ring of stages and
-// refills a stage as soon as the warp has read it; no barrier couples the
-// warps while they stream.
+// Each MMA step covers 16 columns of ONE block for all four quad lanes: step
+// s of block j takes columns 64j + 16q + 4s .. +3 for quad lane q, in the
+// same permuted K order for weights and activations.  A block's four steps
+// accumulate into a fresh fp32 tile that is then added to the running sum
+// times the block's exact fp32 scale c_hat (rows g and g+8 each with their
+// own), so the MMA's weight operand is bf16(level) -- the exactly rounded
+// level -- and the scale costs nothing per weight.  (The GEMM path instead
+// rounds bf16(level * c_hat) per weight; the two differ by at most 2^-9
+// relative per weight, far inside the output tolerance.)
 //
-// Decode and MMA.  A warp computes its slice of a tile with warp-level bf16
-// MMAs (m16n8k16: the 16 weight rows x 8 tokens); each MMA covers 16 columns
-// of ONE block (quad lane q takes columns 16q + 4s .. +3 of the block in step
-// s, the same permuted K order for weights and activations), so a block's
-// four MMAs accumulate into a fresh fp32 tile that is added to the running
-// sum times the block's exact fp32 scale c_hat.  The weight operand is
-// bf16(level), exactly rounded; the GEMM path's bf16(level * c_hat) differs
-// from it by at most 2^-9 relative per weight, far inside the tolerance.
-// Rows g (g = lane / 4) are decoded through a shared-memory table of bf16
-// level pairs (one prmt and one load per code byte); rows g + 8 through a
-// register-resident 16-entry table selected with prmt (no memory access), so
-// the decode splits its work between the load/store unit and the ALUs.
-// A block's scale is computed once per quad lane and passed to the other
-// three lanes by shuffles.
-//
-// Reduction.  Each warp leaves its partial tile (16 rows x tokens) in the
-// free upper halves of the table's rows; every few items the CTA sums the
-// warps' partials in warp order.  With one K group that sum, plus the LoRA
-// term us . B^T, is the output; otherwise it is the group's fp32 partial,
-// and gemv_finalize_kernel adds the groups' partials in group order and the
-// LoRA term.  Every summation order is fixed, so h is deterministic.
+// Decoding is one byte permute and one shared load per nibble pair: the
+// 256-entry table of bf16 level pairs has one 256-byte row per byte value,
+// with one 4-byte copy per lane in its first 128 bytes (so lookups never
+// conflict), and sits on a 64 KB boundary of the shared window, so that a
+// single prmt assembles (window bits 16-17 | byte << 8 | lane * 4), the
+// complete shared address.  Where a CTA's range starts or ends inside a tile
+// it writes an fp32 partial of that tile; the finalize kernel adds a tile's
+// partials in CTA order and the LoRA branch us . B^T ("QLoRA", llm-compass,
+// 方法与公式: h = dequant(W0) x + (alpha/r) B A x).
 #pragma once
 
 #include "common.cuh"
 
 namespace qnf4 {
 
-constexpr int kGvSlice = 256;                             // K columns per warp (four blocks)
-constexpr int kGvTile = 16;                               // weight rows per tile
-constexpr int kGvTileBytes = kGvTile * kGvSlice / 2;      // 2 KB of packed codes
-constexpr int kGvStages = 4;                              // per-warp ring of code tiles
-constexpr int kGvLutBytes = 256 * 256;                    // 256 rows of 256 B on a 64 KB boundary
-constexpr int kGvMaxTok = 16;
-
-template <int NT>
-struct GvCfg {
-  static constexpr int WARPS = NT == 8 ? 16 : 12;         // K slices per CTA (register budget)
-  static constexpr int THREADS = 32 * WARPS;
-  static constexpr int GROUP = WARPS * kGvSlice;          // K columns per group
-  static constexpr int SLOTS = WARPS * kGvStages;
-  static constexpr int CHUNKS_PER_WARP = NT / 2;          // 128-byte pieces of one warp's partial tile
-  static constexpr int RED_ITEMS = 256 / (WARPS * CHUNKS_PER_WARP);   // items per reduction round
-  // the table's 64 KB, the stages (2 KB slots below and above the table; less
-  // than one slot of the gap below it stays unused) and the barriers, plus
-  // alignment slack
-  static constexpr int SMEM = kGvLutBytes + SLOTS * kGvTileBytes + 4096;
-  static_assert(RED_ITEMS >= 1, "reduction round");
-};
+constexpr int kGvWarps = 16;
+constexpr int kGvThreads = 32 * kGvWarps;
+constexpr int kGvRows = 16 * kGvWarps;                    // weight rows per tile (256)
+constexpr int kGvStageK = 256;                            // K columns per unit (four blocks)
+constexpr int kGvStages = 3;                              // ring of unit tiles (2 in flight)
+constexpr int kGvCodeBytes = kGvRows * kGvStageK / 2;     // 32 KB
+constexpr int kGvXBox = 64;                               // activation box: 64 columns x tokens
+constexpr int kGvStageBytes = kGvCodeBytes + 16 * kGvStageK * 2;   // + up to 16 tokens x 256 columns
+constexpr int kGvLutBytes = 256 * 256;                    // 256 rows of 256 bytes
+constexpr int kGvSmem = 192 * 1024;                       // stages, then the table on the next 64 KB boundary
 
 struct GemvArgs {
   const int8_t* q8;
   const float* step2;
   const float* mean;
-  const uint16_t* x;       // [M, in] bf16
-  const uint16_t* us;      // [M, r] bf16, s x A^T (written before this kernel)
-  const uint16_t* B;       // [out, r] bf16
-  uint16_t* h;             // [M, out] bf16
-  float* part;             // [groups, out, M] fp32 group partials (groups > 1)
-  int M, in, out, r;
-  int n_slices;            // ceil(in / 256)
-  int groups;              // ceil(n_slices / WARPS)
-  int tiles;               // out / 16
-  int64_t n_items;         // groups * tiles
-  uint64_t timeout_ns;
+  float* part;             // [ctas][local_tiles][M][kGvRows]
+  int M, in, out;
+  int n_st;                // units per tile = ceil(in / 256)
+  int64_t n_units;         // tiles * n_st
+  int local_tiles;         // partial tiles reserved per CTA
+  uint64_t timeout_ns;     // bound of every pipeline wait
   Levels L;
 };
 
-// Work of the items before item i (group-major; every group but the last has
-// WARPS slices), and the first item whose preceding work reaches w.
-__device__ __forceinline__ int64_t gv_work_before(int64_t i, int64_t tiles, int warps, int last_slices,
-                                                  int groups) {
-  const int64_t full = static_cast<int64_t>(groups - 1) * tiles;
-  return i <= full ? i * warps : full * warps + (i - full) * last_slices;
-}
-__device__ __forceinline__ int64_t gv_item_at(int64_t w, int64_t tiles, int warps, int last_slices, int groups) {
-  const int64_t full = static_cast<int64_t>(groups - 1) * tiles;
-  const int64_t wf = full * warps;
-  if (w <= wf) return (w + warps - 1) / warps;
-  return full + (w - wf + last_slices - 1) / last_slices;
+// First unit of CTA c when n units are split over p CTAs.
+__host__ __device__ __forceinline__ int64_t gemv_unit_begin(int64_t c, int64_t n, int64_t p) {
+  return c * n / p;
 }
 
+// Register-only MMAs and table loads without `volatile`, so that the
+// compiler may interleave the lookups of one step with the MMA of the
+// previous one.  Every table address derives from a value produced after the
+// barrier that publishes the table (a volatile move).
 __device__ __forceinline__ void gv_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
@@ -108,9 +84,15 @@ __device__ __forceinline__ void gv_mma(float (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// Table lookups: not volatile, so the compiler may interleave them with the
-// MMAs; every table address derives from a value loaded after the barrier
-// that publishes the table.
+// d = A B with a zero accumulator input.
+__device__ __forceinline__ void gv_mma_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 __device__ __forceinline__ uint32_t gv_lds(uint32_t addr) {
   uint32_t v;
   asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -124,351 +106,300 @@ __device__ __forceinline__ uint2 gv_lds64(uint32_t addr) {
   return v;
 }
 
-// Bounded wait on the mbarrier at shared address `bar` for the phase of the
-// given parity; false on timeout.
-__device__ __forceinline__ bool gv_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > timeout_ns) return false;
-  }
-}
-
-__device__ __forceinline__ uint4 gv_ldg128(const void* p) {
+__device__ __forceinline__ uint4 gv_lds128(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr) : "memory");
   return v;
 }
 
-// Sum over j < r of us[m][j] * B[o][j] (bf16 inputs, fp32 FMAs in j order).
-__device__ __forceinline__ float gv_lora(const uint16_t* __restrict__ us, const uint16_t* __restrict__ B, int m,
-                                         int o, int r) {
-  const uint16_t* ur = us + static_cast<int64_t>(m) * r;
-  const uint16_t* br = B + static_cast<int64_t>(o) * r;
-  float l = 0.f;
-  for (int j = 0; j < r; j += 8) {
-    const uint4 ua = __ldg(reinterpret_cast<const uint4*>(ur + j));
-    const uint4 ba = __ldg(reinterpret_cast<const uint4*>(br + j));
-    const uint32_t uw[4] = {ua.x, ua.y, ua.z, ua.w}, bw[4] = {ba.x, ba.y, ba.z, ba.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[i]));
-      const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
-      l = fmaf(uf.x, bf.x, l);
-      l = fmaf(uf.y, bf.y, l);
-    }
-  }
-  return l;
+// Byte offset, in a tile of 128-byte rows written with 128-byte swizzle, of
+// the 16-byte chunk c of row `row` (chunk index XOR row % 8) plus `half` * 8.
+__device__ __forceinline__ uint32_t gv_swz128(int row, int c, int half) {
+  return static_cast<uint32_t>(row * 128 + (((c ^ row) & 7) << 4) + half * 8);
 }
 
-// kRegSteps: of the four MMA steps of a block, how many decode the rows g + 8
-// with the register table (ALU) instead of the shared table (load/store unit).
-template <int NT, int kRegSteps>
-__global__ void __launch_bounds__(GvCfg<NT>::THREADS, 1)
-    nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const GemvArgs a) {
-  using C = GvCfg<NT>;
-  constexpr int W = C::WARPS;
-  constexpr int kTok2 = NT == 16;                          // a second 8-token MMA tile
+// kPaired: in % 256 == 0, so every unit holds four whole blocks whose index
+// run starts at a multiple of 4 (one aligned 32-bit load of their q8 codes,
+// one group step for all four).  kTwoTok: 9..16 tokens, a second 8-token MMA
+// tile.
+template <bool kPaired, bool kTwoTok>
+__global__ void __launch_bounds__(kGvThreads, 1)
+    nf4_gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                    const GemvArgs a) {
+  constexpr int XR = kTwoTok ? 16 : 8;                               // token rows of the activation box
+  constexpr uint32_t kTxBytes = kGvCodeBytes + 4 * kGvXBox * 2 * XR;
   extern __shared__ __align__(1024) uint8_t s_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kGvStages], empty_bar[kGvStages];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, q = lane & 3;
+  const int64_t u_begin = gemv_unit_begin(blockIdx.x, a.n_units, gridDim.x);
+  const int64_t u_end = gemv_unit_begin(blockIdx.x + 1, a.n_units, gridDim.x);
+  if (u_begin >= u_end) return;                                     // CTA-uniform
+  const int n_local = static_cast<int>(u_end - u_begin);
+  const int t_first = static_cast<int>(u_begin / a.n_st);
+  const int st_first = static_cast<int>(u_begin - static_cast<int64_t>(t_first) * a.n_st);
 
-  // ---- work range of this CTA (split by work: slices x tiles)
-  const int last_slices = a.n_slices - (a.groups - 1) * W;
-  const int64_t total = gv_work_before(a.n_items, a.tiles, W, last_slices, a.groups);
-  const int64_t i_begin = gv_item_at(total * blockIdx.x / gridDim.x, a.tiles, W, last_slices, a.groups);
-  const int64_t i_end = gv_item_at(total * (blockIdx.x + 1) / gridDim.x, a.tiles, W, last_slices, a.groups);
-  if (i_begin >= i_end) return;                                      // CTA-uniform
-  const int n_local = static_cast<int>(i_end - i_begin);
-
-  // ---- shared-memory layout: the table on the first 64 KB boundary of the
-  // window, code stages in 2 KB slots below and above it, barriers last
+  // contiguous 1024-aligned stages at the start of s_raw, the table on the
+  // next 64 KB boundary of the window after them
   const uint32_t raw = smem_u32(s_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
-  const int below = static_cast<int>((lut - base) / kGvTileBytes);  // slots that fit under the table
-  auto slot_addr = [&](int k) -> uint32_t {
-    return k < below ? base + k * kGvTileBytes : lut + kGvLutBytes + (k - below) * kGvTileBytes;
-  };
-  const uint32_t bar_base = slot_addr(C::SLOTS);
-  const uint32_t end = max(bar_base + C::SLOTS * 8, lut + kGvLutBytes);
-  if (end > raw + C::SMEM || lut >= (1u << 24)) {                    // cannot place them (CTA-uniform)
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  const uint32_t lut = (sbase + kGvStages * kGvStageBytes + 0xFFFFu) & ~0xFFFFu;
+  if (lut + kGvLutBytes > raw + kGvSmem || lut >= (1u << 24)) {     // cannot place them (CTA-uniform)
     if (threadIdx.x == 0) raise_device_error(3);
     return;
   }
-  auto full_bar = [&](int s) -> uint32_t { return bar_base + (warp * kGvStages + s) * 8; };
-
-  if (lane == 0) {
-    for (int s = 0; s < kGvStages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(full_bar(s)) : "memory");
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGvStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kGvWarps);
+    }
     fence_mbar_init();
   }
-  // level-pair table: row b (a code byte) holds bf16(level[b & 15]) | bf16(level[b >> 4]) << 16, one copy per lane
-  for (int e = threadIdx.x; e < 256 * 32; e += C::THREADS) {
+  for (int e = threadIdx.x; e < 256 * 32; e += kGvThreads) {
     const int b = e >> 5, l = e & 31;
     const uint32_t v = pack_bf16x2_rn(a.L.v[b & 15], a.L.v[b >> 4]);
     asm volatile("st.shared.u32 [%0], %1;" :: "r"(lut + b * 256 + l * 4), "r"(v) : "memory");
   }
   __syncthreads();
 
-  // register table of the rows g + 8: bf16(level[j] * 1)
-  const Nf4Table rt = make_table(a.L, 1.0f);
+  // Unit tiles: thread 0 issues unit i's loads into stage i % kGvStages once
+  // every warp has released the unit that used that stage before.
+  const bool producer = threadIdx.x == 0;
+  int p_issued = 0, p_st = st_first, p_t = t_first;
+  bool p_ok = true;
+  auto produce_until = [&](int limit) {                            // issue loads of units < limit
+    for (; p_ok && p_issued < limit && p_issued < n_local; ++p_issued) {
+      const int s = p_issued % kGvStages;
+      if (p_issued >= kGvStages &&
+          !mbar_wait_bounded(&empty_bar[s], ((p_issued / kGvStages) + 1) & 1, a.timeout_ns)) {
+        raise_device_error(1);
+        p_ok = false;
+        break;
+      }
+      const uint32_t dst = sbase + s * kGvStageBytes;
+      mbar_arrive_expect_tx(&full_bar[s], kTxBytes);
+      tma_load_2d(dst, &tm_codes, &full_bar[s], p_st * (kGvStageK / 2), p_t * kGvRows);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        tma_load_2d(dst + kGvCodeBytes + j * (kGvXBox * 2 * XR), &tm_x, &full_bar[s],
+                    p_st * kGvStageK + j * kGvXBox, 0);
+      if (++p_st == a.n_st) { p_st = 0; ++p_t; }
+    }
+  };
+  if (producer) {
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_x);
+    produce_until(kGvStages - 1);
+  }
+
+  const int g = lane >> 2, q = lane & 3;
   uint32_t lane_key;                                                 // bytes 0 and 2 of every table address
   asm volatile("mov.b32 %0, %1;" : "=r"(lane_key) : "r"(lut | static_cast<uint32_t>(lane * 4)) : "memory");
-
-  const int row_blocks = a.in / 64;
-  const float mu = __ldg(a.mean);
-
-  // (group, tile) of an item, advanced item by item (no division in the loop)
-  struct ItemPos { int grp, tile; };
-  const ItemPos first{static_cast<int>(i_begin / a.tiles), static_cast<int>(i_begin % a.tiles)};
-  auto advance = [&](ItemPos p) -> ItemPos {
-    if (++p.tile == a.tiles) { p.tile = 0; ++p.grp; }
-    return p;
-  };
-  auto active_in = [&](int grp) { return grp * W + warp < a.n_slices; };
-
-  // ---- TMA issue of item `it` (at position p) into stage it % kGvStages (lane 0)
-  auto issue = [&](int it, ItemPos p) -> bool {
-    if (it >= n_local || !active_in(p.grp)) return false;
-    const int s = it % kGvStages;
-    const uint32_t dst = slot_addr(warp * kGvStages + s);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                 :: "r"(full_bar(s)), "r"(kGvTileBytes) : "memory");
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        :: "r"(dst), "l"(&tm_codes), "r"((p.grp * W + warp) * (kGvSlice / 2)), "r"(p.tile * kGvTile),
-           "r"(full_bar(s)) : "memory");
-    return true;
-  };
-  // lane 0: the next item to issue, its position, and how many loads were
-  // issued (the warp's active items are a prefix of the CTA's range)
-  int next_issue = 0, n_issued = 0;
-  ItemPos issue_pos = first;
-  if (lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" :: "l"(&tm_codes) : "memory");
-    for (; next_issue < kGvStages; ++next_issue) {
-      n_issued += issue(next_issue, issue_pos) ? 1 : 0;
-      issue_pos = advance(issue_pos);
-    }
-  }
-
-  // stage-relative read offsets (128-byte swizzle): codes of row g (row g+8: + 1024)
-  // for block j: 8 bytes at byte 32 j + 8 q of the row's 128
+  const int row_in_tile0 = warp * 16 + g;
+  const bool tok0 = g < a.M, tok1 = kTwoTok && g + 8 < a.M;
+  // stage-relative read offsets: codes of row g, block j (row g+8: + 1024);
+  // activation chunks 2q, 2q+1 of token g (token g+8: + 1024)
   uint32_t coff[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int c = 2 * j + (q >> 1);
-    coff[j] = static_cast<uint32_t>(g * 128 + (((c ^ g) & 7) << 4) + (q & 1) * 8);
-  }
+  for (int j = 0; j < 4; ++j) coff[j] = gv_swz128(row_in_tile0, 2 * j + (q >> 1), q & 1);
+  const uint32_t xoff0 = kGvCodeBytes + gv_swz128(g, 2 * q, 0);
+  const uint32_t xoff1 = kGvCodeBytes + gv_swz128(g, 2 * q + 1, 0);
+  constexpr uint32_t kXBlk = kGvXBox * 2 * XR;                       // bytes per activation box
 
-  // activations of this warp's slice (per block j: 16 consecutive columns
-  // 64 j + 16 q .. +15 of tokens g and g + 8), loaded when the group changes
-  uint32_t xa[4][8], xc[4][8];
-  int cur_grp = -1;
-  auto load_x = [&](int grp) {
-    const int c0 = (grp * W + warp) * kGvSlice;
+  const int64_t row_blocks = a.in / 64;
+  const float mu = __ldg(a.mean);
+
+  // Block scales are computed once per (row, block) and shared through the
+  // free upper half of the table's rows: lane l of a warp handles row
+  // (l % 16) of the warp's 16 and blocks 2 (l / 16), 2 (l / 16) + 1 of the
+  // unit, writes them to its warp's 256-byte slot (rows 0-7 in table row
+  // 2 warp, rows 8-15 in 2 warp + 1, 16 bytes per row) and reads back the
+  // four scales of rows g and g+8.
+  const int srow = lane & 15, spair = lane >> 4;
+  const uint32_t s_st = lut + (2 * warp + (srow >> 3)) * 256 + 128 + (srow & 7) * 16 + spair * 8;
+  const uint32_t s_ld = lut + 2 * warp * 256 + 128 + g * 16;         // row g; row g+8: + 256
+  int rs = t_first * kGvRows + warp * 16 + srow;                    // this lane's scale row
+  const int8_t* qp = a.q8 + static_cast<int64_t>(rs) * row_blocks + 4 * st_first + 2 * spair;
+  const int64_t b_wrap = kGvRows * row_blocks - 4 * static_cast<int64_t>(a.n_st);
+  // paired: the two q8 codes of the next unit (each byte XOR 0x80), cached group step
+  uint32_t qn = 0x8080u;
+  float sv = 0.f;
+  if (kPaired && rs < a.out) qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(qp))) ^ 0x8080u;
+
+  float acc[2][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+  int t = t_first, st = st_first;
+  int s = 0;
+  uint32_t phase = 0, sb = sbase;
+  bool new_row = true;                                               // group steps to (re)load
+  for (int i = 0; i < n_local; ++i) {
+    const bool ok = mbar_wait_bounded(&full_bar[s], phase, a.timeout_ns);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {                              // warp-uniform give-up
+      if (lane == 0) raise_device_error(1);
+      break;
+    }
+    uint2 cg[4], ch[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const int col = c0 + 64 * j + 16 * q;
-      const bool cok = col < a.in;
-#pragma unroll
-      for (int t2 = 0; t2 < (kTok2 ? 2 : 1); ++t2) {
-        const int tok = g + 8 * t2;
-        uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
-        if (cok && tok < a.M) {
-          const uint16_t* p = a.x + static_cast<int64_t>(tok) * a.in + col;
-          v0 = gv_ldg128(p);
-          v1 = gv_ldg128(p + 8);
-        }
-        if (t2 == 0) {
-          xa[j][0] = v0.x; xa[j][1] = v0.y; xa[j][2] = v0.z; xa[j][3] = v0.w;
-          xa[j][4] = v1.x; xa[j][5] = v1.y; xa[j][6] = v1.z; xa[j][7] = v1.w;
-        } else {
-          xc[j][0] = v0.x; xc[j][1] = v0.y; xc[j][2] = v0.z; xc[j][3] = v0.w;
-          xc[j][4] = v1.x; xc[j][5] = v1.y; xc[j][6] = v1.z; xc[j][7] = v1.w;
-        }
-      }
+      cg[j] = gv_lds64(sb + coff[j]);
+      ch[j] = gv_lds64(sb + coff[j] + 1024);
     }
-  };
 
-  // scale codes of this quad lane's block in rows g and g + 8 of an item's
-  // tile (code 0 and step 0 past the K end), fetched one item ahead
-  struct ScaleIn { int q0, q1; float st0, st1; };
-  auto fetch_scales = [&](int it, ItemPos p, ScaleIn& f) {
-    f.q0 = f.q1 = 0;
-    f.st0 = f.st1 = 0.f;
-    if (it >= n_local) return;
-    const int blk = (p.grp * W + warp) * 4 + q;
-    if (blk >= row_blocks) return;
-    const int64_t b0 = static_cast<int64_t>(p.tile * kGvTile + g) * row_blocks + blk;
-    const int64_t b1 = b0 + 8ll * row_blocks;
-    f.q0 = __ldg(a.q8 + b0);
-    f.q1 = __ldg(a.q8 + b1);
-    f.st0 = __ldg(a.step2 + (b0 >> 8));
-    f.st1 = __ldg(a.step2 + (b1 >> 8));
-  };
-  ScaleIn nxt;
-  fetch_scales(0, first, nxt);
+    const int col0 = st * kGvStageK;
+    const bool last_in_tile = st == a.n_st - 1;
 
-  const uint32_t red_base = lut + 128;                               // upper half of every table row
-  bool ok_all = true;
-  int stuck = n_local;                                               // first item not consumed
-  ItemPos pos = first;
-  ItemPos round_first = first;                                       // position of the round's first item
-  for (int it = 0; it < n_local; ++it, pos = advance(pos)) {
-    const int grp = pos.grp;
-    const bool act = active_in(grp);
-    if (it % C::RED_ITEMS == 0) round_first = pos;
-    float d[2][4];
-#pragma unroll
-    for (int t2 = 0; t2 < 2; ++t2) d[t2][0] = d[t2][1] = d[t2][2] = d[t2][3] = 0.f;
-    if (act && ok_all) {
-      if (grp != cur_grp) {
-        load_x(grp);
-        cur_grp = grp;
-      }
-      // this lane's two block scales (exchanged with its quad below); the
-      // next item's codes are fetched now
-      const ScaleIn cur = nxt;
-      fetch_scales(it + 1, advance(pos), nxt);
-      const float s0 = block_scale(cur.q0, cur.st0, mu);
-      const float s1 = block_scale(cur.q1, cur.st1, mu);
-      const int s = it % kGvStages;
-      const bool landed = gv_wait(full_bar(s), static_cast<uint32_t>((it / kGvStages) & 1), a.timeout_ns);
-      if (!__all_sync(0xFFFFFFFFu, landed)) {                        // warp-uniform give-up
-        if (lane == 0) raise_device_error(1);
-        ok_all = false;
-        stuck = it;
-      } else {
-        const uint32_t sb = slot_addr(warp * kGvStages + s);
-        uint2 cg[4], ch[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          cg[j] = gv_lds64(sb + coff[j]);
-          ch[j] = gv_lds64(sb + coff[j] + 1024);
-        }
-        // the stage is read: hand it back to the copy engine for item it + kGvStages
-        __syncwarp();
-        if (lane == 0) {
-          fence_proxy_async_smem();
-          n_issued += issue(next_issue, issue_pos) ? 1 : 0;          // item it + kGvStages
-          ++next_issue;
-          issue_pos = advance(issue_pos);
-        }
-        float sc0[4], sc1[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          sc0[j] = __shfl_sync(0xFFFFFFFFu, s0, (lane & ~3) | j);
-          sc1[j] = __shfl_sync(0xFFFFFFFFu, s1, (lane & ~3) | j);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float pb[2][4];
-#pragma unroll
-          for (int st = 0; st < 4; ++st) {
-            const uint32_t wg = st < 2 ? cg[j].x : cg[j].y;
-            const uint32_t wh = st < 2 ? ch[j].x : ch[j].y;
-            const int bi = (2 * st) & 3;                             // byte of the column pair 4 st, 4 st + 1
-            const uint32_t a0 = gv_lds(prmt(wg, lane_key, 0x7604u | (bi << 4)));
-            const uint32_t a2 = gv_lds(prmt(wg, lane_key, 0x7604u | ((bi + 1) << 4)));
-            uint32_t a1, a3;
-            if (st < kRegSteps) {
-              decode4(rt, wh >> (8 * bi), a1, a3);                   // ALU: register table
-            } else {
-              a1 = gv_lds(prmt(wh, lane_key, 0x7604u | (bi << 4)));  // load/store unit: shared table
-              a3 = gv_lds(prmt(wh, lane_key, 0x7604u | ((bi + 1) << 4)));
-            }
-            if (st == 0) {
-              pb[0][0] = pb[0][1] = pb[0][2] = pb[0][3] = 0.f;
-              pb[1][0] = pb[1][1] = pb[1][2] = pb[1][3] = 0.f;
-            }
-            gv_mma(pb[0], a0, a1, a2, a3, xa[j][2 * st], xa[j][2 * st + 1]);
-            if (kTok2) gv_mma(pb[1], a0, a1, a2, a3, xc[j][2 * st], xc[j][2 * st + 1]);
-          }
-#pragma unroll
-          for (int t2 = 0; t2 < (kTok2 ? 2 : 1); ++t2) {
-            d[t2][0] = fmaf(pb[t2][0], sc0[j], d[t2][0]);
-            d[t2][1] = fmaf(pb[t2][1], sc0[j], d[t2][1]);
-            d[t2][2] = fmaf(pb[t2][2], sc1[j], d[t2][2]);
-            d[t2][3] = fmaf(pb[t2][3], sc1[j], d[t2][3]);
-          }
-        }
-      }
-    }
-    // ---- this warp's partial tile into its reduction piece: value (row, tok)
-    // at byte 4 (row NT + tok) of the warp's NT/2 chunks of 128 B
-    const int k = it % C::RED_ITEMS;
+    // this lane's two block scales, then the eight of rows g and g+8
     {
-      const int chunk0 = (k * W + warp) * C::CHUNKS_PER_WARP;
+      const bool row_ok = rs < a.out;
+      float s0, s1;
+      if (kPaired) {
+        const uint32_t qc = qn;
+        const int8_t* q_next = last_in_tile ? qp + b_wrap + 4 : qp + 4;
+        const bool next_ok = last_in_tile ? rs + kGvRows < a.out : row_ok;
+        if (next_ok && i + 1 < n_local)
+          qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(q_next))) ^ 0x8080u;
+        // a unit's four blocks share one group; a group starts at a multiple of 256 blocks
+        const int64_t b_unit = (qp - a.q8) - 2 * spair;
+        if (row_ok && (new_row || (static_cast<uint32_t>(b_unit) & 255u) == 0)) sv = __ldg(a.step2 + (b_unit >> 8));
+        // exact floats of the signed codes: 2^23 + (q + 128) - (2^23 + 128)
+        const float q0 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7650u)), -8388736.0f);
+        const float q1 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7651u)), -8388736.0f);
+        s0 = __fadd_rn(__fmul_rn(q0, sv), mu);
+        s1 = __fadd_rn(__fmul_rn(q1, sv), mu);
+      } else {
+        const int c0 = col0 + 128 * spair;
+        const bool l0 = row_ok && c0 < a.in, l1 = row_ok && c0 + 64 < a.in;
+        const int64_t b = qp - a.q8;
+        s0 = block_scale(l0 ? __ldg(qp) : 0, l0 ? __ldg(a.step2 + (b >> 8)) : 0.f, mu);
+        s1 = block_scale(l1 ? __ldg(qp + 1) : 0, l1 ? __ldg(a.step2 + ((b + 1) >> 8)) : 0.f, mu);
+      }
+      asm volatile("st.shared.v2.f32 [%0], {%1, %2};" :: "r"(s_st), "f"(s0), "f"(s1) : "memory");
+    }
+    __syncwarp();
+    float sc[2][4];
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(sc[0][0]), "=f"(sc[0][1]), "=f"(sc[0][2]), "=f"(sc[0][3]) : "r"(s_ld) : "memory");
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(sc[1][0]), "=f"(sc[1][1]), "=f"(sc[1][2]), "=f"(sc[1][3]) : "r"(s_ld + 256) : "memory");
+    new_row = false;
+
 #pragma unroll
-      for (int t2 = 0; t2 < (kTok2 ? 2 : 1); ++t2) {
+    for (int blk = 0; blk < 4; ++blk) {
+      if (kPaired || blk == 0 || col0 + 64 * blk < a.in) {
+        // activations: 16 consecutive columns 64 blk + 16q .. +15 of token rows g, g+8
+        uint4 xa0 = make_uint4(0, 0, 0, 0), xa1 = xa0, xc0 = xa0, xc1 = xa0;
+        if (tok0) {
+          xa0 = gv_lds128(sb + xoff0 + blk * kXBlk);
+          xa1 = gv_lds128(sb + xoff1 + blk * kXBlk);
+        }
+        if (tok1) {
+          xc0 = gv_lds128(sb + xoff0 + blk * kXBlk + 1024);
+          xc1 = gv_lds128(sb + xoff1 + blk * kXBlk + 1024);
+        }
+        const uint32_t xa[8] = {xa0.x, xa0.y, xa0.z, xa0.w, xa1.x, xa1.y, xa1.z, xa1.w};
+        const uint32_t xc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
+        const uint32_t wg[2] = {cg[blk].x, cg[blk].y}, wh[2] = {ch[blk].x, ch[blk].y};
+        float pb[2][4];
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {     // columns 64 blk + 16q + 4 s4 .. +3: bytes 2 s4, 2 s4 + 1
+          const uint32_t sel_lo = 0x7604u | ((2 * (s4 & 1)) << 4);
+          const uint32_t sel_hi = 0x7604u | ((2 * (s4 & 1) + 1) << 4);
+          const uint32_t e0 = gv_lds(prmt(wg[s4 >> 1], lane_key, sel_lo));
+          const uint32_t e1 = gv_lds(prmt(wh[s4 >> 1], lane_key, sel_lo));
+          const uint32_t e2 = gv_lds(prmt(wg[s4 >> 1], lane_key, sel_hi));
+          const uint32_t e3 = gv_lds(prmt(wh[s4 >> 1], lane_key, sel_hi));
+          // a0: row g columns +0,+1; a1: row g+8 same; a2, a3: columns +2,+3
+          if (s4 == 0) {
+            gv_mma_z(pb[0], e0, e1, e2, e3, xa[0], xa[1]);
+            if (kTwoTok) gv_mma_z(pb[1], e0, e1, e2, e3, xc[0], xc[1]);
+          } else {
+            gv_mma(pb[0], e0, e1, e2, e3, xa[2 * s4], xa[2 * s4 + 1]);
+            if (kTwoTok) gv_mma(pb[1], e0, e1, e2, e3, xc[2 * s4], xc[2 * s4 + 1]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < (kTwoTok ? 2 : 1); ++j) {
+          acc[j][0] = fmaf(pb[j][0], sc[0][blk], acc[j][0]);
+          acc[j][1] = fmaf(pb[j][1], sc[0][blk], acc[j][1]);
+          acc[j][2] = fmaf(pb[j][2], sc[1][blk], acc[j][2]);
+          acc[j][3] = fmaf(pb[j][3], sc[1][blk], acc[j][3]);
+        }
+      }
+    }
+    // the stage (codes and activations) is no longer read by this warp
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+    if (producer) produce_until(i + kGvStages);                     // refill the stage of unit i - 1
+
+    // end of this CTA's part of tile t: write the partial and restart
+    if (last_in_tile || i == n_local - 1) {
+      float* dst = a.part + ((static_cast<int64_t>(blockIdx.x) * a.local_tiles + (t - t_first)) * a.M) * kGvRows;
+#pragma unroll
+      for (int j = 0; j < (kTwoTok ? 2 : 1); ++j) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          const int off = ((g + 8 * hh) * NT + 8 * t2 + 2 * q) * 4;
-          const uint32_t addr = red_base + (chunk0 + (off >> 7)) * 256 + (off & 127);
-          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" :: "r"(addr), "f"(d[t2][2 * hh]), "f"(d[t2][2 * hh + 1])
-                       : "memory");
+          const int tk = 8 * j + 2 * q + hh;
+          if (tk < a.M) {
+            dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0] = acc[j][hh];
+            dst[static_cast<int64_t>(tk) * kGvRows + row_in_tile0 + 8] = acc[j][2 + hh];
+          }
         }
+        acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
       }
     }
-    if (k != C::RED_ITEMS - 1 && it != n_local - 1) continue;
-
-    // ---- reduction round over items it0 .. it (CTA-uniform)
-    __syncthreads();
-    const int n_round = k + 1;
-    for (int u = threadIdx.x; u < n_round * kGvTile * NT; u += C::THREADS) {
-      const int kk = u / (kGvTile * NT), v = u % (kGvTile * NT);
-      const int row = v / NT, tok = v % NT;
-      float sum = 0.f;
-#pragma unroll 4
-      for (int w = 0; w < W; ++w) {
-        const int off = v * 4;
-        float t;
-        asm volatile("ld.shared.f32 %0, [%1];" : "=f"(t)
-                     : "r"(red_base + ((kk * W + w) * C::CHUNKS_PER_WARP + (off >> 7)) * 256 + (off & 127))
-                     : "memory");
-        sum += t;
-      }
-      if (tok < a.M) {
-        ItemPos ip = round_first;
-        for (int j = 0; j < kk; ++j) ip = advance(ip);
-        const int gi = ip.grp, ti = ip.tile;
-        const int o = ti * kGvTile + row;
-        if (a.groups == 1)
-          a.h[static_cast<int64_t>(tok) * a.out + o] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(sum + gv_lora(a.us, a.B, tok, o, a.r)));
-        else
-          a.part[(static_cast<int64_t>(gi) * a.out + o) * a.M + tok] = sum;
-      }
-    }
-    __syncthreads();                                                 // the pieces are reused
+    qp += 4;
+    if (++st == a.n_st) { st = 0; ++t; rs += kGvRows; qp += b_wrap; new_row = true; }
+    sb += kGvStageBytes;
+    if (++s == kGvStages) { s = 0; phase ^= 1u; sb = sbase; }
   }
-
-  // leave no copy in flight when the CTA exits: after a give-up at item
-  // `stuck`, the stages of items stuck .. stuck + kGvStages - 1 may have been
-  // issued and not consumed; wait for them, bounded
-  if (lane == 0 && stuck < n_local) {
-    for (int it = stuck; it < n_issued; ++it)                        // the issued loads are items 0 .. n_issued - 1
-      gv_wait(full_bar(it % kGvStages), static_cast<uint32_t>((it / kGvStages) & 1), a.timeout_ns);
-  }
+  // leave no copy in flight when the CTA exits (only on a give-up path can
+  // issued loads still be unconsumed): wait, bounded, for the last ones
+  if (producer)
+    for (int j = p_issued > kGvStages ? p_issued - kGvStages : 0; j < p_issued; ++j)
+      if (!mbar_wait_bounded(&full_bar[j % kGvStages], (j / kGvStages) & 1, a.timeout_ns)) raise_device_error(1);
 }
 
-// h[m][o] = bf16( sum over the K groups, in group order, of part[g][o][m]
-//                 + sum_j us[m][j] * B[o][j] ),  m < M (K split over groups).
-__global__ void __launch_bounds__(256) gemv_finalize_kernel(const float* __restrict__ part, int groups, int M,
-                                                            int out, const uint16_t* __restrict__ us,
-                                                            const uint16_t* __restrict__ B, int r,
-                                                            uint16_t* __restrict__ h) {
+// h[m][o] = bf16( sum of the partials of o's tile, in CTA order
+//                 + sum_j us[m][j] * B[o][j] ),  m < M.
+__global__ void __launch_bounds__(256) gemv_finalize_kernel(
+    const float* __restrict__ part, int ctas, int local_tiles, int64_t n_units, int n_st, int M, int out,
+    const uint16_t* __restrict__ us, const uint16_t* __restrict__ B, int r, uint16_t* __restrict__ h) {
   const int64_t n_el = static_cast<int64_t>(M) * out;
   for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_el;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int o = static_cast<int>(e / M), m = static_cast<int>(e % M);
+    const int m = static_cast<int>(e / out), o = static_cast<int>(e % out);
+    const int t = o / kGvRows, row = o % kGvRows;
+    // CTA holding the tile's first unit: the largest c with begin(c) <= t * n_st
+    const int64_t u = static_cast<int64_t>(t) * n_st;
+    int64_t c = u * ctas / n_units;
+    while (c + 1 < ctas && gemv_unit_begin(c + 1, n_units, ctas) <= u) ++c;
+    while (c > 0 && gemv_unit_begin(c, n_units, ctas) > u) --c;
     float v = 0.f;
-    for (int gg = 0; gg < groups; ++gg) v += __ldg(part + static_cast<int64_t>(gg) * n_el + e);
-    h[static_cast<int64_t>(m) * out + o] = __bfloat16_as_ushort(__float2bfloat16_rn(v + gv_lora(us, B, m, o, r)));
+    for (; c < ctas; ++c) {
+      const int64_t b = gemv_unit_begin(c, n_units, ctas);
+      if (b >= u + n_st) break;                                     // past this tile
+      if (gemv_unit_begin(c + 1, n_units, ctas) <= b) continue;     // empty CTA
+      const int lt = t - static_cast<int>(b / n_st);
+      v += __ldg(part + ((c * local_tiles + lt) * M + m) * static_cast<int64_t>(kGvRows) + row);
+    }
+    const uint16_t* ur = us + static_cast<int64_t>(m) * r;
+    const uint16_t* br = B + static_cast<int64_t>(o) * r;
+    float l = 0.f;
+    for (int j = 0; j < r; j += 8) {
+      const uint4 ua = __ldg(reinterpret_cast<const uint4*>(ur + j));
+      const uint4 ba = __ldg(reinterpret_cast<const uint4*>(br + j));
+      const uint32_t uw[4] = {ua.x, ua.y, ua.z, ua.w}, bw[4] = {ba.x, ba.y, ba.z, ba.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[i]));
+        const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
+        l = fmaf(uf.x, bf.x, l);
+        l = fmaf(uf.y, bf.y, l);
+      }
+    }
+    h[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v + l));
   }
 }
 

@@ -24,8 +24,11 @@
 // partials in rank order (deterministic), and stores it.
 //
 // Roles (128 threads): warp 0 lane 0 issues the TMA loads, warp 1 allocates
-// tensor memory and its lane 0 issues the MMAs; afterwards the four warps
-// read the accumulator (warp w owns rows 32 w .. 32 w + 31, its TMEM lanes).
+// tensor memory and its lane 0 issues the MMAs, and with a LoRA-dropout keep
+// mask warps 2 and 3 zero the dropped activations of each landed stage in
+// shared memory (bit c % 8 of byte c / 8 of a token's row keeps column c)
+// before the MMAs read it; afterwards the four warps read the accumulator
+// (warp w owns rows 32 w .. 32 w + 31, its TMEM lanes).
 // Every wait is bounded: on timeout the CTA sets the device error flag,
 // issues nothing more, waits (bounded) for what it issued and exits.
 // No TMA multicast is used.
@@ -36,7 +39,7 @@
 namespace qnf4 {
 
 constexpr int kLrThreads = 128;
-constexpr int kLrStages = 4;
+constexpr int kLrMaxStages = 8;
 constexpr int kLrTileRows = 128;
 constexpr int kLrAStage = kLrTileRows * 64 * 2;           // 16 KB: 128 rows x 64 k (or two 64-wide MN atoms)
 
@@ -53,6 +56,8 @@ struct LrProblem {
   int tiles;             // ceil(rows / 128)
   int transpose_out;     // col form: write D^T (dA [r, in])
   float scale;
+  const uint8_t* keep;   // LoRA dropout keep bits of the token operand [tokens, features / 8], or null
+  int features;          // columns of the token operand (row form: K; col form: rows)
 };
 
 struct LrArgs {
@@ -62,6 +67,7 @@ struct LrArgs {
   int N;                 // r rounded up to 16
   int n_alloc;           // TMEM columns (power of two >= 32, >= N)
   int stages_per_split;  // 64-wide contraction stages per CTA of the cluster
+  int ring;              // shared-memory stages in flight (<= kLrMaxStages)
   uint64_t timeout_ns;
 };
 
@@ -71,10 +77,10 @@ __host__ __device__ constexpr int lr_b_stage(int N, bool b_mn_major) {
   return b_mn_major ? ((N + 63) / 64) * 8192 : ((N * 128 + 1023) / 1024) * 1024;
 }
 __host__ __device__ constexpr int lr_partial_pitch(int N) { return N * 4 + 16; }
-__host__ __device__ constexpr int lr_smem_bytes(int N, bool b_mn_major) {
-  const int ring = kLrStages * (kLrAStage + lr_b_stage(N, b_mn_major));
+__host__ __device__ constexpr int lr_smem_bytes(int N, bool b_mn_major, int stages) {
+  const int ring = stages * (kLrAStage + lr_b_stage(N, b_mn_major));
   const int part = kLrTileRows * lr_partial_pitch(N);
-  return (ring > part ? ring : part) + 256 + 1024;
+  return (ring > part ? ring : part) + 512 + 1024;
 }
 
 // kCol: col form (A MN-major, output fp32); otherwise row form (A K-major,
@@ -88,14 +94,16 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   const int N = args.N;
   const int b_stage = lr_b_stage(N, kBMN);
-  const int ring_bytes = kLrStages * (kLrAStage + b_stage);
+  const int S = args.ring;                                           // stages of the ring
+  const int ring_bytes = S * (kLrAStage + b_stage);
   const int part_bytes = kLrTileRows * lr_partial_pitch(N);
   uint8_t* a_ring = smem;
-  uint8_t* b_ring = smem + kLrStages * kLrAStage;
+  uint8_t* b_ring = smem + S * kLrAStage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (ring_bytes > part_bytes ? ring_bytes : part_bytes));
   uint64_t* full = bars;
-  uint64_t* empty = bars + kLrStages;
-  uint64_t* acc_full = bars + 2 * kLrStages;
+  uint64_t* empty = bars + kLrMaxStages;
+  uint64_t* masked = bars + 2 * kLrMaxStages;                        // (keep mask) the stage is masked
+  uint64_t* acc_full = bars + 3 * kLrMaxStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acc_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -106,6 +114,9 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
   const int p_rows = prob == 0 ? args.p[0].rows : args.p[1].rows;
   const bool p_transpose = (prob == 0 ? args.p[0].transpose_out : args.p[1].transpose_out) != 0;
   const float p_scale = prob == 0 ? args.p[0].scale : args.p[1].scale;
+  const uint8_t* const p_keep = prob == 0 ? args.p[0].keep : args.p[1].keep;
+  const int p_features = prob == 0 ? args.p[0].features : args.p[1].features;
+  const bool do_mask = p_keep != nullptr;                            // CTA-uniform
   const int tile = prob == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - args.p[0].tiles;
   const CUtensorMap* tm_a = prob == 0 ? &tm_a0 : &tm_a1;
   const CUtensorMap* tm_b = prob == 0 ? &tm_b0 : &tm_b1;
@@ -119,9 +130,10 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
   const uint64_t tmo = args.timeout_ns;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kLrStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
+      mbar_init(masked + s, 2);                                      // one arrive per masking warp
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -152,8 +164,8 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
       tma_prefetch_desc(tm_b);
       int issued = 0;
       for (int it = 0; it < n_iter; ++it) {
-        const int s = it % kLrStages;
-        wait(empty + s, ((it / kLrStages) & 1u) ^ 1u);
+        const int s = it % S;
+        wait(empty + s, ((it / S) & 1u) ^ 1u);
         if (*abort_flag) break;
         mbar_arrive_expect_tx(full + s, stage_tx);
         const uint32_t a_dst = smem_u32(a_ring + s * kLrAStage);
@@ -172,17 +184,18 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
         }
         ++issued;
       }
-      // only the last kLrStages issued stages can still be in flight
-      for (int it = issued > kLrStages ? issued - kLrStages : 0; it < issued; ++it)
-        mbar_wait_bounded(full + (it % kLrStages), (it / kLrStages) & 1u, tmo);
+      // only the last S issued stages can still be in flight
+      for (int it = issued > S ? issued - S : 0; it < issued; ++it)
+        mbar_wait_bounded(full + (it % S), (it / S) & 1u, tmo);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       const uint32_t idesc = umma_idesc_bf16_ab(kLrTileRows, N, kCol, kBMN);
       for (int it = 0; it < n_iter; ++it) {
-        const int s = it % kLrStages;
-        wait(full + s, (it / kLrStages) & 1u);
+        const int s = it % S;
+        wait(full + s, (it / S) & 1u);
+        if (do_mask) wait(masked + s, (it / S) & 1u);
         if (*abort_flag) break;
         tc_fence_after_sync();
         const uint32_t a_base = smem_u32(a_ring + s * kLrAStage);
@@ -199,6 +212,83 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
       }
       umma_commit(acc_full);
       mbar_wait_bounded(acc_full, 0, tmo);
+    }
+  } else if (do_mask) {
+    // ------------------------------------------------------------ keep mask
+    // Thread t (0..63) owns tile row t (row form: token row0 + t and +64;
+    // col form: token k0 + t of both 64-feature atoms) and zeroes, in
+    // each landed stage, the values whose keep bit is 0.
+    const int t = threadIdx.x - 64;
+    const int64_t kb_row = p_features / 8;                           // keep bytes per token
+    auto mask_chunk16 = [](uint32_t addr, uint32_t bits) {           // 8 bf16 at addr, bit e keeps value e
+      uint32_t v[4];
+      asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                   : "r"(addr) : "memory");
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        v[e] &= ((bits >> (2 * e)) & 1u ? 0x0000FFFFu : 0u) | ((bits >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u);
+      sts_v4(addr, v[0], v[1], v[2], v[3]);
+    };
+    // this thread's keep bytes of stage `it` (zero past the token or feature end)
+    auto load_keep = [&](int it, uint2 (&kb)[2]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        kb[h] = make_uint2(0u, 0u);
+        if (it >= n_iter) continue;
+        const int k0 = (st_begin + it) * 64;
+        int64_t tok, f0;
+        if (!kCol) { tok = row0 + t + 64 * h; f0 = k0; }
+        else { tok = k0 + t; f0 = row0 + 64 * h; }
+        const int64_t n_tok = kCol ? args.K : p_rows;
+        if (tok < n_tok && f0 < p_features) {                         // keep bits are 4-byte aligned
+          const uint32_t* src = reinterpret_cast<const uint32_t*>(p_keep + tok * kb_row + f0 / 8);
+          kb[h] = make_uint2(__ldg(src), __ldg(src + 1));
+        }
+      }
+    };
+    // loaded into registers two stages ahead and brought into L2 six stages
+    // ahead, so their latency overlaps the stream
+    auto prefetch_keep = [&](int it) {
+      if (it >= n_iter) return;
+      const int k0 = (st_begin + it) * 64;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int64_t tok, f0;
+        if (!kCol) { tok = row0 + t + 64 * h; f0 = k0; }
+        else { tok = k0 + t; f0 = row0 + 64 * h; }
+        const int64_t n_tok = kCol ? args.K : p_rows;
+        if (tok < n_tok && f0 < p_features)
+          asm volatile("prefetch.global.L2 [%0];" :: "l"(p_keep + tok * kb_row + f0 / 8));
+      }
+    };
+    for (int i = 2; i < 6; ++i) prefetch_keep(i);
+    uint2 kb_n1[2], kb_n2[2];
+    load_keep(0, kb_n1);
+    load_keep(1, kb_n2);
+    for (int it = 0; it < n_iter; ++it) {
+      const int s = it % S;
+      uint2 kb[2] = {kb_n1[0], kb_n1[1]};
+      kb_n1[0] = kb_n2[0];
+      kb_n1[1] = kb_n2[1];
+      load_keep(it + 2, kb_n2);
+      prefetch_keep(it + 6);
+      wait(full + s, (it / S) & 1u);
+      if (*abort_flag) break;
+      const uint32_t a_base = smem_u32(a_ring + s * kLrAStage);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // row form: row t + 64 h of the 128-row tile; col form: row t of atom h
+        const int r = kCol ? t : t + 64 * h;
+        const uint32_t rbase = a_base + (kCol ? h * 8192 : 0) + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t bits = ((c < 4 ? kb[h].x : kb[h].y) >> (8 * (c & 3))) & 0xFFu;
+          if (bits != 0xFFu) mask_chunk16(rbase + (((c ^ r) & 7) << 4), bits);
+        }
+      }
+      fence_proxy_async_smem();                                     // generic writes before the MMAs read
+      __syncwarp();
+      if (lane == 0) mbar_arrive(masked + s);
     }
   }
 

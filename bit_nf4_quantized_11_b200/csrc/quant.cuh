@@ -270,42 +270,51 @@ __global__ void __launch_bounds__(256) dq_scales_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// K4: dequantize to bf16.  A thread handles 32 codes (16 bytes, half a block)
-// at a time -- block scale, the block's 16-entry bf16 table, prmt decode,
-// 64 bytes of bf16 out -- and loads kDqRounds such halves before decoding.
+// K4: dequantize to bf16.  A warp takes 128 consecutive 32-bit code words
+// (8 codes each, 1024 weights) per round; lane l decodes words l, l + 32,
+// l + 64, l + 96, so each of its four 16-byte output stores is part of one
+// 512-byte contiguous warp store, and each code load one 128-byte warp load.
+// A word's block scale and 16-entry bf16 table are built by its lane (the
+// eight lanes of a block share the scale code through a broadcast load).
+// kDqRounds rounds are loaded before any is decoded.
 // ---------------------------------------------------------------------------
-constexpr int kDqRounds = 4;
+constexpr int kDqRounds = 2;
 
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
     const uint8_t* __restrict__ codes, const int8_t* __restrict__ q8,
     const float* __restrict__ step2, const float* __restrict__ mean_ptr,
-    int64_t n_halves, uint16_t* __restrict__ out, Levels L) {
+    int64_t n_words, uint16_t* __restrict__ out, Levels L) {
   const float mu = *mean_ptr;
-  const int64_t n_thr = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (int64_t i0 = tid; i0 < n_halves; i0 += n_thr * kDqRounds) {
-    uint4 cw[kDqRounds];
-    float ch[kDqRounds];
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes);
+  for (int64_t base = warp * 128 * kDqRounds; base < n_words; base += n_warps * 128 * kDqRounds) {
+    uint32_t w[kDqRounds][4];
+    float ch[kDqRounds][4];
 #pragma unroll
     for (int rd = 0; rd < kDqRounds; ++rd) {
-      const int64_t i = i0 + rd * n_thr;
-      if (i < n_halves) {
-        const int64_t b = i >> 1;
-        cw[rd] = ld_stream_v4(codes + i * 16);
-        ch[rd] = block_scale(q8[b], step2[b / kGroup], mu);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t i = base + rd * 128 + k * 32 + lane;           // word index
+        if (i < n_words) {
+          const int64_t b = i >> 3;                                  // 8 words per 64-weight block
+          w[rd][k] = __ldcs(cw + i);
+          ch[rd][k] = block_scale(__ldg(q8 + b), __ldg(step2 + (b >> 8)), mu);
+        }
       }
     }
 #pragma unroll
     for (int rd = 0; rd < kDqRounds; ++rd) {
-      const int64_t i = i0 + rd * n_thr;
-      if (i < n_halves) {
-        const Nf4Table t = make_table(L, ch[rd]);
-        uint32_t o[4];
-        uint16_t* dst = out + i * 32;
-        decode8(t, cw[rd].x, o); st_v4(dst + 0, make_uint4(o[0], o[1], o[2], o[3]));
-        decode8(t, cw[rd].y, o); st_v4(dst + 8, make_uint4(o[0], o[1], o[2], o[3]));
-        decode8(t, cw[rd].z, o); st_v4(dst + 16, make_uint4(o[0], o[1], o[2], o[3]));
-        decode8(t, cw[rd].w, o); st_v4(dst + 24, make_uint4(o[0], o[1], o[2], o[3]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t i = base + rd * 128 + k * 32 + lane;
+        if (i < n_words) {
+          const Nf4Table t = make_table(L, ch[rd][k]);
+          uint32_t o[4];
+          decode8(t, w[rd][k], o);
+          st_v4(out + i * 8, make_uint4(o[0], o[1], o[2], o[3]));
+        }
       }
     }
   }

@@ -54,10 +54,10 @@ def test_dropout_layer_small(cuda_lib, M, n_in, n_out, r, alpha, p):
 
 
 def test_dropout_p0_all_kept_equals_plain_layer(cuda_lib):
-    """p = 0 with every element kept is the plain layer.  The masked calls
-    run their own rank-r kernels (another summation order), so the results
-    agree up to rounding: us to a bf16 ulp, the rest within the layer
-    tolerance."""
+    """p = 0 with every element kept is the plain layer, bit for bit in the
+    forward and in dA, dB (the same rank-r kernels run, the mask changes
+    nothing); dx takes one more bf16 rounding (the masked rank-r term is
+    added after the base GEMM)."""
     q = cuda_lib
     prob = synth.problem(256, 512, 384, 16, seed=3)
     dev = torch.device("cuda")
@@ -66,13 +66,10 @@ def test_dropout_p0_all_kept_equals_plain_layer(cuda_lib):
     keep_bits = torch.full((256, 64), 255, dtype=torch.uint8, device=dev)
     h0, us0 = q.linear_fwd(x, w, A, B, 32.0)
     h1, us1 = q.linear_fwd_dropout(x, w, A, B, 32.0, keep_bits, 0.0)
-    u0, u1 = to_np(us0), to_np(us1)
-    assert np.all(np.abs(u1 - u0) <= 2.0 ** -7 * np.abs(u0) + 1e-30)
-    assert_close(to_np(h1), to_np(h0), "h")
+    assert torch.equal(h0, h1) and torch.equal(us0, us1)
     dx0, dA0, dB0 = q.linear_bwd(dh, x, us0, w, A, B, 32.0)
     dx1, dA1, dB1 = q.linear_bwd_dropout(dh, x, us1, w, A, B, 32.0, keep_bits, 0.0)
-    assert_close(to_np(dA1), to_np(dA0), "dA")
-    assert_close(to_np(dB1), to_np(dB0), "dB")
+    assert torch.equal(dA0, dA1) and torch.equal(dB0, dB1)
     assert_close(to_np(dx1), to_np(dx0).astype(np.float64), "dx")   # dx differs by one extra rounding
 
 
