@@ -777,13 +777,19 @@ def comp_gemv(q, dev, peaks, n=60):
             torch.cuda.synchronize()
             q.timing_enable(False)
             kms, kn = q.timing_collect("gemv")
+            parts = {}
+            for name in ("lora_rowwise", "gemv", "gemv_finalize", "lora_pad"):
+                t_, n_ = q.timing_collect(name)
+                if n_:
+                    parts[name] = 1e3 * t_ / n
             wbytes = workloads.gemv_weight_bytes(n_out, n_in)
             gres[f"{label}_{n_in}x{n_out}_M{M}"] = {
                 "call_us": 1e3 * call_ms, "gemv_kernel_us": 1e3 * kms / kn if kn else None,
                 "packed_weight_GB/s_call": wbytes / (call_ms * 1e-3) / 1e9,
                 "frac_hbm_call": wbytes / (call_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "packed_weight_GB/s_kernel": wbytes / (kms / kn * 1e-3) / 1e9 if kn else None,
-                "frac_hbm_kernel": (wbytes / (kms / kn * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kn else None}
+                "frac_hbm_kernel": (wbytes / (kms / kn * 1e-3) / 1e9 / peaks["hbm_gbs"]) if kn else None,
+                "kernel_us_per_call": parts}
         del ws_list
         torch.cuda.empty_cache()
     return {"gemv_70b": gres}

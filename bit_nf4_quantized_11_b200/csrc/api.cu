@@ -753,10 +753,12 @@ int linear_bwd_impl(const uint16_t* dh, const uint16_t* x, const uint16_t* us, i
   rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);                // dx = dh W0
   if (rc != QLORA_OK) return rc;
   {
-    const int64_t units = cdiv(M, qnf4::kDxRows) * (in / 8);
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(cdiv(units, 256), device_sm_count() * 8)));
+    const int64_t tiles = cdiv(M, qnf4::kDxTileRows) * cdiv(in, qnf4::kDxTileCols);
+    const int smem = qnf4::dx_smem_bytes(r);
+    QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(qnf4::dropout_dx_kernel), smem));
     LaunchTimer lt_("dropout_dx", st);
-    qnf4::dropout_dx_kernel<<<grid, 256, 0, st>>>(dx, du, A, keep, M, in, r, inv_keep);  // + (du A) k/(1-p)
+    qnf4::dropout_dx_kernel<<<static_cast<unsigned>(tiles), qnf4::kDxThreads, smem, st>>>(dx, du, A, keep, M, in, r,
+                                                                                      inv_keep);  // + (du A) k/(1-p)
   }
   QLORA_CUDA_TRY(cudaGetLastError());
   return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st, inv_keep, keep);     // dB, dA

@@ -47,6 +47,7 @@ def _run(q, M, n_in, n_out, r, alpha, p, seed=0, sample_rows=None):
     (200, 256, 192, 136, 16.0, 0.2),
     (9, 1024, 768, 16, 32.0, 0.05),      # few-token path
     (300, 640, 320, 12, 24.0, 0.1),      # rank not a multiple of 8 (padded copies)
+    (130, 576, 320, 8, 16.0, 0.1),       # in % 128 == 64: a half-width column tile in the dx pass
     (7, 512, 384, 5, 10.0, 0.1),
 ])
 def test_dropout_layer_small(cuda_lib, M, n_in, n_out, r, alpha, p):
