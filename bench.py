@@ -219,6 +219,8 @@ class LayerState:
                             for n_in, n_out in self.shapes)
         self.ws_f = torch.empty(ws(q.OP_LINEAR_FWD), dtype=torch.uint8, device=dev)
         self.ws_b = torch.empty(ws(q.OP_LINEAR_BWD), dtype=torch.uint8, device=dev)
+        self.problems = self.make_problems(self.proj, [(c["dA"], c["dB"]) for c in self.proj])
+        self.ws_gf, self.ws_gb = self.group_workspaces(self.problems, dev)
         self.ws_q = torch.empty(max(q.workspace_size(q.OP_QUANTIZE, 0, n_in, n_out, 0) for n_in, n_out in self.shapes),
                                 dtype=torch.uint8, device=dev)
         self.quantize()
@@ -228,12 +230,32 @@ class LayerState:
         for c in self.proj:
             self.q.quantize_nf4(c["W"], out=c["w"], workspace=self.ws_q)
 
-    def step(self, world=1):
+    def make_problems(self, bufs, grads):
+        """One grouped-call problem per projection over the given x, dh, h,
+        us, dx buffers and (dA, dB) gradient views."""
+        return [self.q.LinearProblem(x=b["x"], w=c["w"], A=c["A"], B=c["B"], alpha=self.alpha, h=b["h"], us=b["us"],
+                                     dh=b["dh"], dx=b["dx"], dA=dA, dB=dB)
+                for c, b, (dA, dB) in zip(self.proj, bufs, grads)]
+
+    def group_workspaces(self, problems, dev):
+        q = self.q
+        return tuple(torch.empty(max(1, q.linear_group_workspace_size(bwd, problems)), dtype=torch.uint8, device=dev)
+                     for bwd in (False, True))
+
+    def step(self, world=1, grouped=True, problems=None):
+        """Forward and backward of every projection.  Grouped (the default):
+        two grouped calls, whose rank-r kernels run beside the GEMMs;
+        otherwise one linear_fwd + linear_bwd call per projection."""
         q, a = self.q, self.alpha
-        for c in self.proj:
-            q.linear_fwd(c["x"], c["w"], c["A"], c["B"], a, h=c["h"], us=c["us"], workspace=self.ws_f)
-            q.linear_bwd(c["dh"], c["x"], c["us"], c["w"], c["A"], c["B"], a, dx=c["dx"], dA=c["dA"], dB=c["dB"],
-                         workspace=self.ws_b)
+        if grouped:
+            probs = self.problems if problems is None else problems
+            q.linear_fwd_group(probs, workspace=self.ws_gf)
+            q.linear_bwd_group(probs, workspace=self.ws_gb)
+        else:
+            for c in self.proj:
+                q.linear_fwd(c["x"], c["w"], c["A"], c["B"], a, h=c["h"], us=c["us"], workspace=self.ws_f)
+                q.linear_bwd(c["dh"], c["x"], c["us"], c["w"], c["A"], c["B"], a, dx=c["dx"], dA=c["dA"],
+                             dB=c["dB"], workspace=self.ws_b)
         if world > 1:                       # data-parallel adapter-gradient sum, one all-reduce per layer
             dp.allreduce_adapter_grads(self.flat)
 
@@ -326,6 +348,14 @@ def run_ours(args, world, rank, local):
                 "step_frac_of_peak": value / world / peak,
                 "traffic": profiled_traffic(dom, WL.name)}
 
+    # the same step as single calls per projection (no overlap of the rank-r
+    # kernels with the GEMMs), for comparison
+    ms_seq, clk_seq = timed_region(False, lambda: L.step(world, grouped=False), args.steps)
+    sequential = {"what": "the same step as one linear_fwd + linear_bwd call per projection on one stream",
+                  "ms_per_step": ms_seq / args.steps,
+                  "TFLOP/s": world * args.steps * flops / (ms_seq * 1e-3) / 1e12,
+                  "clocks": clk_seq.summary()}
+
     # quantizing all seven weights, timed on its own (3.24 GB of fp32 weights > L2)
     n_q = max(3, min(20, args.steps))
     ms_q, _ = timed_region(False, L.quantize, n_q)
@@ -358,6 +388,7 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
         "gpu_launches": launches,
         "ms_per_step_with_kernel_events": ms_events / args.steps,
+        "single_calls": sequential,
         "clocks": clk.summary(),
         "kernels": kern,
     }

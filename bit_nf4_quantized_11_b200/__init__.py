@@ -13,6 +13,7 @@ Entry points (same names as the C ABI, without the ``qlora_`` prefix):
   dequantize_nf4(w)               -> bf16 [rows, cols]
   linear_fwd(x, w, A, B, alpha)   -> (h, us)
   linear_bwd(dh, x, us, w, A, B, alpha) -> (dx, dA, dB)
+  linear_fwd_group(problems), linear_bwd_group(problems)   (n projections issued together)
   workspace_size(op, M, in_features, out_features, r)
   last_device_status(), set_wait_timeout_ns(ns), selftest_wait_timeout()
 """
@@ -29,6 +30,7 @@ __all__ = [
     "load", "library_path", "codebook", "NF4Weight", "quantize_nf4", "quantize_nf4_noalloc",
     "dequantize_nf4", "alloc_nf4",
     "linear_fwd", "linear_bwd", "workspace_size", "last_device_status",
+    "LinearProblem", "linear_fwd_group", "linear_bwd_group", "linear_group_workspace_size",
     "set_wait_timeout_ns", "selftest_wait_timeout", "QLoRAError", "status_string",
     "timing_enable", "timing_reset", "timing_collect", "KERNEL_NAMES", "merge_adapter",
     "quantize_codebook", "dequantize_codebook", "CODEBOOK_NF4", "CODEBOOK_INT4",
@@ -61,6 +63,13 @@ class _Weight(ctypes.Structure):
                 ("mean", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
+class _Problem(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("w", ctypes.POINTER(_Weight)), ("A", ctypes.c_void_p),
+                ("B", ctypes.c_void_p), ("M", ctypes.c_int64), ("r", ctypes.c_int), ("alpha", ctypes.c_float),
+                ("h", ctypes.c_void_p), ("us", ctypes.c_void_p), ("dh", ctypes.c_void_p), ("dx", ctypes.c_void_p),
+                ("dA", ctypes.c_void_p), ("dB", ctypes.c_void_p)]
+
+
 def load():
     """Load libqlora_nf4.so (built in-tree); raises if it is missing."""
     global _LIB
@@ -82,6 +91,9 @@ def load():
         "qlora_linear_fwd": (I, [P, I64, W, P, P, I, F, P, P, P, SZ, P]),
         "qlora_linear_bwd": (I, [P, P, P, I64, W, P, P, I, F, P, P, P, P, SZ, P]),
         "qlora_last_device_status": (I, [P]),
+        "qlora_linear_group_workspace_size": (SZ, [I, I, ctypes.POINTER(_Problem)]),
+        "qlora_linear_fwd_group": (I, [I, ctypes.POINTER(_Problem), P, SZ, P]),
+        "qlora_linear_bwd_group": (I, [I, ctypes.POINTER(_Problem), P, SZ, P]),
         "qlora_set_wait_timeout_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
         "qlora_selftest_wait_timeout": (I, [P]),
         "qlora_status_string": (ctypes.c_char_p, [I]),
@@ -362,6 +374,89 @@ def linear_bwd(dh, x, us, w: NF4Weight, A, B, alpha: float, dx=None, dA=None, dB
                                    float(alpha), _ptr(dx), _ptr(dA), _ptr(dB), _ptr(ws),
                                    ws.numel() if ws is not None else 0, _stream()), "qlora_linear_bwd")
     return dx, dA, dB
+
+
+@dataclass
+class LinearProblem:
+    """One projection of a grouped call: inputs x, w, A, B, alpha; forward
+    outputs h, us; backward input dh and outputs dx, dA, dB (allocated by the
+    grouped calls when None)."""
+    x: torch.Tensor
+    w: "NF4Weight"
+    A: torch.Tensor
+    B: torch.Tensor
+    alpha: float
+    h: torch.Tensor | None = None
+    us: torch.Tensor | None = None
+    dh: torch.Tensor | None = None
+    dx: torch.Tensor | None = None
+    dA: torch.Tensor | None = None
+    dB: torch.Tensor | None = None
+
+
+def _group_array(problems, backward: bool):
+    arr = (_Problem * len(problems))()
+    keep = []                                      # ctypes weight structs must outlive the call
+    for i, p in enumerate(problems):
+        M, r, w = p.x.shape[0], p.A.shape[0], p.w
+        _need(p.x, torch.bfloat16, "x", (M, w.cols))
+        _need(p.A, torch.bfloat16, "A", (r, w.cols))
+        _need(p.B, torch.bfloat16, "B", (w.rows, r))
+        dev = p.x.device
+        if not backward:
+            p.h = p.h if p.h is not None else torch.empty((M, w.rows), dtype=torch.bfloat16, device=dev)
+            p.us = p.us if p.us is not None else torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+            _need(p.h, torch.bfloat16, "h", (M, w.rows))
+        else:
+            _need(p.dh, torch.bfloat16, "dh", (M, w.rows))
+            p.dx = p.dx if p.dx is not None else torch.empty((M, w.cols), dtype=torch.bfloat16, device=dev)
+            p.dA = p.dA if p.dA is not None else torch.empty((r, w.cols), dtype=torch.float32, device=dev)
+            p.dB = p.dB if p.dB is not None else torch.empty((w.rows, r), dtype=torch.float32, device=dev)
+            _need(p.dx, torch.bfloat16, "dx", (M, w.cols))
+            _need(p.dA, torch.float32, "dA", (r, w.cols))
+            _need(p.dB, torch.float32, "dB", (w.rows, r))
+        _need(p.us, torch.bfloat16, "us", (M, r))
+        cw = w._c()
+        keep.append(cw)
+        arr[i] = _Problem(_ptr(p.x).value, ctypes.pointer(cw), _ptr(p.A).value, _ptr(p.B).value, M, r,
+                          float(p.alpha), _ptr(p.h).value, _ptr(p.us).value, _ptr(p.dh).value, _ptr(p.dx).value,
+                          _ptr(p.dA).value, _ptr(p.dB).value)
+    return arr, keep
+
+
+def linear_group_workspace_size(backward: bool, problems) -> int:
+    arr, _keep = _group_array(problems, backward)
+    n = load().qlora_linear_group_workspace_size(int(bool(backward)), len(problems), arr)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid grouped workspace query")
+    return n
+
+
+def linear_fwd_group(problems, workspace=None):
+    """Forward of independent projections (LinearProblem list), the same
+    results as linear_fwd on each; rank-r products overlap the GEMMs.  Fills
+    and returns the problems' h and us."""
+    if not problems:
+        return problems
+    arr, _keep = _group_array(problems, False)
+    n = load().qlora_linear_group_workspace_size(0, len(problems), arr)
+    ws = _workspace(n, problems[0].x.device, workspace)
+    _check(load().qlora_linear_fwd_group(len(problems), arr, _ptr(ws), ws.numel() if ws is not None else 0,
+                                         _stream()), "qlora_linear_fwd_group")
+    return problems
+
+
+def linear_bwd_group(problems, workspace=None):
+    """Backward of independent projections, the same results as linear_bwd on
+    each; fills and returns the problems' dx, dA and dB."""
+    if not problems:
+        return problems
+    arr, _keep = _group_array(problems, True)
+    n = load().qlora_linear_group_workspace_size(1, len(problems), arr)
+    ws = _workspace(n, problems[0].x.device, workspace)
+    _check(load().qlora_linear_bwd_group(len(problems), arr, _ptr(ws), ws.numel() if ws is not None else 0,
+                                         _stream()), "qlora_linear_bwd_group")
+    return problems
 
 
 OP_LINEAR_FWD_DROPOUT, OP_LINEAR_BWD_DROPOUT = 4, 5

@@ -804,6 +804,71 @@ int check_dropout_args(const uint8_t* keep_bits, float p) {
   return QLORA_OK;
 }
 
+int check_bwd_args(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M, const qlora_nf4_weight* w,
+                   const uint16_t* A, const uint16_t* B, int r, float alpha, const uint16_t* dx, const float* dA,
+                   const float* dB) {
+  if (!dh || !x || !us || !weight_ok(w) || !A || !B || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(dh, 16) || !aligned(x, 16) || !aligned(us, 16) || !aligned(A, 16) || !aligned(B, 16) ||
+      !aligned(dx, 16) || !aligned(dA, 16) || !aligned(dB, 16))
+    return QLORA_ERR_INVALID_ARG;
+  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  return check_linear_shapes(M, w, r);
+}
+
+// ------------------------------------------------------------------ grouped projections
+// Two internal streams per device (highest and lowest priority), created on
+// first use and kept for the process, and a pool of events.  The mutex
+// covers one group call's issue (the streams and events are shared).
+struct GroupStreams {
+  std::mutex mu;
+  cudaStream_t hi = nullptr, lo = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+
+GroupStreams& group_streams() {
+  static GroupStreams g[kMaxDevices];
+  return g[current_device()];
+}
+
+// The rank-r work of a projection moves to the low-priority stream only on
+// the path where it is separate from the GEMM (M > 16, r % 8 == 0).
+bool group_split(const qlora_linear_problem& p) { return p.M > 16 && p.r % 8 == 0; }
+
+size_t group_ws_each(bool backward, const qlora_linear_problem& p) {
+  const size_t n = backward ? bwd_ws(p.M, p.w->cols, p.w->rows, p.r).total : fwd_ws(p.M, p.w->cols, p.w->rows, p.r);
+  return round256(n);
+}
+
+// Issue a group: fork both internal streams from `st`, run `body`, join
+// both back into `st` (also after an error, so that `st` stays ordered
+// after everything that was issued).
+template <typename Body>
+int group_issue(int n_events, cudaStream_t st, Body body) {
+  GroupStreams& g = group_streams();
+  std::lock_guard<std::mutex> lock(g.mu);
+  if (g.hi == nullptr) {
+    int least = 0, greatest = 0;
+    QLORA_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.hi, cudaStreamNonBlocking, greatest));
+    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.lo, cudaStreamNonBlocking, least));
+  }
+  while (static_cast<int>(g.ev.size()) < n_events + 3) {
+    cudaEvent_t e;
+    QLORA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    g.ev.push_back(e);
+  }
+  cudaEvent_t fork = g.ev[0], j_hi = g.ev[1], j_lo = g.ev[2];
+  QLORA_CUDA_TRY(cudaEventRecord(fork, st));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(g.hi, fork, 0));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(g.lo, fork, 0));
+  const int rc = body(g.hi, g.lo, g.ev.data() + 3);
+  QLORA_CUDA_TRY(cudaEventRecord(j_hi, g.hi));
+  QLORA_CUDA_TRY(cudaEventRecord(j_lo, g.lo));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(st, j_hi, 0));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(st, j_lo, 0));
+  return rc;
+}
+
 
 }  // namespace
 
@@ -1035,12 +1100,7 @@ int qlora_linear_fwd_dropout(const uint16_t* x, int64_t M, const qlora_nf4_weigh
 int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us, int64_t M,
                      const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
                      uint16_t* dx, float* dA, float* dB, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!dh || !x || !us || !weight_ok(w) || !A || !B || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(dh, 16) || !aligned(x, 16) || !aligned(us, 16) || !aligned(A, 16) || !aligned(B, 16) ||
-      !aligned(dx, 16) || !aligned(dA, 16) || !aligned(dB, 16))
-    return QLORA_ERR_INVALID_ARG;
-  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-  const int sc = check_linear_shapes(M, w, r);
+  const int sc = check_bwd_args(dh, x, us, M, w, A, B, r, alpha, dx, dA, dB);
   if (sc != QLORA_OK) return sc;
   const BwdWs ws = bwd_ws(M, w->cols, w->rows, r);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
@@ -1052,18 +1112,122 @@ int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16
                              const qlora_nf4_weight* w, const uint16_t* A, const uint16_t* B, int r, float alpha,
                              const uint8_t* keep_bits, float p, uint16_t* dx, float* dA, float* dB, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  if (!dh || !x || !us || !weight_ok(w) || !A || !B || !dx || !dA || !dB) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(dh, 16) || !aligned(x, 16) || !aligned(us, 16) || !aligned(A, 16) || !aligned(B, 16) ||
-      !aligned(dx, 16) || !aligned(dA, 16) || !aligned(dB, 16))
-    return QLORA_ERR_INVALID_ARG;
-  if (!std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
-  int sc = check_linear_shapes(M, w, r);
+  int sc = check_bwd_args(dh, x, us, M, w, A, B, r, alpha, dx, dA, dB);
   if (sc != QLORA_OK) return sc;
   if ((sc = check_dropout_args(keep_bits, p)) != QLORA_OK) return sc;
   const BwdWs ws = bwd_ws(M, w->cols, w->rows, r);
   if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < ws.total) return QLORA_ERR_WORKSPACE;
   return linear_bwd_any_rank(dh, x, us, M, w, A, B, r, alpha / static_cast<float>(r), keep_bits, 1.f / (1.f - p), dx,
                              dA, dB, workspace, static_cast<cudaStream_t>(stream));
+}
+
+size_t qlora_linear_group_workspace_size(int backward, int n, const qlora_linear_problem* problems) {
+  if (n < 0 || (n > 0 && problems == nullptr)) return static_cast<size_t>(-1);
+  size_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    const qlora_linear_problem& p = problems[i];
+    if (!weight_ok(p.w) || p.M < 1 || p.r < 1) return static_cast<size_t>(-1);
+    total += group_ws_each(backward != 0, p);
+  }
+  return total;
+}
+
+int qlora_linear_fwd_group(int n, const qlora_linear_problem* problems, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (n < 0 || (n > 0 && problems == nullptr)) return QLORA_ERR_INVALID_ARG;
+  size_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    const qlora_linear_problem& p = problems[i];
+    const int sc = check_fwd_args(p.x, p.M, p.w, p.A, p.B, p.r, p.alpha, p.h, p.us);
+    if (sc != QLORA_OK) return sc;
+    need += group_ws_each(false, p);
+  }
+  if (n == 0) return QLORA_OK;
+  if (need > 0 && (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need))
+    return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return group_issue(n, st, [&](cudaStream_t hi, cudaStream_t lo, cudaEvent_t* ev) -> int {
+    // us_i = bf16(s x_i A_i^T) on the low-priority stream, then ev[i]
+    auto rank_r = [&](int i) -> int {
+      const qlora_linear_problem& p = problems[i];
+      if (!group_split(p)) return QLORA_OK;
+      const int rc = launch_rowwise<false>(p.x, p.A, p.us, p.M, p.w->cols, p.r, p.alpha / static_cast<float>(p.r), lo);
+      if (rc != QLORA_OK) return rc;
+      QLORA_CUDA_TRY(cudaEventRecord(ev[i], lo));
+      return QLORA_OK;
+    };
+    int rc = rank_r(0);
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    for (int i = 0; i < n && rc == QLORA_OK; ++i) {
+      const qlora_linear_problem& p = problems[i];
+      const int64_t in = p.w->cols, out = p.w->rows;
+      if (group_split(p)) {
+        QLORA_CUDA_TRY(cudaStreamWaitEvent(hi, ev[i], 0));
+        rc = launch_gemm(false, p.w, p.x, p.M, in, p.us, p.B, p.r, p.h, out, hi);   // h = [x|us] [W0|B]^T
+      } else {
+        rc = linear_fwd_any_rank(p.x, nullptr, p.M, p.w, p.A, p.B, p.r, p.alpha / static_cast<float>(p.r), p.h,
+                                 p.us, base, hi);
+      }
+      base += group_ws_each(false, p);
+      if (rc == QLORA_OK && i + 1 < n) rc = rank_r(i + 1);
+    }
+    return rc;
+  });
+}
+
+int qlora_linear_bwd_group(int n, const qlora_linear_problem* problems, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (n < 0 || (n > 0 && problems == nullptr)) return QLORA_ERR_INVALID_ARG;
+  size_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    const qlora_linear_problem& p = problems[i];
+    const int sc = check_bwd_args(p.dh, p.x, p.us, p.M, p.w, p.A, p.B, p.r, p.alpha, p.dx, p.dA, p.dB);
+    if (sc != QLORA_OK) return sc;
+    need += group_ws_each(true, p);
+  }
+  if (n == 0) return QLORA_OK;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < need) return QLORA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<uint8_t*> ws(n);
+  {
+    uint8_t* base = static_cast<uint8_t*>(workspace);
+    for (int i = 0; i < n; ++i) {
+      ws[i] = base;
+      base += group_ws_each(true, problems[i]);
+    }
+  }
+  return group_issue(n, st, [&](cudaStream_t hi, cudaStream_t lo, cudaEvent_t* ev) -> int {
+    // du_i = bf16(s dh_i B_i) into projection i's workspace, then ev[i]
+    auto du_of = [&](int i) { return reinterpret_cast<uint16_t*>(ws[i] + bwd_ws(problems[i].M, problems[i].w->cols,
+                                                                                  problems[i].w->rows,
+                                                                                  problems[i].r).du_off); };
+    auto rank_r = [&](int i) -> int {
+      const qlora_linear_problem& p = problems[i];
+      if (!group_split(p)) return QLORA_OK;
+      const int rc = launch_rowwise<true>(p.dh, p.B, du_of(i), p.M, p.w->rows, p.r, p.alpha / static_cast<float>(p.r),
+                                          lo);
+      if (rc != QLORA_OK) return rc;
+      QLORA_CUDA_TRY(cudaEventRecord(ev[i], lo));
+      return QLORA_OK;
+    };
+    int rc = rank_r(0);
+    for (int i = 0; i < n && rc == QLORA_OK; ++i) {
+      const qlora_linear_problem& p = problems[i];
+      const int64_t in = p.w->cols, out = p.w->rows;
+      if (group_split(p)) {
+        QLORA_CUDA_TRY(cudaStreamWaitEvent(hi, ev[i], 0));
+        rc = launch_gemm(true, p.w, p.dh, p.M, out, du_of(i), p.A, p.r, p.dx, in, hi);   // dx = [dh|du][W0;A]
+        if (rc == QLORA_OK && i + 1 < n) rc = rank_r(i + 1);                             // next du first
+        if (rc == QLORA_OK)
+          rc = launch_lora_grads(p.dh, p.us, p.x, du_of(i), p.M, in, out, p.r, p.dB, p.dA, lo);   // dB, dA
+      } else {
+        rc = linear_bwd_any_rank(p.dh, p.x, p.us, p.M, p.w, p.A, p.B, p.r, p.alpha / static_cast<float>(p.r), nullptr,
+                                 1.f, p.dx, p.dA, p.dB, ws[i], hi);
+        if (rc == QLORA_OK && i + 1 < n) rc = rank_r(i + 1);
+      }
+    }
+    return rc;
+  });
 }
 
 int qlora_last_device_status(void* stream) {

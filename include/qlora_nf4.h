@@ -325,6 +325,61 @@ int qlora_linear_bwd_dropout(const uint16_t* dh, const uint16_t* x, const uint16
                              size_t workspace_bytes, void* stream);
 
 /*
+ * Grouped projections: n independent QLoRA linears issued together, e.g.
+ * the seven projections of one decoder layer ("QLoRA", llm-compass, 实现要点:
+ * target_modules q/k/v/o and gate/up/down).  One problem per projection:
+ *
+ *   x, w, A, B, M, r, alpha   as in qlora_linear_fwd
+ *   h, us                     forward outputs (us is the backward's input)
+ *   dh                        backward input [M, out]
+ *   dx, dA, dB                backward outputs
+ *
+ * qlora_linear_fwd_group computes what n calls of qlora_linear_fwd would, in
+ * order, on `stream`; qlora_linear_bwd_group what n calls of qlora_linear_bwd
+ * would (the fields a direction does not use may be null).  Results are bit
+ * for bit those of the single calls.  The difference is the issue order: the
+ * rank-r products (us in the forward; du, dA and dB in the backward) run on
+ * an internal low-priority stream and the fused GEMMs on an internal
+ * high-priority stream of the current device, projection i + 1's rank-r work
+ * beside projection i's GEMM, so that it fills the SMs the GEMM's last
+ * partial wave of CTA pairs leaves idle.  Both internal streams first wait for
+ * the work issued to `stream` before the call, and `stream` waits for both
+ * before anything issued after it.  Projections with M <= 16 or r % 8 != 0
+ * run as the single call would, on the high-priority stream.
+ *
+ * The projections must not overlap: no output of one may alias any input or
+ * output of another.  workspace: qlora_linear_group_workspace_size(backward,
+ * n, problems) bytes (each projection's single-call workspace, one after
+ * another).  Returns the first failing projection's error before anything is
+ * issued when an argument check fails; QLORA_ERR_INVALID_ARG for n < 0 or a
+ * null `problems` with n > 0.  Calls from several host threads on one device
+ * are serialized while they issue work.  Dropout is not offered grouped.
+ */
+typedef struct qlora_linear_problem {
+  const uint16_t* x;
+  const qlora_nf4_weight* w;
+  const uint16_t* A;
+  const uint16_t* B;
+  int64_t M;
+  int r;
+  float alpha;
+  uint16_t* h;
+  uint16_t* us;
+  const uint16_t* dh;
+  uint16_t* dx;
+  float* dA;
+  float* dB;
+} qlora_linear_problem;
+
+/* (size_t)-1 for n < 0, a null `problems` with n > 0 or a projection whose
+ * sizes qlora_workspace_size rejects. */
+size_t qlora_linear_group_workspace_size(int backward, int n, const qlora_linear_problem* problems);
+int qlora_linear_fwd_group(int n, const qlora_linear_problem* problems, void* workspace, size_t workspace_bytes,
+                           void* stream);
+int qlora_linear_bwd_group(int n, const qlora_linear_problem* problems, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/*
  * qlora_last_device_status -- synchronizes `stream`, then reads and clears
  * the current device's error flag.  Kernels that wait on another part of the
  * device (pipeline barriers inside the GEMMs) give up after a bounded time

@@ -162,6 +162,39 @@ def test_linear_argument_errors(lib):
     assert bwd(FAKE, FAKE, FAKE, 64, wb, FAKE, FAKE, 257, 16.0, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ESHAPE
 
 
+def test_group_argument_errors(lib):
+    fwd, bwd, wsz = lib.qlora_linear_fwd_group, lib.qlora_linear_bwd_group, lib.qlora_linear_group_workspace_size
+    w1, w2 = _weight(128, 128), _weight(256, 192)
+    keep = (w1, w2)
+
+    def prob(w, M=64, r=8, x=FAKE):
+        return q._Problem(x, ctypes.pointer(w), FAKE, FAKE, M, r, 16.0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+
+    arr = (q._Problem * 2)(prob(w1), prob(w2, M=300, r=12))
+    # each projection's single-call workspace, rounded to 256 bytes, one after another
+    for backward, op in ((0, q.OP_LINEAR_FWD), (1, q.OP_LINEAR_BWD)):
+        each = [q.workspace_size(op, 64, 128, 128, 8), q.workspace_size(op, 300, 192, 256, 12)]
+        assert wsz(backward, 2, arr) == sum(-(-n // 256) * 256 for n in each)
+    assert wsz(0, 2, arr) > 0                       # r = 12 runs on padded copies
+    size_max = ctypes.c_size_t(-1).value
+    assert wsz(0, -1, arr) == size_max and wsz(0, 1, None) == size_max
+    assert wsz(0, 0, None) == 0
+    assert fwd(-1, arr, None, 0, None) == EINVAL and bwd(-1, arr, None, 0, None) == EINVAL
+    assert fwd(1, None, None, 0, None) == EINVAL
+    assert fwd(0, None, None, 0, None) == OK and bwd(0, None, None, 0, None) == OK
+    # the first failing projection's status, before anything is issued
+    bad = (q._Problem * 3)(prob(w1), prob(w2, r=0), prob(w1, x=FAKE + 8))
+    assert fwd(3, bad, FAKE, 1 << 30, None) == ESHAPE
+    assert bwd(3, bad, FAKE, 1 << 30, None) == ESHAPE
+    bad[1] = prob(w2)
+    assert fwd(3, bad, FAKE, 1 << 30, None) == EINVAL
+    # a missing or short workspace
+    assert fwd(2, arr, None, 0, None) == EWS
+    assert bwd(2, arr, FAKE, wsz(1, 2, arr) - 256, None) == EWS
+    assert bwd(2, arr, FAKE + 16, 1 << 30, None) == EWS            # not 256-byte aligned
+    del keep
+
+
 def test_dropout_argument_errors(lib):
     fwd, bwd = lib.qlora_linear_fwd_dropout, lib.qlora_linear_bwd_dropout
     w = _weight(128, 128)
