@@ -813,9 +813,36 @@ def comp_gemv(q, dev, peaks, n=60):
                 t_, n_ = q.timing_collect(name)
                 if n_:
                     parts[name] = 1e3 * t_ / n
+            # the same three calls captured once in a CUDA graph and replayed:
+            # the device time of a call without the host's per-call work
+            try:
+                side = torch.cuda.Stream()
+                side.wait_stream(torch.cuda.current_stream())
+                with torch.cuda.stream(side):
+                    for i in range(3):
+                        call(i)
+                torch.cuda.current_stream().wait_stream(side)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph):
+                    for i in range(3):
+                        call(i)
+                graph.replay()
+                torch.cuda.synchronize()
+                reps = max(1, n // 3)
+                a.record()
+                for _ in range(reps):
+                    graph.replay()
+                b.record()
+                torch.cuda.synchronize()
+                graph_us = 1e3 * a.elapsed_time(b) / (3 * reps)
+                del graph
+            except Exception as e:              # report, do not fail the benchmark
+                graph_us = f"capture failed: {type(e).__name__}: {e}"[:200]
             wbytes = workloads.gemv_weight_bytes(n_out, n_in)
             gres[f"{label}_{n_in}x{n_out}_M{M}"] = {
                 "call_us": 1e3 * call_ms, "gemv_kernel_us": 1e3 * kms / kn if kn else None,
+                "graph_replay_call_us": graph_us,
                 "packed_weight_GB/s_call": wbytes / (call_ms * 1e-3) / 1e9,
                 "frac_hbm_call": wbytes / (call_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "packed_weight_GB/s_kernel": wbytes / (kms / kn * 1e-3) / 1e9 if kn else None,

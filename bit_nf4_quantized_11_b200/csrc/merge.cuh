@@ -102,11 +102,25 @@ __global__ void __launch_bounds__(256, 2) merge_adapter_kernel(
         *reinterpret_cast<float4*>(d) = make_float4(bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y));
         *reinterpret_cast<float4*>(d + 4) = make_float4(bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w));
       }
-      // B[o0 + row][j0 + jj] as fp32, transposed to [jj][row]
-      for (int e = threadIdx.x; e < jc * kMergeTileRows; e += 256) {
+      // B[o0 + row][j0 + jj] as fp32, transposed to [jj][row]: eight rank
+      // indices of one row per 16-byte load when r % 8 == 0, else one by one
+      for (int e = threadIdx.x; r % 8 != 0 && e < jc * kMergeTileRows; e += 256) {
         const int row = e / jc, jj = e % jc;
         Bs[jj * kMergeTileRows + row] =
             __uint_as_float(static_cast<uint32_t>(__ldg(B + (o0 + row) * r + j0 + jj)) << 16);
+      }
+      for (int e = threadIdx.x; r % 8 == 0 && e < (jc / 8) * kMergeTileRows; e += 256) {
+        const int row = e / (jc / 8), j8 = 8 * (e % (jc / 8));
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(B + (o0 + row) * r + j0 + j8));
+        float* d = Bs + j8 * kMergeTileRows + row;
+        d[0 * kMergeTileRows] = bf16_lo(b.x);
+        d[1 * kMergeTileRows] = bf16_hi(b.x);
+        d[2 * kMergeTileRows] = bf16_lo(b.y);
+        d[3 * kMergeTileRows] = bf16_hi(b.y);
+        d[4 * kMergeTileRows] = bf16_lo(b.z);
+        d[5 * kMergeTileRows] = bf16_hi(b.z);
+        d[6 * kMergeTileRows] = bf16_lo(b.w);
+        d[7 * kMergeTileRows] = bf16_hi(b.w);
       }
       __syncthreads();
       for (int jj = 0; jj < jc; ++jj) {
