@@ -809,7 +809,7 @@ def comp_gemv(q, dev, peaks, n=60):
             q.timing_enable(False)
             kms, kn = q.timing_collect("gemv")
             parts = {}
-            for name in ("lora_rowwise", "gemv", "gemv_finalize", "lora_pad"):
+            for name in ("lora_fewtok", "lora_rowwise", "gemv", "gemv_finalize", "lora_pad"):
                 t_, n_ = q.timing_collect(name)
                 if n_:
                     parts[name] = 1e3 * t_ / n

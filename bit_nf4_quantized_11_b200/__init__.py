@@ -531,7 +531,7 @@ def selftest_wait_timeout() -> int:
 
 KERNEL_NAMES = ("quantize_blocks", "scale_mean_tree", "dq_scales", "dequantize", "gemm_fwd", "gemm_dx",
                 "gemv", "gemv_finalize", "lora_rowwise", "lora_rowwise_du", "lora_colwise",
-                "merge_adapter", "dropout_dx")
+                "merge_adapter", "dropout_dx", "lora_fewtok", "lora_pad")
 
 
 def timing_enable(on: bool = True) -> bool:

@@ -24,6 +24,7 @@
 #include "quant.cuh"
 #include "lora_sm100.cuh"
 #include "pad.cuh"
+#include "fewtok.cuh"
 
 namespace qnf4_host {
 void build_codebook(float levels[16], float thresholds[15]);
@@ -320,8 +321,19 @@ PadWs pad_ws(int64_t M, int64_t in, int64_t out, int r, bool backward, size_t ba
   return w;
 }
 
+// Few-token rank-r product (fewtok.cuh): its partials, then its ticket.
+size_t fewtok_ws(int64_t in, int r) {
+  return round256(static_cast<size_t>(qnf4::fewtok_part_floats(in, padded_rank(r))) * 4) + 256;
+}
+
+// Forward workspace: for M <= 16 the GEMV partials, then the few-token
+// rank-r partials and ticket; then the padded copies (r % 8 != 0).
+size_t fwd_base_ws(int64_t M, int64_t in, int64_t out, int r) {
+  return M <= 16 ? gemv_ws(M, in, out) + fewtok_ws(in, r) : 0;
+}
+
 size_t fwd_ws(int64_t M, int64_t in, int64_t out, int r) {
-  return pad_ws(M, in, out, r, false, M <= 16 ? gemv_ws(M, in, out) : 0).total;
+  return pad_ws(M, in, out, r, false, fwd_base_ws(M, in, out, r)).total;
 }
 
 size_t fwd_dropout_ws(int64_t M, int64_t in, int64_t out, int r) { return fwd_ws(M, in, out, r); }
@@ -665,6 +677,37 @@ int check_linear_shapes(int64_t M, const qlora_nf4_weight* w, int r) {
   return QLORA_OK;
 }
 
+// ------------------------------------------------------------------ internal streams
+// Two internal streams per device (highest and lowest priority), created on
+// first use and kept for the process, and a pool of events.  The mutex
+// covers one call's issue (the streams and events are shared).
+struct GroupStreams {
+  std::mutex mu;
+  cudaStream_t hi = nullptr, lo = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+
+GroupStreams& group_streams() {
+  static GroupStreams g[kMaxDevices];
+  return g[current_device()];
+}
+
+// With g.mu held: the streams exist and the pool has at least n events.
+int ensure_group_streams(GroupStreams& g, int n) {
+  if (g.hi == nullptr) {
+    int least = 0, greatest = 0;
+    QLORA_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.hi, cudaStreamNonBlocking, greatest));
+    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.lo, cudaStreamNonBlocking, least));
+  }
+  while (static_cast<int>(g.ev.size()) < n) {
+    cudaEvent_t e;
+    QLORA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    g.ev.push_back(e);
+  }
+  return QLORA_OK;
+}
+
 // Forward after validation: us = bf16(s_lora * (x * k) A^T) (k all ones, or
 // the keep mask of LoRA dropout with s_lora = s / (1 - p)), then
 // h = [x | us] [W0 | B]^T; `workspace` is the GEMV part (M <= 16).
@@ -672,8 +715,25 @@ int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlo
                     const uint16_t* A, const uint16_t* B, int r, float s_lora, uint16_t* h, uint16_t* us_out,
                     void* workspace, cudaStream_t st) {
   const int64_t in = w->cols, out = w->rows;
-  int rc = launch_rowwise<false>(x, A, us_out, M, in, r, s_lora, st, keep);   // us = bf16(s (x k) A^T)
+  int rc = QLORA_OK;
+  if (M <= 16) {                                                            // us = bf16(s (x k) A^T)
+    uint8_t* ft = static_cast<uint8_t*>(workspace) + gemv_ws(M, in, out);
+    float* ft_part = reinterpret_cast<float*>(ft);
+    unsigned int* ticket = reinterpret_cast<unsigned int*>(ft + fewtok_ws(in, r) - 256);
+    QLORA_CUDA_TRY(cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st));
+    const unsigned chunks = static_cast<unsigned>(cdiv(in, qnf4::kFtChunk));
+    LaunchTimer lt_("lora_fewtok", st);
+    if (M > 8)
+      qnf4::fewtok_us_kernel<16><<<chunks, qnf4::kFtThreads, 0, st>>>(x, keep, A, static_cast<int>(M), in, r, s_lora,
+                                                                      ft_part, ticket, us_out);
+    else
+      qnf4::fewtok_us_kernel<8><<<chunks, qnf4::kFtThreads, 0, st>>>(x, keep, A, static_cast<int>(M), in, r, s_lora,
+                                                                     ft_part, ticket, us_out);
+  } else {
+    rc = launch_rowwise<false>(x, A, us_out, M, in, r, s_lora, st, keep);    // us = bf16(s (x k) A^T)
+  }
   if (rc != QLORA_OK) return rc;
+  QLORA_CUDA_TRY(cudaGetLastError());
   if (M <= 16) {
     const GemvPlan p = gemv_plan(in, out);
     qnf4::GemvArgs g{};
@@ -702,10 +762,10 @@ int linear_fwd_impl(const uint16_t* x, const uint8_t* keep, int64_t M, const qlo
       kern<<<p.ctas, qnf4::kGvThreads, qnf4::kGvSmem, st>>>(tm_codes, tm_x, g);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
-    const int64_t n_el = M * out;
     {
       LaunchTimer lt_("gemv_finalize", st);
-      qnf4::gemv_finalize_kernel<<<static_cast<unsigned>(std::min<int64_t>(cdiv(n_el, 256), 4096)), 256, 0, st>>>(
+      const dim3 grid(static_cast<unsigned>(cdiv(out, qnf4::kGvRows)), static_cast<unsigned>(M));
+      qnf4::gemv_finalize_kernel<<<grid, qnf4::kGvRows, 0, st>>>(
           g.part, p.ctas, p.local_tiles, p.n_units, p.n_st, static_cast<int>(M), static_cast<int>(out), us_out, B, r, h);
     }
     QLORA_CUDA_TRY(cudaGetLastError());
@@ -723,7 +783,7 @@ int linear_fwd_any_rank(const uint16_t* x, const uint8_t* keep, int64_t M, const
   if (r % 8 == 0) return linear_fwd_impl(x, keep, M, w, A, B, r, s_lora, h, us_out, workspace, st);
   const int64_t in = w->cols, out = w->rows;
   const int rp = padded_rank(r);
-  const PadWs pw = pad_ws(M, in, out, r, false, M <= 16 ? gemv_ws(M, in, out) : 0);
+  const PadWs pw = pad_ws(M, in, out, r, false, fwd_base_ws(M, in, out, r));
   uint8_t* base = static_cast<uint8_t*>(workspace);
   uint16_t* A_p = reinterpret_cast<uint16_t*>(base + pw.a_off);
   uint16_t* B_p = reinterpret_cast<uint16_t*>(base + pw.b_off);
@@ -815,21 +875,6 @@ int check_bwd_args(const uint16_t* dh, const uint16_t* x, const uint16_t* us, in
   return check_linear_shapes(M, w, r);
 }
 
-// ------------------------------------------------------------------ grouped projections
-// Two internal streams per device (highest and lowest priority), created on
-// first use and kept for the process, and a pool of events.  The mutex
-// covers one group call's issue (the streams and events are shared).
-struct GroupStreams {
-  std::mutex mu;
-  cudaStream_t hi = nullptr, lo = nullptr;
-  std::vector<cudaEvent_t> ev;
-};
-
-GroupStreams& group_streams() {
-  static GroupStreams g[kMaxDevices];
-  return g[current_device()];
-}
-
 // The rank-r work of a projection moves to the low-priority stream only on
 // the path where it is separate from the GEMM (M > 16, r % 8 == 0).
 bool group_split(const qlora_linear_problem& p) { return p.M > 16 && p.r % 8 == 0; }
@@ -846,17 +891,8 @@ template <typename Body>
 int group_issue(int n_events, cudaStream_t st, Body body) {
   GroupStreams& g = group_streams();
   std::lock_guard<std::mutex> lock(g.mu);
-  if (g.hi == nullptr) {
-    int least = 0, greatest = 0;
-    QLORA_CUDA_TRY(cudaDeviceGetStreamPriorityRange(&least, &greatest));
-    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.hi, cudaStreamNonBlocking, greatest));
-    QLORA_CUDA_TRY(cudaStreamCreateWithPriority(&g.lo, cudaStreamNonBlocking, least));
-  }
-  while (static_cast<int>(g.ev.size()) < n_events + 3) {
-    cudaEvent_t e;
-    QLORA_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
-    g.ev.push_back(e);
-  }
+  const int rc0 = ensure_group_streams(g, n_events + 3);
+  if (rc0 != QLORA_OK) return rc0;
   cudaEvent_t fork = g.ev[0], j_hi = g.ev[1], j_lo = g.ev[2];
   QLORA_CUDA_TRY(cudaEventRecord(fork, st));
   QLORA_CUDA_TRY(cudaStreamWaitEvent(g.hi, fork, 0));

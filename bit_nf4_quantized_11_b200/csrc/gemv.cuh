@@ -363,44 +363,73 @@ __global__ void __launch_bounds__(kGvThreads, 1)
 
 // h[m][o] = bf16( sum of the partials of o's tile, in CTA order
 //                 + sum_j us[m][j] * B[o][j] ),  m < M.
-__global__ void __launch_bounds__(256) gemv_finalize_kernel(
+// One CTA per (256-row tile, token), one thread per row.  Thread 0 lists the
+// CTAs whose unit ranges touch the tile (with the tile's slot in each CTA's
+// partials); longer lists than kGvFinMax are walked by every thread.
+constexpr int kGvFinMax = 32;
+
+__global__ void __launch_bounds__(kGvRows) gemv_finalize_kernel(
     const float* __restrict__ part, int ctas, int local_tiles, int64_t n_units, int n_st, int M, int out,
     const uint16_t* __restrict__ us, const uint16_t* __restrict__ B, int r, uint16_t* __restrict__ h) {
-  const int64_t n_el = static_cast<int64_t>(M) * out;
-  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < n_el;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int m = static_cast<int>(e / out), o = static_cast<int>(e % out);
-    const int t = o / kGvRows, row = o % kGvRows;
+  __shared__ int s_c[kGvFinMax], s_lt[kGvFinMax];
+  __shared__ int s_n, s_c0;
+  const int t = blockIdx.x, m = blockIdx.y, row = threadIdx.x;
+  const int o = t * kGvRows + row;
+  const int64_t u = static_cast<int64_t>(t) * n_st;
+  if (threadIdx.x == 0) {
     // CTA holding the tile's first unit: the largest c with begin(c) <= t * n_st
-    const int64_t u = static_cast<int64_t>(t) * n_st;
-    int64_t c = u * ctas / n_units;
-    while (c + 1 < ctas && gemv_unit_begin(c + 1, n_units, ctas) <= u) ++c;
-    while (c > 0 && gemv_unit_begin(c, n_units, ctas) > u) --c;
-    float v = 0.f;
-    for (; c < ctas; ++c) {
-      const int64_t b = gemv_unit_begin(c, n_units, ctas);
-      if (b >= u + n_st) break;                                     // past this tile
-      if (gemv_unit_begin(c + 1, n_units, ctas) <= b) continue;     // empty CTA
-      const int lt = t - static_cast<int>(b / n_st);
-      v += __ldg(part + ((c * local_tiles + lt) * M + m) * static_cast<int64_t>(kGvRows) + row);
-    }
-    const uint16_t* ur = us + static_cast<int64_t>(m) * r;
-    const uint16_t* br = B + static_cast<int64_t>(o) * r;
-    float l = 0.f;
-    for (int j = 0; j < r; j += 8) {
-      const uint4 ua = __ldg(reinterpret_cast<const uint4*>(ur + j));
-      const uint4 ba = __ldg(reinterpret_cast<const uint4*>(br + j));
-      const uint32_t uw[4] = {ua.x, ua.y, ua.z, ua.w}, bw[4] = {ba.x, ba.y, ba.z, ba.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[i]));
-        const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
-        l = fmaf(uf.x, bf.x, l);
-        l = fmaf(uf.y, bf.y, l);
+    int c0 = static_cast<int>(u * ctas / n_units);
+    while (c0 + 1 < ctas && gemv_unit_begin(c0 + 1, n_units, ctas) <= u) ++c0;
+    while (c0 > 0 && gemv_unit_begin(c0, n_units, ctas) > u) --c0;
+    int n = 0;
+    int64_t b = gemv_unit_begin(c0, n_units, ctas);
+    for (int c = c0; c < ctas && b < u + n_st; ++c) {
+      const int64_t b_next = gemv_unit_begin(c + 1, n_units, ctas);
+      if (b_next > b) {                                             // a CTA with units
+        if (n < kGvFinMax) {
+          s_c[n] = c;
+          s_lt[n] = t - static_cast<int>(b / n_st);
+        }
+        ++n;
       }
+      b = b_next;
     }
-    h[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v + l));
+    s_n = n;
+    s_c0 = c0;
   }
+  __syncthreads();
+  if (o >= out) return;
+  float v = 0.f;
+  const int n = s_n;
+  if (n <= kGvFinMax) {
+    for (int i = 0; i < n; ++i)
+      v += __ldg(part + ((static_cast<int64_t>(s_c[i]) * local_tiles + s_lt[i]) * M + m) * kGvRows + row);
+  } else {
+    int64_t b = gemv_unit_begin(s_c0, n_units, ctas);
+    for (int c = s_c0; c < ctas && b < u + n_st; ++c) {
+      const int64_t b_next = gemv_unit_begin(c + 1, n_units, ctas);
+      if (b_next > b)
+        v += __ldg(part + ((static_cast<int64_t>(c) * local_tiles + (t - static_cast<int>(b / n_st))) * M + m) *
+                              kGvRows + row);
+      b = b_next;
+    }
+  }
+  const uint16_t* ur = us + static_cast<int64_t>(m) * r;
+  const uint16_t* br = B + static_cast<int64_t>(o) * r;
+  float l = 0.f;
+  for (int j = 0; j < r; j += 8) {
+    const uint4 ua = __ldg(reinterpret_cast<const uint4*>(ur + j));
+    const uint4 ba = __ldg(reinterpret_cast<const uint4*>(br + j));
+    const uint32_t uw[4] = {ua.x, ua.y, ua.z, ua.w}, bw[4] = {ba.x, ba.y, ba.z, ba.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 uf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uw[i]));
+      const float2 bf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw[i]));
+      l = fmaf(uf.x, bf.x, l);
+      l = fmaf(uf.y, bf.y, l);
+    }
+  }
+  h[static_cast<int64_t>(m) * out + o] = __bfloat16_as_ushort(__float2bfloat16_rn(v + l));
 }
 
 }  // namespace qnf4
