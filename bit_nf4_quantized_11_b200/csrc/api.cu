@@ -570,7 +570,8 @@ int launch_lora_umma(const CUtensorMap (&tm)[4], const qnf4::LrArgs& a, int ks, 
   QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(kern), smem));
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid_x, static_cast<unsigned>(ks), 1);
-  cfg.blockDim = dim3(qnf4::kLrThreads);
+  const bool masked = a.p[0].keep != nullptr || a.p[1].keep != nullptr;
+  cfg.blockDim = dim3(masked ? qnf4::kLrMaskThreads : qnf4::kLrThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

@@ -23,12 +23,13 @@
 // adds up its share of the tile's rows over distributed shared memory,
 // partials in rank order (deterministic), and stores it.
 //
-// Roles (128 threads): warp 0 lane 0 issues the TMA loads, warp 1 allocates
-// tensor memory and its lane 0 issues the MMAs, and with a LoRA-dropout keep
-// mask warps 2 and 3 zero the dropped activations of each landed stage in
-// shared memory (bit c % 8 of byte c / 8 of a token's row keeps column c)
-// before the MMAs read it; afterwards the four warps read the accumulator
-// (warp w owns rows 32 w .. 32 w + 31, its TMEM lanes).
+// Roles (128 threads, 320 with a keep mask): warp 0 lane 0 issues the TMA
+// loads, warp 1 allocates tensor memory and its lane 0 issues the MMAs, and
+// with a LoRA-dropout keep mask warps 2-9 zero the dropped activations of
+// each landed stage in shared memory (bit c % 8 of byte c / 8 of a token's
+// row keeps column c) before the MMAs read it; afterwards warps 0-3 read the
+// accumulator (warp w owns rows 32 w .. 32 w + 31, its TMEM lanes) and all
+// warps take part in the cluster reduction.
 // Every wait is bounded: on timeout the CTA sets the device error flag,
 // issues nothing more, waits (bounded) for what it issued and exits.
 // No TMA multicast is used.
@@ -39,6 +40,7 @@
 namespace qnf4 {
 
 constexpr int kLrThreads = 128;
+constexpr int kLrMaskThreads = 320;                        // with a keep mask: eight masking warps
 constexpr int kLrMaxStages = 8;
 constexpr int kLrTileRows = 128;
 constexpr int kLrAStage = kLrTileRows * 64 * 2;           // 16 KB: 128 rows x 64 k (or two 64-wide MN atoms)
@@ -86,7 +88,7 @@ __host__ __device__ constexpr int lr_smem_bytes(int N, bool b_mn_major, int stag
 // kCol: col form (A MN-major, output fp32); otherwise row form (A K-major,
 // output bf16).  kBMN: B operand N-major.
 template <bool kCol, bool kBMN>
-__global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
+__global__ void __launch_bounds__(kLrMaskThreads) lora_umma_kernel(
     const __grid_constant__ CUtensorMap tm_a0, const __grid_constant__ CUtensorMap tm_b0,
     const __grid_constant__ CUtensorMap tm_a1, const __grid_constant__ CUtensorMap tm_b1, const LrArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -133,7 +135,7 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
     for (int s = 0; s < S; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
-      mbar_init(masked + s, 2);                                      // one arrive per masking warp
+      mbar_init(masked + s, (blockDim.x - 64) / 32);                 // one arrive per masking warp
     }
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -215,10 +217,15 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
     }
   } else if (do_mask) {
     // ------------------------------------------------------------ keep mask
-    // Thread t (0..63) owns tile row t (row form: token row0 + t and +64;
-    // col form: token k0 + t of both 64-feature atoms) and zeroes, in
-    // each landed stage, the values whose keep bit is 0.
+    // The MT = blockDim - 64 masking threads split a stage into 256 items,
+    // (row i, half q) = (j % 128, j / 128) for j = t + MT h: row form, token
+    // row0 + i; col form, token k0 + i % 64 of the 64-feature atom i / 64;
+    // half q is 16-byte chunks 4q .. 4q + 3 of the row (32 values, one
+    // 32-bit word of keep bits).  In each landed stage the thread zeroes the
+    // values of its items whose keep bit is 0.
     const int t = threadIdx.x - 64;
+    const int MT = static_cast<int>(blockDim.x) - 64;
+    const int n_items = 2 * kLrTileRows / MT;                        // 1, 2 or 4 per thread
     const int64_t kb_row = p_features / 8;                           // keep bytes per token
     auto mask_chunk16 = [](uint32_t addr, uint32_t bits) {           // 8 bf16 at addr, bit e keeps value e
       uint32_t v[4];
@@ -229,61 +236,62 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
         v[e] &= ((bits >> (2 * e)) & 1u ? 0x0000FFFFu : 0u) | ((bits >> (2 * e + 1)) & 1u ? 0xFFFF0000u : 0u);
       sts_v4(addr, v[0], v[1], v[2], v[3]);
     };
-    // this thread's keep bytes of stage `it` (zero past the token or feature end)
-    auto load_keep = [&](int it, uint2 (&kb)[2]) {
+    // keep-bit address of item h of stage `it`, or null past the token or feature end
+    auto keep_ptr = [&](int it, int h) -> const uint32_t* {
+      if (it >= n_iter || h >= n_items) return nullptr;
+      const int j = t + MT * h, i = j & (kLrTileRows - 1), q = j >> 7;
+      const int k0 = (st_begin + it) * 64;
+      int64_t tok, f0;
+      if (!kCol) { tok = row0 + i; f0 = k0; }
+      else { tok = k0 + (i & 63); f0 = row0 + 64 * (i >> 6); }
+      const int64_t n_tok = kCol ? args.K : p_rows;
+      if (tok >= n_tok || f0 >= p_features) return nullptr;
+      return reinterpret_cast<const uint32_t*>(p_keep + tok * kb_row + f0 / 8) + q;   // 4-byte aligned
+    };
+    auto load_keep = [&](int it, uint32_t (&kb)[4]) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        kb[h] = make_uint2(0u, 0u);
-        if (it >= n_iter) continue;
-        const int k0 = (st_begin + it) * 64;
-        int64_t tok, f0;
-        if (!kCol) { tok = row0 + t + 64 * h; f0 = k0; }
-        else { tok = k0 + t; f0 = row0 + 64 * h; }
-        const int64_t n_tok = kCol ? args.K : p_rows;
-        if (tok < n_tok && f0 < p_features) {                         // keep bits are 4-byte aligned
-          const uint32_t* src = reinterpret_cast<const uint32_t*>(p_keep + tok * kb_row + f0 / 8);
-          kb[h] = make_uint2(__ldg(src), __ldg(src + 1));
-        }
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t* src = keep_ptr(it, h);
+        kb[h] = src != nullptr ? __ldg(src) : 0u;
       }
     };
     // loaded into registers two stages ahead and brought into L2 six stages
     // ahead, so their latency overlaps the stream
     auto prefetch_keep = [&](int it) {
-      if (it >= n_iter) return;
-      const int k0 = (st_begin + it) * 64;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        int64_t tok, f0;
-        if (!kCol) { tok = row0 + t + 64 * h; f0 = k0; }
-        else { tok = k0 + t; f0 = row0 + 64 * h; }
-        const int64_t n_tok = kCol ? args.K : p_rows;
-        if (tok < n_tok && f0 < p_features)
-          asm volatile("prefetch.global.L2 [%0];" :: "l"(p_keep + tok * kb_row + f0 / 8));
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t* src = keep_ptr(it, h);
+        if (src != nullptr) asm volatile("prefetch.global.L2 [%0];" :: "l"(src));
       }
     };
     for (int i = 2; i < 6; ++i) prefetch_keep(i);
-    uint2 kb_n1[2], kb_n2[2];
+    uint32_t kb_n1[4], kb_n2[4];
     load_keep(0, kb_n1);
     load_keep(1, kb_n2);
     for (int it = 0; it < n_iter; ++it) {
       const int s = it % S;
-      uint2 kb[2] = {kb_n1[0], kb_n1[1]};
-      kb_n1[0] = kb_n2[0];
-      kb_n1[1] = kb_n2[1];
+      uint32_t kb[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        kb[h] = kb_n1[h];
+        kb_n1[h] = kb_n2[h];
+      }
       load_keep(it + 2, kb_n2);
       prefetch_keep(it + 6);
       wait(full + s, (it / S) & 1u);
       if (*abort_flag) break;
       const uint32_t a_base = smem_u32(a_ring + s * kLrAStage);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        // row form: row t + 64 h of the 128-row tile; col form: row t of atom h
-        const int r = kCol ? t : t + 64 * h;
-        const uint32_t rbase = a_base + (kCol ? h * 8192 : 0) + r * 128;
+      for (int h = 0; h < 4; ++h) {
+        if (h >= n_items) continue;
+        const int j = t + MT * h, i = j & (kLrTileRows - 1), q = j >> 7;
+        // row form: row i of the 128-row tile; col form: row i % 64 of atom i / 64
+        const int r = kCol ? (i & 63) : i;
+        const uint32_t rbase = a_base + (kCol ? (i >> 6) * 8192 : 0) + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t bits = ((c < 4 ? kb[h].x : kb[h].y) >> (8 * (c & 3))) & 0xFFu;
-          if (bits != 0xFFu) mask_chunk16(rbase + (((c ^ r) & 7) << 4), bits);
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t bits = (kb[h] >> (8 * c)) & 0xFFu;
+          if (bits != 0xFFu) mask_chunk16(rbase + ((((4 * q + c) ^ r) & 7) << 4), bits);
         }
       }
       fence_proxy_async_smem();                                     // generic writes before the MMAs read
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
   const int pitch = lr_partial_pitch(N);
   uint8_t* part = smem;                                              // the ring is free once acc_full completed
   __syncthreads();                                                   // every stage read by the tensor cores
-  for (int c0 = 0; c0 < N; c0 += 32) {
+  for (int c0 = 0; warp < 4 && c0 < N; c0 += 32) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(warp * 32) << 16) + c0, v);
     tmem_ld_wait();
@@ -323,7 +331,7 @@ __global__ void __launch_bounds__(kLrThreads) lora_umma_kernel(
   const int share = kLrTileRows / ks;
   const int r_lo = split * share;
   const int n4 = args.r / 4;                                         // float4 groups of the rank
-  for (int e = threadIdx.x; e < share * n4; e += kLrThreads) {
+  for (int e = threadIdx.x; e < share * n4; e += static_cast<int>(blockDim.x)) {
     int rr, c4;
     if (kCol && p_transpose) {                                   // rows fastest: coalesced dA^T stores
       rr = r_lo + e % share;
