@@ -23,9 +23,8 @@ namespace qnf4 {
 // and A[:r, columns] in shared memory, its four warps compute P for 16 rows
 // each with warp-level bf16 MMAs (m16n8k16, the rank in 16-wide steps, rows
 // of du and A past r are zero), leave P in shared memory, and then every
-// thread applies 8 consecutive columns of one row per unit: one 16-byte read
-// (issued at the start of the kernel) and write of dx, one keep byte, two
-// 16-byte reads of P.
+// thread applies 8 consecutive columns of one row: one 16-byte read and
+// write of dx, one keep byte, two 16-byte reads of P.
 constexpr int kDxTileRows = 64;
 constexpr int kDxTileCols = 128;
 constexpr int kDxThreads = 128;
@@ -53,23 +52,6 @@ __global__ void __launch_bounds__(kDxThreads) dropout_dx_kernel(
   const int64_t i0 = (static_cast<int64_t>(blockIdx.x) % tiles_n) * kDxTileCols;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // this thread's dx and keep loads (8 columns of one row per unit), issued
-  // first so that their latency is spent under the staging and the MMAs
-  constexpr int kUnits = kDxTileRows * (kDxTileCols / 8) / kDxThreads;   // 8
-  uint4 dv[kUnits];
-  uint32_t kv[kUnits];
-#pragma unroll
-  for (int u = 0; u < kUnits; ++u) {
-    const int e = threadIdx.x + u * kDxThreads;
-    const int row = e / (kDxTileCols / 8), c8 = e % (kDxTileCols / 8);
-    const int64_t m = m0 + row, i = i0 + c8 * 8;
-    dv[u] = make_uint4(0, 0, 0, 0);
-    kv[u] = 0;
-    if (m < M && i < n) {
-      dv[u] = *reinterpret_cast<const uint4*>(dx + m * n + i);
-      kv[u] = __ldg(keep_bits + m * (n / 8) + i / 8);
-    }
-  }
   // stage du[m0 .. m0+63][0 .. rk) and A[0 .. rk)[i0 .. i0+127] (zero past M and r)
   for (int e = threadIdx.x; e < kDxTileRows * (rk / 8); e += kDxThreads) {
     const int row = e / (rk / 8), ch = e % (rk / 8);
@@ -125,7 +107,23 @@ __global__ void __launch_bounds__(kDxThreads) dropout_dx_kernel(
   }
   __syncthreads();
 
-  // dx += (k / (1 - p)) * P, 8 columns of one row per thread and unit
+  // dx += (k / (1 - p)) * P, 8 columns of one row per thread and unit; all
+  // of a thread's dx and keep loads are issued before any store
+  constexpr int kUnits = kDxTileRows * (kDxTileCols / 8) / kDxThreads;   // 8
+  uint4 dv[kUnits];
+  uint32_t kv[kUnits];
+#pragma unroll
+  for (int u = 0; u < kUnits; ++u) {
+    const int e = threadIdx.x + u * kDxThreads;
+    const int row = e / (kDxTileCols / 8), c8 = e % (kDxTileCols / 8);
+    const int64_t m = m0 + row, i = i0 + c8 * 8;
+    dv[u] = make_uint4(0, 0, 0, 0);
+    kv[u] = 0;
+    if (m < M && i < n) {
+      dv[u] = *reinterpret_cast<const uint4*>(dx + m * n + i);
+      kv[u] = __ldg(keep_bits + m * (n / 8) + i / 8);
+    }
+  }
 #pragma unroll
   for (int u = 0; u < kUnits; ++u) {
     const int e = threadIdx.x + u * kDxThreads;
