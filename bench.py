@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", choices=["quantize", "gemv", "workloads", "merge", "dropout", "layer_step",
-                                       "q_proj_steps"],
+                                       "q_proj_steps", "dropout_steps"],
                     default=None,
                     help="run one component measurement alone and print it (for profiling)")
     return ap.parse_args()
@@ -720,6 +720,22 @@ def comp_dropout(q, dev, peaks, n=50):
     return {"lora_dropout_llama7b_attn": res}
 
 
+def dropout_steps_once(q, dev, steps=2):
+    """Untimed LoRA-dropout steps of the 7B attention projection (p = 0.05),
+    for a profiler's capture of the masked kernels alone."""
+    M, n_in, n_out, r, alpha, p = 4096, 4096, 4096, 16, 32.0, 0.05
+    prob = synth.problem(M, n_in, n_out, r, seed=4)
+    w = q.quantize_nf4(prob["W"].to(dev))
+    x, A, B, dh = (prob[k].to(dev) for k in ("x", "A", "B", "dh"))
+    keep = torch.from_numpy(np.random.default_rng(4).random((M, n_in)) >= p).to(dev)
+    kb = q.pack_keep_mask(keep)
+    for _ in range(1 + steps):
+        _, us = q.linear_fwd_dropout(x, w, A, B, alpha, kb, p)
+        q.linear_bwd_dropout(dh, x, us, w, A, B, alpha, kb, p)
+    torch.cuda.synchronize()
+    return {"ok": q.last_device_status() == 0, "steps": 1 + steps}
+
+
 def comp_merge(q, dev, peaks, src, reps=5):
     """Adapter merge into a bf16 base and its lossy re-quantization to NF4, on
     the 7B attention projection (r=16) and the 65B down projection (r=64).
@@ -921,6 +937,8 @@ def components(q, dev, only=None):
         out.update(layer_step_once(q, dev))
     if only == "q_proj_steps":
         out.update(layer_step_once(q, dev, projections=(0,), steps=4))
+    if only == "dropout_steps":
+        out.update(dropout_steps_once(q, dev))
     return out
 
 
