@@ -555,10 +555,15 @@ struct LrShape {
   int ks, ring;
 };
 
-LrShape lr_shape(int64_t tiles, int64_t stages) {
+// Split count ks (a power of two <= 8, the cluster size): doubled while the
+// grid stays within the CTAs that fit at once (one or two per SM, by the
+// kernel's shared memory for this rank) and every split keeps at least two
+// 64-wide stages.
+LrShape lr_shape(int64_t tiles, int64_t stages, int N, bool b_mn_major) {
   const int sms = device_sm_count();
   LrShape sh{1, 4};
-  while (sh.ks < 8 && tiles * sh.ks * 2 <= sms && stages / (2 * sh.ks) >= 2) sh.ks *= 2;
+  const int per_sm = 2 * (qnf4::lr_smem_bytes(N, b_mn_major, sh.ring) + 1024) <= 228 * 1024 ? 2 : 1;
+  while (sh.ks < 8 && tiles * sh.ks * 2 <= per_sm * sms && stages / (2 * sh.ks) >= 2) sh.ks *= 2;
   return sh;
 }
 
@@ -603,7 +608,7 @@ int launch_lora_row(const uint16_t* act, const uint16_t* w, uint16_t* out, int64
   a.p[1] = a.p[0];
   a.timeout_ns = g_timeout_ns.load();
   const int64_t stages = cdiv(K, 64);
-  const LrShape sh = lr_shape(a.p[0].tiles, stages);
+  const LrShape sh = lr_shape(a.p[0].tiles, stages, a.N, w_n_major);
   const int ks = sh.ks;
   a.ring = sh.ring;
   a.stages_per_split = static_cast<int>(cdiv(stages, ks));
@@ -634,7 +639,7 @@ int launch_lora_col(const uint16_t* dh, const uint16_t* us, const uint16_t* x, c
                            static_cast<int>(in)};
   a.timeout_ns = g_timeout_ns.load();
   const int64_t stages = cdiv(M, 64);
-  const LrShape sh = lr_shape(a.p[0].tiles + a.p[1].tiles, stages);
+  const LrShape sh = lr_shape(a.p[0].tiles + a.p[1].tiles, stages, a.N, true);
   const int ks = sh.ks;
   a.ring = sh.ring;
   a.stages_per_split = static_cast<int>(cdiv(stages, ks));
