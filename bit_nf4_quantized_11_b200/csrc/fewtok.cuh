@@ -73,22 +73,51 @@ __global__ void __launch_bounds__(kFtThreads) fewtok_us_kernel(
       a[4] = fewtok_bf16_lo(v.z); a[5] = fewtok_bf16_hi(v.z);
       a[6] = fewtok_bf16_lo(v.w); a[7] = fewtok_bf16_hi(v.w);
     }
+    float p[kTok];
 #pragma unroll
     for (int m = 0; m < kTok; ++m) {
       const float4 x0 = *reinterpret_cast<const float4*>(&xs[m][8 * lane]);
       const float4 x1 = *reinterpret_cast<const float4*>(&xs[m][8 * lane + 4]);
-      float p = a[0] * x0.x;
-      p = fmaf(a[1], x0.y, p);
-      p = fmaf(a[2], x0.z, p);
-      p = fmaf(a[3], x0.w, p);
-      p = fmaf(a[4], x1.x, p);
-      p = fmaf(a[5], x1.y, p);
-      p = fmaf(a[6], x1.z, p);
-      p = fmaf(a[7], x1.w, p);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xFFFFFFFFu, p, off);
-      if (lane == 0) part[(static_cast<int64_t>(c) * kFtMaxTok + m) * r + j] = p;
+      float v = a[0] * x0.x;
+      v = fmaf(a[1], x0.y, v);
+      v = fmaf(a[2], x0.z, v);
+      v = fmaf(a[3], x0.w, v);
+      v = fmaf(a[4], x1.x, v);
+      v = fmaf(a[5], x1.y, v);
+      v = fmaf(a[6], x1.z, v);
+      v = fmaf(a[7], x1.w, v);
+      p[m] = v;
     }
+    // Sum each token's value over the 32 lanes with the xor butterfly
+    // (offsets 16, 8, 4, 2, 1), halving the values a lane carries at each of
+    // the first steps: a lane keeps the tokens whose bit matches its own lane
+    // bit and adds its partner's copy of them.  The pairs added are those of
+    // a per-token butterfly, so every sum is the same.
+    int width = kTok;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      if (width > 1) {
+        const bool upper = (lane & off) != 0;
+        width >>= 1;
+#pragma unroll
+        for (int i = 0; i < kTok / 2; ++i) {
+          if (i < width) {
+            const float send = upper ? p[i] : p[i + width];
+            const float keep = upper ? p[i + width] : p[i];
+            p[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+          }
+        }
+      } else {
+        p[0] += __shfl_xor_sync(0xFFFFFFFFu, p[0], off);
+      }
+    }
+    // lane bits 4, 3, ... (one per halving) name the token whose sum it holds
+    int m = 0;
+#pragma unroll
+    for (int off = 16, w = kTok / 2; w > 0; off >>= 1, w >>= 1)
+      if (lane & off) m += w;
+    constexpr int kLowMask = 32 / kTok - 1;                        // lanes with these bits 0 write
+    if ((lane & kLowMask) == 0 && m < M) part[(static_cast<int64_t>(c) * kFtMaxTok + m) * r + j] = p[0];
   }
 
   // the last CTA to finish adds the chunks' partials in chunk order
@@ -104,12 +133,12 @@ __global__ void __launch_bounds__(kFtThreads) fewtok_us_kernel(
     const float* pe = part + static_cast<int64_t>(m) * r + j;
     const int64_t stride = static_cast<int64_t>(kFtMaxTok) * r;
     float v = 0.f;
-    for (int cc = 0; cc < chunks; cc += 8) {        // eight loads in flight, added in chunk order
-      float t[8];
+    for (int cc = 0; cc < chunks; cc += 16) {       // sixteen loads in flight, added in chunk order
+      float t[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) t[i] = cc + i < chunks ? __ldcg(pe + (cc + i) * stride) : 0.f;
+      for (int i = 0; i < 16; ++i) t[i] = cc + i < chunks ? __ldcg(pe + (cc + i) * stride) : 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) v += t[i];
+      for (int i = 0; i < 16; ++i) v += t[i];
     }
     us[e] = __bfloat16_as_ushort(__float2bfloat16_rn(s * v));
   }

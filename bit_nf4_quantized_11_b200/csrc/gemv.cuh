@@ -377,14 +377,21 @@ __global__ void __launch_bounds__(kGvRows) gemv_finalize_kernel(
   const int o = t * kGvRows + row;
   const int64_t u = static_cast<int64_t>(t) * n_st;
   if (threadIdx.x == 0) {
+    // unit ranges in 32-bit arithmetic when the products fit (the same floors)
+    const bool small = static_cast<uint64_t>(n_units) * static_cast<uint64_t>(ctas) < (1ull << 32);
+    auto begin = [&](int c) -> int64_t {
+      return small ? static_cast<int64_t>(static_cast<uint32_t>(c) * static_cast<uint32_t>(n_units) /
+                                          static_cast<uint32_t>(ctas))
+                   : gemv_unit_begin(c, n_units, ctas);
+    };
     // CTA holding the tile's first unit: the largest c with begin(c) <= t * n_st
     int c0 = static_cast<int>(u * ctas / n_units);
-    while (c0 + 1 < ctas && gemv_unit_begin(c0 + 1, n_units, ctas) <= u) ++c0;
-    while (c0 > 0 && gemv_unit_begin(c0, n_units, ctas) > u) --c0;
+    while (c0 + 1 < ctas && begin(c0 + 1) <= u) ++c0;
+    while (c0 > 0 && begin(c0) > u) --c0;
     int n = 0;
-    int64_t b = gemv_unit_begin(c0, n_units, ctas);
+    int64_t b = begin(c0);
     for (int c = c0; c < ctas && b < u + n_st; ++c) {
-      const int64_t b_next = gemv_unit_begin(c + 1, n_units, ctas);
+      const int64_t b_next = begin(c + 1);
       if (b_next > b) {                                             // a CTA with units
         if (n < kGvFinMax) {
           s_c[n] = c;
