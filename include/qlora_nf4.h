@@ -23,10 +23,12 @@
  *   Every pointer except the host arrays of qlora_nf4_codebook is a DEVICE
  *   pointer on the current CUDA device and must be 16-byte aligned.
  *   `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *   All device work is enqueued on `stream` and the calls return without
+ *   All device work is enqueued on `stream` (the grouped calls fork it onto
+ *   internal streams and join them back) and the calls return without
  *   synchronizing; outputs are valid once the stream reaches that point.
  *   The caller owns every buffer, including the workspace; the library never
- *   allocates device memory and keeps no per-call state.
+ *   allocates device memory and keeps no per-call state (the grouped calls
+ *   keep their internal streams and events for the process).
  *   Arguments are validated before anything is launched: a call that returns
  *   a negative status has enqueued no work and written no output.
  *
