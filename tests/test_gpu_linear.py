@@ -75,6 +75,13 @@ def test_few_token_gemv(cuda_lib, M):
     _run(cuda_lib, M, 1024, 768, 16, 32.0, seed=M, backward=True)
 
 
+@pytest.mark.parametrize("M,r", [(9, 256), (16, 136), (2, 64)])
+def test_few_token_ranks(cuda_lib, M, r):
+    # the few-token rank-r kernel at the largest rank, a rank spanning three
+    # 64-wide stages, and with its partials over four K chunks
+    _run(cuda_lib, M, 1024, 768, r, 16.0, seed=300 + r, backward=True)
+
+
 @pytest.mark.parametrize("M,n_in,n_out", [(3, 576, 320), (12, 192, 448), (1, 64, 64), (16, 64, 1088),
                                            (7, 4160, 576)])
 def test_few_token_ragged(cuda_lib, M, n_in, n_out):
