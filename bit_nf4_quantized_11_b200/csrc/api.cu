@@ -811,25 +811,49 @@ int linear_bwd_impl(const uint16_t* dh, const uint16_t* x, const uint16_t* us, i
                     const uint8_t* keep, float inv_keep, uint16_t* dx, float* dA, float* dB, uint16_t* du,
                     cudaStream_t st) {
   const int64_t in = w->cols, out = w->rows;
-  int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                           // du = bf16(s dh B)
-  if (rc != QLORA_OK) return rc;
   if (keep == nullptr) {
+    int rc = launch_rowwise<true>(dh, B, du, M, out, r, s, st);                         // du = bf16(s dh B)
+    if (rc != QLORA_OK) return rc;
     rc = launch_gemm(true, w, dh, M, out, du, A, r, dx, in, st);                         // dx = [dh|du][W0;A]
     if (rc != QLORA_OK) return rc;
     return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st);                  // dB, dA
   }
-  rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, st);                // dx = dh W0
-  if (rc != QLORA_OK) return rc;
-  {
+  // LoRA dropout: the dx GEMM runs without its rank-r tail, so du and the
+  // adapter gradients do not wait for it.  The GEMM goes first on the internal
+  // high-priority stream; du, dB and dA run on the low-priority one, on the
+  // SMs the GEMM's last wave leaves free; the masked dx term waits for the
+  // GEMM and for du.  Both streams are forked from and joined back into `st`.
+  GroupStreams& g = group_streams();
+  std::lock_guard<std::mutex> lock(g.mu);
+  const int rc0 = ensure_group_streams(g, 4);
+  if (rc0 != QLORA_OK) return rc0;
+  QLORA_CUDA_TRY(cudaEventRecord(g.ev[0], st));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(g.hi, g.ev[0], 0));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(g.lo, g.ev[0], 0));
+  int rc = launch_gemm(true, w, dh, M, out, nullptr, nullptr, 0, dx, in, g.hi);          // dx = dh W0
+  if (rc == QLORA_OK) rc = launch_rowwise<true>(dh, B, du, M, out, r, s, g.lo);         // du = bf16(s dh B)
+  if (rc == QLORA_OK && cudaEventRecord(g.ev[1], g.lo) != cudaSuccess) rc = QLORA_ERR_CUDA;
+  if (rc == QLORA_OK)
+    rc = launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, g.lo, inv_keep, keep);  // dB, dA
+  if (rc == QLORA_OK && cudaStreamWaitEvent(g.hi, g.ev[1], 0) != cudaSuccess) rc = QLORA_ERR_CUDA;
+  if (rc == QLORA_OK) {
     const int64_t tiles = cdiv(M, qnf4::kDxTileRows) * cdiv(in, qnf4::kDxTileCols);
     const int smem = qnf4::dx_smem_bytes(r);
-    QLORA_CUDA_TRY(set_max_smem(reinterpret_cast<const void*>(qnf4::dropout_dx_kernel), smem));
-    LaunchTimer lt_("dropout_dx", st);
-    qnf4::dropout_dx_kernel<<<static_cast<unsigned>(tiles), qnf4::kDxThreads, smem, st>>>(dx, du, A, keep, M, in, r,
-                                                                                      inv_keep);  // + (du A) k/(1-p)
+    if (set_max_smem(reinterpret_cast<const void*>(qnf4::dropout_dx_kernel), smem) != cudaSuccess) {
+      rc = QLORA_ERR_CUDA;
+    } else {
+      LaunchTimer lt_("dropout_dx", g.hi);
+      qnf4::dropout_dx_kernel<<<static_cast<unsigned>(tiles), qnf4::kDxThreads, smem, g.hi>>>(
+          dx, du, A, keep, M, in, r, inv_keep);                                           // + (du A) k/(1-p)
+      if (cudaGetLastError() != cudaSuccess) rc = QLORA_ERR_CUDA;
+    }
   }
-  QLORA_CUDA_TRY(cudaGetLastError());
-  return launch_lora_grads(dh, us, x, du, M, in, out, r, dB, dA, st, inv_keep, keep);     // dB, dA
+  // join both streams back into `st` (after an error too)
+  QLORA_CUDA_TRY(cudaEventRecord(g.ev[2], g.hi));
+  QLORA_CUDA_TRY(cudaEventRecord(g.ev[3], g.lo));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(st, g.ev[2], 0));
+  QLORA_CUDA_TRY(cudaStreamWaitEvent(st, g.ev[3], 0));
+  return rc;
 }
 
 // Backward at any rank (the padded copies as in linear_fwd_any_rank; dA and

@@ -307,7 +307,9 @@ int qlora_linear_bwd(const uint16_t* dh, const uint16_t* x, const uint16_t* us,
  * of dh W0 in fp32 and rounds again to bf16.
  *
  * The masked input x * k is never stored: the rank-r kernels zero the
- * dropped elements of the activation tiles they stage.
+ * dropped elements of the activation tiles they stage.  The backward forks
+ * `stream` onto the library's internal streams (the dx GEMM beside du, dB
+ * and dA) and joins them back before returning, like the grouped calls.
  *
  * keep_bits  device uint8 [M, in/8], 4-byte aligned: bit (i % 8) of byte i/8
  *            of row m is the keep flag of x[m][i] (the caller draws the mask).
