@@ -244,3 +244,37 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError, match="no fallback"):
         q.load()
     importlib.reload(q)
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    # the boundary is plain C: the header compiles as C99 with warnings as
+    # errors, and a C program links against the library and calls a host-only
+    # entry point through it
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi.c"
+    src.write_text(
+        '#include "qlora_nf4.h"\n'
+        "#include <stdio.h>\n"
+        "int main(void) {\n"
+        "  float levels[16], thr[15];\n"
+        "  qlora_linear_problem p = {0};\n"
+        "  (void)p;\n"
+        "  if (qlora_nf4_codebook(levels, thr) != QLORA_OK) return 1;\n"
+        "  if (qlora_linear_group_workspace_size(0, 0, NULL) != 0) return 2;\n"
+        '  printf("%.9g %.9g\\n", levels[0], levels[15]);\n'
+        "  return levels[7] == 0.0f ? 0 : 3;\n"
+        "}\n")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(q.library_path())
+    res = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                          str(src), "-o", str(exe), "-L", libdir, "-lqlora_nf4", f"-Wl,-rpath,{libdir}"],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert run.stdout.split()[0] == "-1" and run.stdout.split()[1] == "1"
