@@ -116,10 +116,12 @@ def test_quantized_base_forward_uses_dequantized_weight():
     assert np.all(err <= np.abs(x).sum(axis=1, keepdims=True) * 0.2 * np.abs(W0).max())
 
 
-def test_lora_grads_equal_linear_bwd():
+@pytest.mark.parametrize("alpha", [3.0, 16.0])
+def test_lora_grads_equal_linear_bwd(alpha):
+    # alpha != r as well, so that the scale s = alpha / r is visible
     x, W, A, B, dh = _problem(M=5, n_in=6, n_out=4, r=3, seed=6)
-    _, dA, dB = linear.linear_bwd(dh, x, W, A, B, 3.0)
-    gA, gB = linear.lora_grads(dh, x, A, B, 3.0)
+    _, dA, dB = linear.linear_bwd(dh, x, W, A, B, alpha)
+    gA, gB = linear.lora_grads(dh, x, A, B, alpha)
     assert np.allclose(gA, dA, rtol=1e-13, atol=1e-14) and np.allclose(gB, dB, rtol=1e-13, atol=1e-14)
 
 

@@ -90,3 +90,39 @@ def test_merged_weight_reproduces_the_layer():
     h_ref, _ = linear.linear_fwd(x, nf4.bf16_to_f64(w), nf4.bf16_to_f64(A), nf4.bf16_to_f64(B), alpha)
     h = x @ Wm.T
     assert np.linalg.norm(h - h_ref) <= 2.0 ** -8 * np.linalg.norm(np.abs(x) @ np.abs(Wm).T)
+
+
+def _bf16_exact_bits(x: float) -> int:
+    """bf16 bit pattern of a value that bf16 represents exactly."""
+    b = int(np.float32(x).view(np.uint32))
+    assert b & 0xFFFF == 0
+    return b >> 16
+
+
+def test_merge_accumulates_in_fp32_in_rank_order():
+    """Reading M1: acc is the in-order fp32 sum of the exact products.  Here
+    the first product is 1 + 2^-3 + 2^-8 (a bf16 tie) and the next two,
+    0.75 * 2^-24 each, are dropped one by one in fp32, so W' rounds the tie
+    to even (0x3F90); the exact sum (1.5 * 2^-24 more) would round up."""
+    B = np.array([[_bf16_exact_bits(1 + 2 ** -4), _bf16_exact_bits(1.5 * 2 ** -12), _bf16_exact_bits(1.5 * 2 ** -12)]], dtype=np.uint16)
+    A = np.array([[_bf16_exact_bits(1 + 2 ** -4)], [_bf16_exact_bits(2 ** -13)], [_bf16_exact_bits(2 ** -13)]], dtype=np.uint16)
+    acc = merge.lora_product_f32(A, B)
+    assert acc[0, 0] == 1 + 2 ** -3 + 2 ** -8
+    w_hat = np.array([[0]], dtype=np.uint16)
+    assert merge.merge_adapter_bits(w_hat, A, B, 3.0)[0, 0] == 0x3F90         # s = fl32(3 / 3) = 1
+    assert nf4.bf16_bits_from_f32(1 + 2 ** -3 + 2 ** -8 + 1.5 * 2 ** -24) == 0x3F91   # the exact sum's bf16
+
+
+def test_merge_rounds_the_scaled_product_before_adding_the_base():
+    """Reading M1: W' = bf16(fl32(w_hat + fl32(s * acc))).  With r = 1,
+    s = 16647415 * 2^-24, acc = 2^-8 (1 + 2^-7): s * acc = 2^-8 + 2^-24 +
+    119 * 2^-39 rounds to 2^-8 + 2^-24 in fp32, so 1 + that is an fp32 tie
+    (to 1 + 2^-8, then a bf16 tie to 1.0); without the inner rounding the sum
+    lies above both ties and W' would be 1 + 2^-7."""
+    alpha = 16647415 * 2.0 ** -24
+    B = np.array([[_bf16_exact_bits(2 ** -4 * (1 + 2 ** -7))]], dtype=np.uint16)
+    A = np.array([[_bf16_exact_bits(2 ** -4)]], dtype=np.uint16)
+    w_hat = np.array([[_bf16_exact_bits(1.0)]], dtype=np.uint16)
+    assert merge.merge_adapter_bits(w_hat, A, B, alpha)[0, 0] == 0x3F80
+    exact = 1 + (16647415 * 2.0 ** -24) * (2 ** -8 * (1 + 2 ** -7))          # exact in fp64 (41 bits)
+    assert nf4.bf16_bits_from_f32(nf4.fl32(exact)) == 0x3F81                   # one rounding only

@@ -4,6 +4,7 @@ round trips, error bounds, zero handling and the storage arithmetic the pages
 print."""
 
 import os
+import struct
 from fractions import Fraction
 
 import numpy as np
@@ -345,3 +346,60 @@ def test_second_level_reciprocal_overflow():
     want = np.clip(np.rint([float(np.float32(float(Fraction(x) / Fraction(st)))) for x in d]), -127, 127)
     assert np.array_equal(q8, want.astype(np.int8))
     assert q8[0] == 127 and q8[1] == -127 and 0 < abs(int(q8[2])) < 127 and q8[4] == 0
+
+
+# ---------------------------------------------------------------- rounding order of readings R3 and R6
+# Independent IEEE binary32 rounding (round to nearest, ties to even; normal
+# range) on exact rationals, to pin which operations the readings round.
+def _round32(q: Fraction) -> Fraction:
+    if q == 0:
+        return Fraction(0)
+    sign, a = (-1 if q < 0 else 1), abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    m = a / ulp
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * n * ulp
+
+
+def _from_bits(h: int) -> Fraction:
+    return Fraction(struct.unpack("<f", struct.pack("<I", h))[0])
+
+
+def _bits(q: Fraction) -> int:
+    return struct.unpack("<I", struct.pack("<f", float(q)))[0]
+
+
+@pytest.mark.parametrize("w_hex,c_hex,code_recip,code_div", [
+    (0xBEE8D8AC, 0x3FF81F9C, 5, 4), (0xBEFF6C6F, 0x3FBBFD1D, 3, 4), (0xBDB60F98, 0x3FF9F248, 7, 6)])
+def test_normalisation_multiplies_by_the_fp32_reciprocal(w_hex, c_hex, code_recip, code_div):
+    """Reading R3: v = fl32(w * fl32(1/c)), not fl32(w / c).  Blocks where the
+    two normalisations fall on different sides of a decision midpoint."""
+    w, c = _from_bits(w_hex), _from_bits(c_hex)
+    levels = [Fraction(float(v)) for v in nf4.codebook()]
+    mids = [(levels[i] + levels[i + 1]) / 2 for i in range(15)]
+    v_recip = _round32(w * _round32(1 / c))
+    v_div = _round32(w / c)
+    assert sum(m < v_recip for m in mids) == code_recip
+    assert sum(m < v_div for m in mids) == code_div
+    W = np.zeros((1, 64), dtype=np.float32)
+    W[0, 0], W[0, 1] = float(c), float(w)               # c is the block's absmax
+    assert nf4.quantize(W)["codes"][0, 1] == code_recip
+
+
+def test_block_scale_rounds_the_product_then_the_sum():
+    """Reading R6: c_hat = fl32(fl32(q8 * step2) + mean), two roundings; a
+    case where one rounding of the exact sum gives the neighbouring float."""
+    q, st, mu = -67, _from_bits(0x3C4DA4F9), _from_bits(0x3E1A6916)
+    twice = _round32(_round32(q * st) + mu)
+    once = _round32(q * st + mu)
+    assert _bits(twice) == 0xBF30AE70 and _bits(once) == 0xBF30AE6F
+    got = nf4.dequant_scales(np.array([q], dtype=np.int8), np.array([float(st)]), float(mu))
+    assert _bits(Fraction(float(got[0]))) == 0xBF30AE70
