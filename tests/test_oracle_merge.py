@@ -126,3 +126,27 @@ def test_merge_rounds_the_scaled_product_before_adding_the_base():
     assert merge.merge_adapter_bits(w_hat, A, B, alpha)[0, 0] == 0x3F80
     exact = 1 + (16647415 * 2.0 ** -24) * (2 ** -8 * (1 + 2 ** -7))          # exact in fp64 (41 bits)
     assert nf4.bf16_bits_from_f32(nf4.fl32(exact)) == 0x3F81                   # one rounding only
+
+
+def test_merge_rounds_the_scale_alpha_over_r_to_fp32():
+    """Reading M1: s = fl32(alpha / r).  With alpha = 11107844 * 2^-22 and
+    r = 3, alpha / 3 = 14810458.67 * 2^-24 rounds up to s = 14810459 * 2^-24.
+    One rank carries acc = 2^-4 * 145 * 2^-11 (the other two are zero), and
+    s * acc = 8388736.54 * 2^-31 rounds to 2^-8 + 2^-24 + 2^-31: above the
+    fp32 tie of 1 + 2^-8 + 2^-24, so W' = bf16(1 + 2^-8 + 2^-23) = 1 + 2^-7.
+    With the quotient left unrounded the product, 8388736.36 * 2^-31, rounds to
+    2^-8 + 2^-24, both ties round to even and W' would be 1.0."""
+    alpha = 11107844 * 2.0 ** -22
+    assert float(np.float32(alpha)) == alpha
+    s = np.float32(alpha) / np.float32(3)                                      # IEEE fp32 division
+    assert float(s) == 14810459 * 2.0 ** -24
+    B = np.array([[_bf16_exact_bits(2 ** -4), 0, 0]], dtype=np.uint16)
+    A = np.array([[_bf16_exact_bits(145 * 2.0 ** -11)], [0], [0]], dtype=np.uint16)
+    w_hat = np.array([[_bf16_exact_bits(1.0)]], dtype=np.uint16)
+    prod = np.float32(float(s) * (145 * 2.0 ** -15))                            # the fp64 product is exact
+    assert float(prod) == 2 ** -8 + 2 ** -24 + 2 ** -31
+    assert int((np.float32(1) + prod).view(np.uint32)) == 0x3F808001           # 1 + 2^-8 + 2^-23
+    assert merge.merge_adapter_bits(w_hat, A, B, alpha)[0, 0] == 0x3F81
+    unrounded = np.float32((alpha / 3) * (145 * 2.0 ** -15))
+    assert float(unrounded) == 2 ** -8 + 2 ** -24
+    assert int((np.float32(1) + unrounded).view(np.uint32)) == 0x3F808000      # tie to even: 1 + 2^-8
