@@ -15,8 +15,8 @@
 // warp-level bf16 MMA); per unit a thread reads, for rows g and g+8, 16
 // consecutive codes of each of the four blocks, and its warp releases the
 // code part of the stage as soon as they are in registers.  Second-level
-// scale codes (four per row and unit) are fetched one unit ahead, group
-// steps are cached.
+// scale codes (four per row and unit) and group steps are fetched two units
+// ahead (one unit ahead, with cached steps, in the 16-token kernel).
 //
 // Each MMA step covers 16 columns of ONE block for all four quad lanes: step
 // s of block j takes columns 64j + 16q + 4s .. +3 for quad lane q, in the
@@ -221,10 +221,33 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   int rs = t_first * kGvRows + warp * 16 + srow;                    // this lane's scale row
   const int8_t* qp = a.q8 + static_cast<int64_t>(rs) * row_blocks + 4 * st_first + 2 * spair;
   const int64_t b_wrap = kGvRows * row_blocks - 4 * static_cast<int64_t>(a.n_st);
-  // paired: the two q8 codes of the next unit (each byte XOR 0x80), cached group step
+  // Paired, 9..16 tokens: the two q8 codes of the next unit (each byte XOR
+  // 0x80) and a cached group step.  Paired, 1..8 tokens: the q8 codes and
+  // group steps of units i + 1 and i + 2, read by a cursor that walks this
+  // lane's (row, block pair) sequence two units ahead, so that no scale
+  // waits on a load issued one unit earlier while the stream holds HBM busy
+  // (the two-token kernel has no registers to spare for it).
+  constexpr bool kAhead = kPaired && !kTwoTok;
   uint32_t qn = 0x8080u;
   float sv = 0.f;
-  if (kPaired && rs < a.out) qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(qp))) ^ 0x8080u;
+  if (kPaired && !kAhead && rs < a.out)
+    qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(qp))) ^ 0x8080u;
+  uint32_t qa = 0x8080u, qb = 0x8080u;
+  float sa = 0.f, sb2 = 0.f;
+  const int8_t* qpf = qp;
+  int rpf = rs, spf = st_first;
+  auto pf_load = [&](uint32_t& qd, float& sd) {
+    if (rpf < a.out) {
+      qd = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(qpf))) ^ 0x8080u;
+      sd = __ldg(a.step2 + (((qpf - a.q8) - 2 * spair) >> 8));
+    }
+    qpf += 4;
+    if (++spf == a.n_st) { spf = 0; rpf += kGvRows; qpf += b_wrap; }
+  };
+  if (kAhead) {
+    pf_load(qa, sa);
+    if (n_local > 1) pf_load(qb, sb2);
+  }
 
   float acc[2][4];
 #pragma unroll
@@ -255,19 +278,30 @@ __global__ void __launch_bounds__(kGvThreads, 1)
       const bool row_ok = rs < a.out;
       float s0, s1;
       if (kPaired) {
-        const uint32_t qc = qn;
-        const int8_t* q_next = last_in_tile ? qp + b_wrap + 4 : qp + 4;
-        const bool next_ok = last_in_tile ? rs + kGvRows < a.out : row_ok;
-        if (next_ok && i + 1 < n_local)
-          qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(q_next))) ^ 0x8080u;
-        // a unit's four blocks share one group; a group starts at a multiple of 256 blocks
-        const int64_t b_unit = (qp - a.q8) - 2 * spair;
-        if (row_ok && (new_row || (static_cast<uint32_t>(b_unit) & 255u) == 0)) sv = __ldg(a.step2 + (b_unit >> 8));
+        uint32_t qc;
+        float svc;
+        if constexpr (kAhead) {
+          qc = qa;
+          svc = sa;
+          qa = qb;
+          sa = sb2;
+          if (i + 2 < n_local) pf_load(qb, sb2);
+        } else {
+          qc = qn;
+          const int8_t* q_next = last_in_tile ? qp + b_wrap + 4 : qp + 4;
+          const bool next_ok = last_in_tile ? rs + kGvRows < a.out : row_ok;
+          if (next_ok && i + 1 < n_local)
+            qn = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(q_next))) ^ 0x8080u;
+          // a unit's four blocks share one group; a group starts at a multiple of 256 blocks
+          const int64_t b_unit = (qp - a.q8) - 2 * spair;
+          if (row_ok && (new_row || (static_cast<uint32_t>(b_unit) & 255u) == 0)) sv = __ldg(a.step2 + (b_unit >> 8));
+          svc = sv;
+        }
         // exact floats of the signed codes: 2^23 + (q + 128) - (2^23 + 128)
         const float q0 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7650u)), -8388736.0f);
         const float q1 = __fadd_rn(__uint_as_float(prmt(qc, 0x4B000000u, 0x7651u)), -8388736.0f);
-        s0 = __fadd_rn(__fmul_rn(q0, sv), mu);
-        s1 = __fadd_rn(__fmul_rn(q1, sv), mu);
+        s0 = __fadd_rn(__fmul_rn(q0, svc), mu);
+        s1 = __fadd_rn(__fmul_rn(q1, svc), mu);
       } else {
         const int c0 = col0 + 128 * spair;
         const bool l0 = row_ok && c0 < a.in, l1 = row_ok && c0 + 64 < a.in;
